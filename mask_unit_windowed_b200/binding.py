@@ -1,0 +1,348 @@
+"""Thin Python binding of libhiera.so (include/hiera.h): argument marshalling only.
+
+Every step of the Hiera block runs inside the library's CUDA kernels. PyTorch supplies
+device memory (outputs, workspaces, packed weights) and the current CUDA stream; the
+calls below pass raw pointers and sizes through ctypes and raise HieraError on any
+non-OK status. If libhiera.so has not been built the import of `lib()` fails loudly:
+there is no fallback implementation.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libhiera.so")
+HEADER = os.path.join(os.path.dirname(_HERE), "include", "hiera.h")
+
+HIERA_F32, HIERA_BF16 = 0, 1
+STATUS = {0: "HIERA_OK", 1: "HIERA_ERR_INVALID_ARG", 2: "HIERA_ERR_SHAPE", 3: "HIERA_ERR_DTYPE",
+          4: "HIERA_ERR_ALIGNMENT", 5: "HIERA_ERR_WORKSPACE", 6: "HIERA_ERR_CUDA",
+          7: "HIERA_ERR_TIMEOUT", 8: "HIERA_ERR_DEVICE"}
+PATCH_PACKED_BYTES = (196 * 112 + 112) * 4
+
+
+class HieraError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {STATUS.get(code, code)}")
+
+
+class BlockDescC(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("tokens", ctypes.c_int), ("dim_in", ctypes.c_int),
+                ("dim_out", ctypes.c_int), ("heads", ctypes.c_int), ("head_dim", ctypes.c_int),
+                ("q_stride", ctypes.c_int), ("window_tokens", ctypes.c_int),
+                ("mask_unit_attn", ctypes.c_int), ("ln_eps", ctypes.c_float),
+                ("dtype", ctypes.c_int)]
+
+
+WEIGHT_NAMES = ("norm1_w", "norm1_b", "qkv_w", "qkv_b", "proj_w", "proj_b", "attn_proj_w",
+                "attn_proj_b", "norm2_w", "norm2_b", "fc1_w", "fc1_b", "fc2_w", "fc2_b")
+
+
+class BlockWeightsC(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in WEIGHT_NAMES]
+
+
+class BackboneDescC(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("img", ctypes.c_int),
+                ("mask_unit_attn_stage2_first", ctypes.c_int), ("dtype", ctypes.c_int)]
+
+
+class BackboneWeightsC(ctypes.Structure):
+    _fields_ = [("patch_w", ctypes.c_void_p), ("patch_b", ctypes.c_void_p),
+                ("pos_embed", ctypes.c_void_p), ("blocks", BlockWeightsC * 24)]
+
+
+_lib = None
+
+
+def header_symbols() -> list:
+    """Names of every entry point declared in include/hiera.h."""
+    with open(HEADER) as f:
+        text = f.read()
+    return re.findall(r"HIERA_API\s+[\w\s\*]+?\b(hiera_\w+)\s*\(", text)
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m mask_unit_windowed_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, S, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+        sig = {
+            "hiera_status_string": ([I], ctypes.c_char_p),
+            "hiera_get_device_status": ([P], I),
+            "hiera_unroll": ([P, P, I, I, I, I, I, P], I),
+            "hiera_reroll": ([P, P, I, I, I, I, I, P], I),
+            "hiera_linear": ([P, P, P, P, P, I, I, I, I, P], I),
+            "hiera_block_packed_bytes": ([ctypes.POINTER(BlockDescC)], S),
+            "hiera_block_pack": ([ctypes.POINTER(BlockDescC), ctypes.POINTER(BlockWeightsC), P, S,
+                                  P], I),
+            "hiera_block_workspace_bytes": ([ctypes.POINTER(BlockDescC)], S),
+            "hiera_block_forward": ([ctypes.POINTER(BlockDescC), P, P, P, P, S, P], I),
+            "hiera_block_workspace_layout": ([ctypes.POINTER(BlockDescC),
+                                              ctypes.POINTER(ctypes.c_longlong)], I),
+            "hiera_patch_pack": ([P, P, P, I, P], I),
+            "hiera_patch_embed": ([P, P, P, P, I, I, I, P], I),
+            "hiera_backbone_packed_bytes": ([ctypes.POINTER(BackboneDescC)], S),
+            "hiera_backbone_pack": ([ctypes.POINTER(BackboneDescC),
+                                     ctypes.POINTER(BackboneWeightsC), P, S, P], I),
+            "hiera_backbone_workspace_bytes": ([ctypes.POINTER(BackboneDescC)], S),
+            "hiera_backbone_forward": ([ctypes.POINTER(BackboneDescC), P, P,
+                                        ctypes.POINTER(ctypes.c_void_p), P, S, P], I),
+            "hiera_debug_timeout_probe": ([I, P], I),
+        }
+        for name, (args, res) in sig.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        del F
+        _lib = L
+    return _lib
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        raise HieraError(code, where)
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return HIERA_BF16
+    if t.dtype == torch.float32:
+        return HIERA_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str):
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+
+
+# ----------------------------------------------------------------------------- Unroll / Reroll
+def unroll(x: torch.Tensor, G: int, levels: int, out=None, stream=None) -> torch.Tensor:
+    _need(x, "x")
+    B, N, C = x.shape
+    out = torch.empty_like(x) if out is None else out
+    _check(lib().hiera_unroll(_ptr(x), _ptr(out), B, G, C, levels, _dt(x), _stream(stream)),
+           "hiera_unroll")
+    return out
+
+
+def reroll(x: torch.Tensor, G: int, levels: int, out=None, stream=None) -> torch.Tensor:
+    _need(x, "x")
+    B, N, C = x.shape
+    out = torch.empty((B, G, G, C), dtype=x.dtype, device=x.device) if out is None else out
+    _check(lib().hiera_reroll(_ptr(x), _ptr(out), B, G, C, levels, _dt(x), _stream(stream)),
+           "hiera_reroll")
+    return out
+
+
+def linear(x, w, bias=None, residual=None, out=None, stream=None) -> torch.Tensor:
+    _need(x, "x")
+    M, K = x.shape
+    N = w.shape[0]
+    out = torch.empty((M, N), dtype=x.dtype, device=x.device) if out is None else out
+    _check(lib().hiera_linear(_ptr(x), _ptr(w), _ptr(bias), _ptr(residual), _ptr(out), M, N, K,
+                              _dt(x), _stream(stream)), "hiera_linear")
+    return out
+
+
+# ----------------------------------------------------------------------------- block
+@dataclass
+class BlockDesc:
+    B: int
+    tokens: int
+    dim_in: int
+    dim_out: int
+    heads: int
+    q_stride: int = 1
+    window_tokens: int = 64
+    mask_unit_attn: bool = True
+    dtype: torch.dtype = torch.bfloat16
+    head_dim: int = 56
+    ln_eps: float = 1e-6
+
+    def c(self) -> BlockDescC:
+        return BlockDescC(self.B, self.tokens, self.dim_in, self.dim_out, self.heads,
+                          self.head_dim, self.q_stride, self.window_tokens,
+                          int(bool(self.mask_unit_attn)), self.ln_eps,
+                          HIERA_BF16 if self.dtype == torch.bfloat16 else HIERA_F32)
+
+    @property
+    def out_tokens(self) -> int:
+        return self.tokens // self.q_stride
+
+
+def _weights_c(w: dict) -> BlockWeightsC:
+    wc = BlockWeightsC()
+    for n in WEIGHT_NAMES:
+        t = w.get(n)
+        if t is not None:
+            _need(t, n)
+        setattr(wc, n, None if t is None else t.data_ptr())
+    return wc
+
+
+def block_packed_bytes(desc: BlockDesc) -> int:
+    d = desc.c()
+    n = lib().hiera_block_packed_bytes(ctypes.byref(d))
+    if n == 0:
+        raise HieraError(2, "hiera_block_packed_bytes")
+    return n
+
+
+def block_workspace_bytes(desc: BlockDesc) -> int:
+    d = desc.c()
+    n = lib().hiera_block_workspace_bytes(ctypes.byref(d))
+    if n == 0:
+        raise HieraError(2, "hiera_block_workspace_bytes")
+    return n
+
+
+def block_workspace_layout(desc: BlockDesc) -> list:
+    d = desc.c()
+    offs = (ctypes.c_longlong * 7)()
+    _check(lib().hiera_block_workspace_layout(ctypes.byref(d), offs),
+           "hiera_block_workspace_layout")
+    return list(offs)
+
+
+def block_pack(desc: BlockDesc, weights: dict, device="cuda", stream=None) -> torch.Tensor:
+    d = desc.c()
+    nbytes = block_packed_bytes(desc)
+    packed = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    wc = _weights_c(weights)
+    _check(lib().hiera_block_pack(ctypes.byref(d), ctypes.byref(wc), _ptr(packed), nbytes,
+                                  _stream(stream)), "hiera_block_pack")
+    return packed
+
+
+def block_forward(desc: BlockDesc, packed: torch.Tensor, x: torch.Tensor, out=None,
+                  workspace=None, stream=None) -> torch.Tensor:
+    _need(x, "x")
+    d = desc.c()
+    if out is None:
+        out = torch.empty((desc.B, desc.out_tokens, desc.dim_out), dtype=x.dtype,
+                          device=x.device)
+    if workspace is None:
+        workspace = torch.empty(block_workspace_bytes(desc), dtype=torch.uint8, device=x.device)
+    _check(lib().hiera_block_forward(ctypes.byref(d), _ptr(packed), _ptr(x), _ptr(out),
+                                     _ptr(workspace), workspace.numel(), _stream(stream)),
+           "hiera_block_forward")
+    return out
+
+
+# ----------------------------------------------------------------------------- patch embed
+def patch_pack(patch_w, patch_b=None, stream=None) -> torch.Tensor:
+    _need(patch_w, "patch_w")
+    packed = torch.empty(PATCH_PACKED_BYTES, dtype=torch.uint8, device=patch_w.device)
+    _check(lib().hiera_patch_pack(_ptr(patch_w), _ptr(patch_b), _ptr(packed), _dt(patch_w),
+                                  _stream(stream)), "hiera_patch_pack")
+    return packed
+
+
+def patch_embed(img, packed_patch, pos_embed, out=None, stream=None) -> torch.Tensor:
+    _need(img, "img")
+    B, H, W, _ = img.shape
+    G = H // 4
+    out = torch.empty((B, G * G, 112), dtype=img.dtype, device=img.device) if out is None else out
+    _check(lib().hiera_patch_embed(_ptr(img), _ptr(packed_patch), _ptr(pos_embed), _ptr(out), B,
+                                   H, _dt(img), _stream(stream)), "hiera_patch_embed")
+    return out
+
+
+# ----------------------------------------------------------------------------- backbone
+@dataclass
+class BackboneDesc:
+    B: int
+    img: int
+    dtype: torch.dtype = torch.bfloat16
+    mask_unit_attn_stage2_first: bool = False
+
+    def c(self) -> BackboneDescC:
+        return BackboneDescC(self.B, self.img, int(bool(self.mask_unit_attn_stage2_first)),
+                             HIERA_BF16 if self.dtype == torch.bfloat16 else HIERA_F32)
+
+    def feature_shapes(self):
+        dims = (112, 224, 448, 896)
+        return [(self.B, self.img >> (s + 2), self.img >> (s + 2), dims[s]) for s in range(4)]
+
+
+def backbone_packed_bytes(desc: BackboneDesc) -> int:
+    d = desc.c()
+    n = lib().hiera_backbone_packed_bytes(ctypes.byref(d))
+    if n == 0:
+        raise HieraError(2, "hiera_backbone_packed_bytes")
+    return n
+
+
+def backbone_workspace_bytes(desc: BackboneDesc) -> int:
+    d = desc.c()
+    n = lib().hiera_backbone_workspace_bytes(ctypes.byref(d))
+    if n == 0:
+        raise HieraError(2, "hiera_backbone_workspace_bytes")
+    return n
+
+
+def backbone_pack(desc: BackboneDesc, weights: dict, device="cuda", stream=None) -> torch.Tensor:
+    d = desc.c()
+    wc = BackboneWeightsC()
+    wc.patch_w = weights["patch_w"].data_ptr()
+    wc.patch_b = None if weights.get("patch_b") is None else weights["patch_b"].data_ptr()
+    wc.pos_embed = weights["pos_embed"].data_ptr()
+    for i, bw in enumerate(weights["blocks"]):
+        wc.blocks[i] = _weights_c(bw)
+    nbytes = backbone_packed_bytes(desc)
+    packed = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    _check(lib().hiera_backbone_pack(ctypes.byref(d), ctypes.byref(wc), _ptr(packed), nbytes,
+                                     _stream(stream)), "hiera_backbone_pack")
+    return packed
+
+
+def backbone_forward(desc: BackboneDesc, packed, img, feats=None, workspace=None,
+                     stream=None):
+    _need(img, "img")
+    d = desc.c()
+    if feats is None:
+        feats = [torch.empty(s, dtype=img.dtype, device=img.device)
+                 for s in desc.feature_shapes()]
+    if workspace is None:
+        workspace = torch.empty(backbone_workspace_bytes(desc), dtype=torch.uint8,
+                                device=img.device)
+    fp = (ctypes.c_void_p * 4)(*[f.data_ptr() for f in feats])
+    _check(lib().hiera_backbone_forward(ctypes.byref(d), _ptr(packed), _ptr(img), fp,
+                                        _ptr(workspace), workspace.numel(), _stream(stream)),
+           "hiera_backbone_forward")
+    return feats
+
+
+# ----------------------------------------------------------------------------- status
+def device_status(stream=None) -> int:
+    """Synchronise and return (then clear) the first device-side error code."""
+    return lib().hiera_get_device_status(_stream(stream))
+
+
+def timeout_probe(limit_us: int, stream=None):
+    _check(lib().hiera_debug_timeout_probe(limit_us, _stream(stream)), "hiera_debug_timeout_probe")
+
+
+def status_string(code: int) -> str:
+    return lib().hiera_status_string(code).decode()

@@ -1,0 +1,588 @@
+// Persistent, warp-specialised tcgen05 GEMM for the Hiera block's Linear layers
+// ("Phase 4: Hiera Backbone MLX Port", Architecture Summary: qkv = Linear(dim_in,
+// 3 dim_out), proj = Linear(dim_out, dim_out), MLP fc1 -> GELU -> fc2, and the
+// transition's proj Linear + max-pool).
+//
+//   C[M, N] = A[M, K] * W[N, K]^T      bf16 operands, fp32 accumulation in TMEM
+//
+// Roles (one CTA per SM, tiles strided over the grid):
+//   warp 0      TMA producer: A tile 128 x 64 and W tile BN x 64 per stage, 128-byte
+//               swizzle, STAGES-deep ring guarded by full/empty mbarriers.
+//   warp 1      owns TMEM (2 accumulators of BN fp32 columns) and issues tcgen05.mma
+//               (M = 128, N = BN, K = 16 per instruction) from one thread.
+//   warps 2-5   epilogue: tcgen05.ld of the accumulator (TMEM lane = tile row), the
+//               LayerNorm fold / bias / GELU / residual, and the store or the scatter
+//               into head-major q/k/v with the q_stride max-pool.
+//   warps 6-9   (LayerNorm-fold GEMMs only) row statistics of A read from the same
+//               shared-memory stages as they stream past: per-64-column mean and M2,
+//               merged with Chan's parallel update, so LayerNorm costs no extra pass.
+//
+// LayerNorm fold: with W' = W diag(gamma) (packed once), s_n = sum_k W'_nk and
+// c_n = sum_k beta_k W_nk + b_n,  LN(x) W^T + b = rstd * (x W'^T - mean * s) + c.
+// Transition pooling: a 4-D tensor map loads, for 32 pooled tokens n, the four rows
+// n + c*T/4 (c = 0..3) interleaved, so the four pooling candidates are adjacent TMEM
+// lanes and the max is two warp shuffles.
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace hiera {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int STAGES = 4;
+
+struct KParams {
+  int M, N, K;
+  const float* colsum;
+  const float* colconst;
+  const bf16* bias16;
+  float ln_eps;
+  bf16* out;
+  const bf16* residual;
+  int ldo;
+  bf16* q;
+  bf16* k;
+  bf16* v;
+  bf16* r;
+  int tokens, nW, heads, d_out, Tq, Tkv;
+  uint64_t limit_ns;
+  unsigned int* status;
+};
+
+template <int BN>
+struct Cfg {
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int ACC_STRIDE = BN <= 128 ? 128 : 256;
+  static constexpr int TMEM_COLS = 2 * ACC_STRIDE;
+  static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
+  static constexpr int STATS_OFF = BAR_OFF + 256;
+  static constexpr int SMEM_BYTES = STATS_OFF + 2 * 128 * 8 + 1024;
+  static_assert(B_BYTES % 1024 == 0, "W tile must keep 1024-byte alignment");
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128");
+};
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint64_t limit,
+                                          unsigned int* status, volatile int* abort_flag) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) {
+    ok = mbar_wait(bar, parity, limit, status, abort_flag) ? 1 : 0;
+    if (!ok) *abort_flag = 1;
+  }
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  __syncwarp();  // order lane 0's acquire before the other lanes' reads
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint4 add_bf16x8(uint4 a, uint4 b) {
+  uint4 o;
+  o.x = pack_bf16x2(bf16_lo(a.x) + bf16_lo(b.x), bf16_hi(a.x) + bf16_hi(b.x));
+  o.y = pack_bf16x2(bf16_lo(a.y) + bf16_lo(b.y), bf16_hi(a.y) + bf16_hi(b.y));
+  o.z = pack_bf16x2(bf16_lo(a.z) + bf16_lo(b.z), bf16_hi(a.z) + bf16_hi(b.z));
+  o.w = pack_bf16x2(bf16_lo(a.w) + bf16_lo(b.w), bf16_hi(a.w) + bf16_hi(b.w));
+  return o;
+}
+
+// Epilogue of one 128 x BN tile for one thread (= one TMEM lane = one tile row).
+template <int BN, int EPI, bool FOLD, bool POOLED>
+__device__ __forceinline__ void epilogue_tile(const KParams& p, uint32_t tbase, int mt, int nt,
+                                              int rt, float mean, float rstd) {
+  const int n0 = nt * BN;
+  long long m;
+  int b = 0, tok = 0, np = 0;
+  if (POOLED) {
+    const int per = p.tokens >> 2;
+    const int pm = mt * 32 + (rt >> 2);
+    b = pm / per;
+    np = pm - b * per;
+    tok = (rt & 3) * per + np;
+    m = (long long)b * p.tokens + tok;
+  } else {
+    m = (long long)mt * BM + rt;
+    if (EPI == EPI_QKV) {
+      b = (int)(m / p.tokens);
+      tok = (int)(m - (long long)b * p.tokens);
+    }
+  }
+  const bool row_ok = m < p.M;
+  const int which = (EPI == EPI_QKV) ? n0 / p.d_out : 0;
+  const bool pool_this = POOLED && (which == 0 || which == 3);
+  const bool writer = row_ok && (!pool_this || (rt & 3) == 0);
+  const int colw0 = (EPI == EPI_QKV) ? n0 - which * p.d_out : 0;
+
+#pragma unroll 1
+  for (int c0 = 0; c0 < BN; c0 += 16) {
+    uint32_t r[16];
+    tc_ld_32x32b_x16(tbase + (uint32_t)c0, r);
+    tc_wait_ld();
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int n = n0 + c0 + i;
+      const float acc = __uint_as_float(r[i]);
+      const float cc = p.colconst != nullptr ? __ldg(p.colconst + n)
+                       : (p.bias16 != nullptr ? __bfloat162float(p.bias16[n]) : 0.f);
+      float x;
+      if (FOLD) {
+        x = rstd * (acc - mean * __ldg(p.colsum + n)) + cc;
+      } else {
+        x = acc + cc;
+      }
+      if (EPI == EPI_GELU) x = gelu_erf(x);
+      v[i] = x;
+    }
+    if (EPI == EPI_QKV) {
+      if (pool_this) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          v[i] = fmaxf(v[i], __shfl_xor_sync(0xffffffffu, v[i], 1));
+          v[i] = fmaxf(v[i], __shfl_xor_sync(0xffffffffu, v[i], 2));
+        }
+      }
+#pragma unroll
+      for (int g = 0; g < 2; ++g) {
+        const int colw = colw0 + c0 + 8 * g;
+        uint4 pk;
+        pk.x = pack_bf16x2(v[8 * g + 0], v[8 * g + 1]);
+        pk.y = pack_bf16x2(v[8 * g + 2], v[8 * g + 3]);
+        pk.z = pack_bf16x2(v[8 * g + 4], v[8 * g + 5]);
+        pk.w = pack_bf16x2(v[8 * g + 6], v[8 * g + 7]);
+        if (!writer) continue;
+        bf16* dst;
+        if (which == 3) {
+          const int nq = POOLED ? (p.tokens >> 2) : p.tokens;
+          const int tq = POOLED ? np : tok;
+          dst = p.r + ((long long)b * nq + tq) * p.d_out + colw;
+        } else {
+          const int h = colw / 56, e = colw - h * 56;
+          const int tt = pool_this ? np : tok;
+          const int w = tt % p.nW, j = tt / p.nW;
+          const int T = which == 0 ? p.Tq : p.Tkv;
+          bf16* base = which == 0 ? p.q : (which == 1 ? p.k : p.v);
+          dst = base + ((((long long)b * p.nW + w) * p.heads + h) * T + j) * 64 + e;
+        }
+        *reinterpret_cast<uint4*>(dst) = pk;
+      }
+    } else {
+#pragma unroll
+      for (int g = 0; g < 2; ++g) {
+        uint4 pk;
+        pk.x = pack_bf16x2(v[8 * g + 0], v[8 * g + 1]);
+        pk.y = pack_bf16x2(v[8 * g + 2], v[8 * g + 3]);
+        pk.z = pack_bf16x2(v[8 * g + 4], v[8 * g + 5]);
+        pk.w = pack_bf16x2(v[8 * g + 6], v[8 * g + 7]);
+        if (!row_ok) continue;
+        const long long off = m * p.ldo + n0 + c0 + 8 * g;
+        if (p.residual != nullptr) {
+          // residual added in fp32 before the single rounding to bf16
+          const uint4 rr = __ldg(reinterpret_cast<const uint4*>(p.residual + off));
+          pk.x = pack_bf16x2(v[8 * g + 0] + bf16_lo(rr.x), v[8 * g + 1] + bf16_hi(rr.x));
+          pk.y = pack_bf16x2(v[8 * g + 2] + bf16_lo(rr.y), v[8 * g + 3] + bf16_hi(rr.y));
+          pk.z = pack_bf16x2(v[8 * g + 4] + bf16_lo(rr.z), v[8 * g + 5] + bf16_hi(rr.z));
+          pk.w = pack_bf16x2(v[8 * g + 6] + bf16_lo(rr.w), v[8 * g + 7] + bf16_hi(rr.w));
+        }
+        *reinterpret_cast<uint4*>(p.out + off) = pk;
+      }
+    }
+  }
+  // channels 56..63 of every q/k/v head row written above are zero padding
+  if (EPI == EPI_QKV && which != 3 && writer) {
+    const int tt = pool_this ? np : tok;
+    const int w = tt % p.nW, j = tt / p.nW;
+    const int T = which == 0 ? p.Tq : p.Tkv;
+    bf16* base = which == 0 ? p.q : (which == 1 ? p.k : p.v);
+    for (int h = colw0 / 56; h < (colw0 + BN) / 56; ++h) {
+      bf16* dst = base + ((((long long)b * p.nW + w) * p.heads + h) * T + j) * 64 + 56;
+      *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+}
+
+template <int BN, int EPI, bool FOLD, bool POOLED>
+__global__ void __launch_bounds__(FOLD ? 320 : 192, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const KParams p) {
+  using C = Cfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  uint8_t* smem = smem_raw + pad;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* acc_full = bars + 2 * STAGES;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* st_full = acc_empty + 2;
+  uint64_t* st_empty = st_full + 2;
+  uint64_t* drain = st_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float2* stats = reinterpret_cast<float2*>(smem + C::STATS_OFF);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m_tiles = POOLED ? ((p.M >> 2) + 31) / 32 : (p.M + BM - 1) / BM;
+  const int n_tiles = p.N / BN;
+  const int num_tiles = m_tiles * n_tiles;
+  const int kblocks = (p.K + BK - 1) / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1 + (FOLD ? 128 : 0));
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 128);
+      mbar_init(&st_full[a], 128);
+      mbar_init(&st_empty[a], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tc_alloc(tmem_slot, C::TMEM_COLS);
+    tc_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      long long issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int mt = tile / n_tiles, nt = tile - (tile / n_tiles) * n_tiles;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&empty[s], ph ^ 1u, p.limit_ns, p.status, abort_flag)) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + s * C::STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
+          if (POOLED) {
+            const int per = p.tokens >> 2;
+            if (per >= 32) {
+              const int pm0 = mt * 32;
+              tma_load_4d(sa, &tmA, &full[s], kb * BK, 0, pm0 % per, pm0 / per);
+            } else {
+              // 32 / per whole images per tile, one box of per x 4 rows each
+              for (int i = 0; i < 32 / per; ++i)
+                tma_load_4d(sa + i * per * 512, &tmA, &full[s], kb * BK, 0, 0,
+                            mt * (32 / per) + i);
+            }
+          } else {
+            tma_load_2d(sa, &tmA, &full[s], kb * BK, mt * BM);
+          }
+          tma_load_2d(sa + C::A_BYTES, &tmB, &full[s], kb * BK, nt * BN);
+          ++issued;
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // let copies already in flight land before the CTA's shared memory goes away
+        for (long long i = issued > STAGES ? issued - STAGES : 0; i < issued; ++i)
+          mbar_wait(&full[i % STAGES], (uint32_t)((i / STAGES) & 1), p.limit_ns, p.status);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
+      int s = 0, acc = 0;
+      uint32_t ph = 0, aph = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        if (!mbar_wait(&acc_empty[acc], aph ^ 1u, p.limit_ns, p.status, abort_flag)) {
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(acc * C::ACC_STRIDE);
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&full[s], ph, p.limit_ns, p.status, abort_flag)) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
+          const uint64_t adesc = smem_desc_sw128(sa);
+          const uint64_t bdesc = smem_desc_sw128(sa + C::A_BYTES);
+#pragma unroll
+          for (int j = 0; j < BK / 16; ++j) {
+            if (kb * BK + j * 16 < p.K)
+              tc_mma_bf16(d, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(2 * j), IDESC,
+                          (kb | j) != 0 ? 1u : 0u);
+          }
+          tc_commit(&empty[s]);
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&acc_full[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          aph ^= 1u;
+        }
+      }
+      // no MMA may still be writing TMEM when it is released
+      tc_commit(drain);
+      mbar_wait(drain, 0, p.limit_ns, p.status);
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;
+    const int rt = quarter * 32 + lane;
+    int acc = 0;
+    uint32_t aph = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      const int mt = tile / n_tiles, nt = tile - (tile / n_tiles) * n_tiles;
+      if (!warp_wait(&acc_full[acc], aph, p.limit_ns, p.status, abort_flag)) break;
+      float mean = 0.f, rstd = 1.f;
+      if (FOLD) {
+        if (!warp_wait(&st_full[acc], aph, p.limit_ns, p.status, abort_flag)) break;
+        const float2 st = stats[acc * 128 + rt];
+        mean = st.x;
+        rstd = st.y;
+        mbar_arrive(&st_empty[acc]);
+      }
+      tc_fence_after();
+      const uint32_t tbase = tmem + (uint32_t)(acc * C::ACC_STRIDE) + ((uint32_t)(quarter * 32) << 16);
+      epilogue_tile<BN, EPI, FOLD, POOLED>(p, tbase, mt, nt, rt, mean, rstd);
+      tc_fence_before();
+      mbar_arrive(&acc_empty[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        aph ^= 1u;
+      }
+    }
+  } else if (FOLD) {
+    // ------------------------------------------------------------ LayerNorm row statistics
+    const int t = (warp - 6) * 32 + lane;
+    int s = 0, acc = 0;
+    uint32_t ph = 0, aph = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      if (!warp_wait(&st_empty[acc], aph ^ 1u, p.limit_ns, p.status, abort_flag)) break;
+      float mean = 0.f, m2 = 0.f;
+      int cnt = 0;
+      for (int kb = 0; kb < kblocks; ++kb) {
+        if (!warp_wait(&full[s], ph, p.limit_ns, p.status, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const uint4* row = reinterpret_cast<const uint4*>(smem + s * C::STAGE_BYTES + t * 128);
+        uint4 ch[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) ch[c] = row[c];
+        mbar_arrive(&empty[s]);
+        const int kvalid = min(BK, p.K - kb * BK);
+        // physical 16-byte chunk c of this 128-byte row holds logical chunk c ^ (row & 7)
+        float sum = 0.f;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const int k0 = ((c ^ (t & 7)) << 3);
+          const uint32_t wv[4] = {ch[c].x, ch[c].y, ch[c].z, ch[c].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            if (k0 + 2 * e < kvalid) sum += bf16_lo(wv[e]);
+            if (k0 + 2 * e + 1 < kvalid) sum += bf16_hi(wv[e]);
+          }
+        }
+        const float bmean = sum / (float)kvalid;
+        float bm2 = 0.f;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const int k0 = ((c ^ (t & 7)) << 3);
+          const uint32_t wv[4] = {ch[c].x, ch[c].y, ch[c].z, ch[c].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float d0 = bf16_lo(wv[e]) - bmean, d1 = bf16_hi(wv[e]) - bmean;
+            if (k0 + 2 * e < kvalid) bm2 += d0 * d0;
+            if (k0 + 2 * e + 1 < kvalid) bm2 += d1 * d1;
+          }
+        }
+        // Chan et al. pairwise update of (count, mean, M2)
+        const int tot = cnt + kvalid;
+        const float delta = bmean - mean;
+        mean += delta * ((float)kvalid / (float)tot);
+        m2 += bm2 + delta * delta * ((float)cnt * (float)kvalid / (float)tot);
+        cnt = tot;
+        if (++s == STAGES) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+      if (!ok) break;
+      stats[acc * 128 + t] = make_float2(mean, rsqrtf(m2 / (float)p.K + p.ln_eps));
+      mbar_arrive(&st_full[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        aph ^= 1u;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tc_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+bool encode_bf16(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
+                 const cuuint64_t* strides_bytes, const cuuint32_t* box) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (fn == nullptr) return false;
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base),
+                  dims, strides_bytes, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN, int EPI, bool FOLD, bool POOLED>
+hiera_status run(const TcGemmArgs& a, cudaStream_t stream) {
+  using C = Cfg<BN>;
+  CUtensorMap tmA, tmB;
+  if (POOLED) {
+    const int per = a.tokens / 4;
+    const int B = a.M / a.tokens;
+    cuuint64_t dims[4] = {(cuuint64_t)a.K, 4, (cuuint64_t)per, (cuuint64_t)B};
+    cuuint64_t str[3] = {(cuuint64_t)per * a.K * 2, (cuuint64_t)a.K * 2,
+                         (cuuint64_t)a.tokens * a.K * 2};
+    cuuint32_t box[4] = {BK, 4, (cuuint32_t)(per < 32 ? per : 32), 1};
+    if (!encode_bf16(&tmA, a.A, 4, dims, str, box)) return HIERA_ERR_CUDA;
+  } else {
+    cuuint64_t dims[2] = {(cuuint64_t)a.K, (cuuint64_t)a.M};
+    cuuint64_t str[1] = {(cuuint64_t)a.K * 2};
+    cuuint32_t box[2] = {BK, BM};
+    if (!encode_bf16(&tmA, a.A, 2, dims, str, box)) return HIERA_ERR_CUDA;
+  }
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)a.K, (cuuint64_t)a.N};
+    cuuint64_t str[1] = {(cuuint64_t)a.K * 2};
+    cuuint32_t box[2] = {BK, BN};
+    if (!encode_bf16(&tmB, a.W, 2, dims, str, box)) return HIERA_ERR_CUDA;
+  }
+  KParams p;
+  p.M = a.M;
+  p.N = a.N;
+  p.K = a.K;
+  p.colsum = a.colsum;
+  p.colconst = a.colconst;
+  p.bias16 = static_cast<const bf16*>(a.bias_bf16);
+  p.ln_eps = a.ln_eps;
+  p.out = static_cast<bf16*>(a.out);
+  p.residual = static_cast<const bf16*>(a.residual);
+  p.ldo = a.ldo;
+  p.q = static_cast<bf16*>(a.q);
+  p.k = static_cast<bf16*>(a.k);
+  p.v = static_cast<bf16*>(a.v);
+  p.r = static_cast<bf16*>(a.r);
+  p.tokens = a.tokens;
+  p.nW = a.nW;
+  p.heads = a.heads;
+  p.d_out = a.d_out;
+  p.Tq = a.Tq;
+  p.Tkv = a.Tkv;
+  p.limit_ns = g_wait_limit_ns();
+  p.status = g_status_ptr();
+
+  auto kern = tc_gemm_kernel<BN, EPI, FOLD, POOLED>;
+  static bool attr_done[64] = {false};  // per device
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_done[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+        cudaSuccess)
+      return HIERA_ERR_CUDA;
+    attr_done[dev] = true;
+  }
+  const int m_tiles = POOLED ? (a.M / 4 + 31) / 32 : (a.M + BM - 1) / BM;
+  const int tiles = m_tiles * (a.N / BN);
+  if (tiles == 0) return HIERA_OK;
+  int grid = g_num_sms();
+  if (grid > tiles) grid = tiles;
+  kern<<<grid, FOLD ? 320 : 192, C::SMEM_BYTES, stream>>>(tmA, tmB, p);
+  return cudaGetLastError() == cudaSuccess ? HIERA_OK : HIERA_ERR_CUDA;
+}
+
+}  // namespace
+
+hiera_status launch_tc_gemm(int epi, const TcGemmArgs& a, cudaStream_t stream) {
+  if (a.M <= 0 || a.N <= 0 || a.K <= 0) return HIERA_OK;
+  if (a.N % 16 != 0 || a.K % 8 != 0) return HIERA_ERR_SHAPE;
+  if (epi == EPI_QKV) {
+    if (!a.ln_fold) return HIERA_ERR_INVALID_ARG;
+    const bool pooled = a.pooled != 0;
+    if (pooled) {
+      // tiles of 32 pooled tokens: whole 32-row slices of one image, or whole images
+      const int per = a.tokens / 4;
+      if (a.tokens % 4 != 0 || per < 2 || (per >= 32 ? per % 32 != 0 : 32 % per != 0))
+        return HIERA_ERR_SHAPE;
+    }
+    if (a.d_out % 224 == 0)
+      return pooled ? run<224, EPI_QKV, true, true>(a, stream)
+                    : run<224, EPI_QKV, true, false>(a, stream);
+    if (a.d_out % 112 == 0)
+      return pooled ? run<112, EPI_QKV, true, true>(a, stream)
+                    : run<112, EPI_QKV, true, false>(a, stream);
+    return HIERA_ERR_SHAPE;
+  }
+  if (epi == EPI_GELU) {
+    if (!a.ln_fold) return HIERA_ERR_INVALID_ARG;
+    if (a.N % 224 == 0) return run<224, EPI_GELU, true, false>(a, stream);
+    if (a.N % 112 == 0) return run<112, EPI_GELU, true, false>(a, stream);
+    return HIERA_ERR_SHAPE;
+  }
+  if (a.ln_fold) return HIERA_ERR_INVALID_ARG;
+  if (a.N % 224 == 0) return run<224, EPI_STORE, false, false>(a, stream);
+  if (a.N % 128 == 0) return run<128, EPI_STORE, false, false>(a, stream);
+  if (a.N % 112 == 0) return run<112, EPI_STORE, false, false>(a, stream);
+  if (a.N % 64 == 0) return run<64, EPI_STORE, false, false>(a, stream);
+  if (a.N % 32 == 0) return run<32, EPI_STORE, false, false>(a, stream);
+  return run<16, EPI_STORE, false, false>(a, stream);
+}
+
+}  // namespace hiera

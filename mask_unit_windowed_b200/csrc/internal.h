@@ -1,0 +1,95 @@
+// Internal (non-ABI) declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "hiera.h"
+
+namespace hiera {
+
+int g_num_sms();                         // SM count of the current device (cached per device)
+uint64_t g_wait_limit_ns();              // bound on every device-side wait
+unsigned int* g_status_ptr();            // device address of the status word (current device)
+
+cudaError_t launch_permute(bool unroll, const void* x, void* y, int B, int G, int C, int L,
+                           int elem_bytes, cudaStream_t stream);
+
+// ---------------------------------------------------------------- tcgen05 GEMM (bf16)
+enum EpiKind { EPI_STORE = 0, EPI_GELU = 1, EPI_QKV = 2 };
+
+struct TcGemmArgs {
+  int M, N, K;            // C[M, N] = A[M, K] * W[N, K]^T  (M = rows of A)
+  const void* A;          // bf16 [M, K]
+  const void* W;          // bf16 [N, K]
+  // epilogue: v = ln_fold ? rstd*(acc - mean*colsum[n]) + colconst[n] : acc + colconst[n]
+  const float* colsum;    // [N] (ln_fold only)
+  const float* colconst;  // [N] or nullptr
+  const void* bias_bf16;  // [N] bf16 bias used when colconst is nullptr (may be nullptr)
+  float ln_eps;
+  int ln_fold;            // 1: LayerNorm of A's rows folded into the epilogue
+  // EPI_STORE / EPI_GELU: out[m * ldo + n] (+ residual[m * ldo + n])
+  void* out;
+  const void* residual;
+  int ldo;
+  // EPI_QKV: scatter into head-major q/k/v [B][nW][heads][T][64] (+ pooled residual r)
+  void* q;
+  void* k;
+  void* v;
+  void* r;                // transition residual [B, tokens/4, d_out] (columns 3*d_out..)
+  int tokens, nW, heads, d_out, Tq, Tkv;
+  int pooled;             // 1: rows n, n+T/4, n+T/2, n+3T/4 of each image loaded together and
+                          //    q / r columns max-pooled over them (q_stride 4)
+};
+
+hiera_status launch_tc_gemm(int epi, const TcGemmArgs& a, cudaStream_t stream);
+
+// ---------------------------------------------------------------- attention (bf16, mma.sync)
+struct AttnArgs {
+  const void* q;  // [B][nW][heads][Tq][64]
+  const void* k;  // [B][nW][heads][Tkv][64]
+  const void* v;
+  void* o;        // [B][Tq*nW][d_out], token j*nW + w, channel h*56 + e
+  int B, nW, heads, Tq, Tkv, d_out;
+};
+hiera_status launch_attention_bf16(const AttnArgs& a, cudaStream_t stream);
+
+// ---------------------------------------------------------------- fp32 SIMT path
+hiera_status launch_row_stats_f32(const float* x, int M, int K, float eps, float2* stats,
+                                  cudaStream_t stream);
+struct F32GemmArgs {
+  int M, N, K;
+  const float* A; int lda;
+  const float* W;              // [N, K]
+  const float2* stats;         // per-row (mean, rstd) for the LayerNorm fold, or nullptr
+  const float* colsum;         // [N] (fold only)
+  const float* colconst;       // [N] or nullptr
+  int gelu;
+  const float* residual; int ldr;
+  int resid_pool_tokens;       // >0: residual row m = max over 4 chunk rows of an image
+                               //     with this many (un-pooled) tokens
+  float* out; int ldo;
+};
+hiera_status launch_gemm_f32(const F32GemmArgs& a, cudaStream_t stream);
+struct F32AttnArgs {
+  const float* T; int ldT;     // token-major [B, tokens, ldT]; q/k/v at channel offsets
+  int q_off, k_off, v_off;
+  float* o;                    // [B, tokens/q_stride, d_out]
+  int B, tokens, nW, heads, q_stride, d_out;
+};
+hiera_status launch_attention_f32(const F32AttnArgs& a, cudaStream_t stream);
+
+// ---------------------------------------------------------------- pack / patch embed
+hiera_status launch_fold_pack(const void* w, const void* gamma, const void* beta,
+                              const void* bias, int N, int K, int dtype_bf16, void* w_out,
+                              float* colsum, float* colconst, cudaStream_t stream);
+hiera_status launch_copy_pack(const void* w, const void* bias, int N, int K, int dtype_bf16,
+                              void* w_out, float* bias_out, cudaStream_t stream);
+hiera_status launch_patch_pack(const void* w, const void* bias, int dtype_bf16, float* wt,
+                               float* bias_out, cudaStream_t stream);
+hiera_status launch_patch_embed(const void* img, const void* w, const float* b,
+                                const void* pos, void* out, int B, int img_side,
+                                int dtype_bf16, cudaStream_t stream);
+
+}  // namespace hiera

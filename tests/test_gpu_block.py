@@ -1,0 +1,126 @@
+"""HieraBlock forward through the C ABI against the fp64 oracle.
+
+Tolerances (stated for the block): fp32 mode max-abs <= 1e-4; bf16 mode (bf16 inputs and
+weights, fp32 accumulation) rel-L2 <= 1e-2.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from mask_unit_windowed_b200 import binding as hb
+from mask_unit_windowed_b200 import synthetic as syn
+from oracle import unrolled as U
+
+from helpers import TORCH_DT, block_weights_dev, dev, host, max_abs, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+F32_MAX_ABS = 1e-4
+BF16_REL_L2 = 1e-2
+
+
+def run_case(B, tokens, d_in, d_out, heads, q_stride, window, mua, dtype, seed, affine):
+    transition = d_in != d_out
+    p = syn.block_params(seed, d_in, d_out, transition, dtype=dtype, affine=affine)
+    x = syn.activations(seed, (B, tokens, d_in), dtype=dtype)
+    desc = hb.BlockDesc(B=B, tokens=tokens, dim_in=d_in, dim_out=d_out, heads=heads,
+                        q_stride=q_stride, window_tokens=window, mask_unit_attn=mua,
+                        dtype=TORCH_DT[dtype])
+    packed = hb.block_pack(desc, block_weights_dev(p, dtype))
+    y = hb.block_forward(desc, packed, dev(x, dtype))
+    assert hb.device_status() == 0
+    ref = U.block_forward(x, p, heads, q_stride, window, mua)
+    return host(y), ref, desc, packed, p, x
+
+
+CASES = {
+    # name: (B, tokens, d_in, d_out, heads, q_stride, window, mask_unit_attn)
+    "stage0_windowed": (2, 256, 112, 112, 2, 1, 64, True),
+    "stage1_windowed": (2, 1024, 224, 224, 4, 1, 16, True),
+    "stage1_transition": (2, 256, 112, 224, 4, 4, 64, True),
+    "stage2_transition_lagged_mu": (2, 256, 224, 448, 8, 4, 16, True),
+    "stage2_transition_global": (2, 1024, 224, 448, 8, 4, 16, False),
+    "stage3_transition_small": (3, 64, 448, 896, 16, 4, 4, False),
+    "global_ragged": (3, 1000, 448, 448, 8, 1, 1, False),
+    "stage3_global": (2, 256, 896, 896, 16, 1, 1, False),
+}
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_block_bf16(name):
+    y, ref, *_ = run_case(*CASES[name], dtype="bf16", seed=5, affine="random")
+    assert y.shape == ref.shape
+    assert np.isfinite(y).all()
+    assert rel_l2(y, ref) <= BF16_REL_L2, rel_l2(y, ref)
+
+
+@pytest.mark.parametrize("name", ["stage0_windowed", "stage1_transition", "global_ragged",
+                                  "stage2_transition_lagged_mu", "stage3_transition_small"])
+def test_block_f32(name):
+    y, ref, *_ = run_case(*CASES[name], dtype="f32", seed=6, affine="random")
+    assert max_abs(y, ref) <= F32_MAX_ABS, max_abs(y, ref)
+
+
+def test_cfg1_stage0_block_f32():
+    """Single stage-0 block, fp32, batch 1: 32x32 grid unrolled into 16 mask units of 64,
+    dim 112, 2 heads, no q-pool, MLP 448; x ~ N(0,1), W ~ N(0,0.02), b=0, gamma=1, beta=0,
+    seed 0."""
+    y, ref, *_ = run_case(1, 1024, 112, 112, 2, 1, 64, True, dtype="f32", seed=0, affine="init")
+    assert max_abs(y, ref) <= F32_MAX_ABS, max_abs(y, ref)
+
+
+def test_cfg2_stage1_transition_bf16():
+    """Stage-1 transition block, bf16, batch 4: 128x128 tokens at dim 112 -> 224, 4 heads,
+    q_stride 4 (64 keys, 16 pooled queries per unit), MLP 896, seed 1."""
+    y, ref, *_ = run_case(4, 16384, 112, 224, 4, 4, 64, True, dtype="bf16", seed=1,
+                          affine="init")
+    assert rel_l2(y, ref) <= BF16_REL_L2, rel_l2(y, ref)
+
+
+def test_cfg3_stage2_global_bf16():
+    """Stage-2 global block, bf16, batch 8: 1024 tokens, dim 448, 8 heads, MLP 1792, seed 2."""
+    y, ref, *_ = run_case(8, 1024, 448, 448, 8, 1, 1, False, dtype="bf16", seed=2,
+                          affine="init")
+    assert rel_l2(y, ref) <= BF16_REL_L2, rel_l2(y, ref)
+
+
+def test_qkv_scatter_layout_bf16():
+    """The qkv GEMM writes q (pooled), k, v head-major with zero padding: compare the
+    workspace against the oracle's projections."""
+    B, tokens, d_in, d_out, heads, qs, window = 2, 256, 112, 224, 4, 4, 64
+    p = syn.block_params(7, d_in, d_out, True, dtype="bf16", affine="random")
+    x = syn.activations(7, (B, tokens, d_in), dtype="bf16")
+    desc = hb.BlockDesc(B=B, tokens=tokens, dim_in=d_in, dim_out=d_out, heads=heads,
+                        q_stride=qs, window_tokens=window)
+    packed = hb.block_pack(desc, block_weights_dev(p, "bf16"))
+    ws = torch.empty(hb.block_workspace_bytes(desc), dtype=torch.uint8, device="cuda")
+    hb.block_forward(desc, packed, dev(x), workspace=ws)
+    torch.cuda.synchronize()
+    offs = hb.block_workspace_layout(desc)
+    nW = tokens // window
+    Tkv, Tq = window, window // qs
+    xn = U.layer_norm(x, p["norm1_w"], p["norm1_b"])
+    qkv = U.linear(xn, p["qkv_w"], p["qkv_b"]).reshape(B, Tkv, nW, 3, heads, 56)
+    qkv = qkv.transpose(3, 0, 2, 4, 1, 5)               # [3, B, nW, h, T, 56]
+    q = qkv[0].reshape(B, nW, heads, qs, Tq, 56).max(axis=3)
+
+    def view(off, T):
+        n = B * nW * heads * T * 64
+        t = ws[off:off + 2 * n].view(torch.bfloat16).reshape(B, nW, heads, T, 64)
+        return host(t)
+    for got, want in ((view(offs[0], Tq), q), (view(offs[1], Tkv), qkv[1]),
+                      (view(offs[2], Tkv), qkv[2])):
+        assert np.all(got[..., 56:] == 0)
+        assert rel_l2(got[..., :56], want) < 5e-3
+    r = host(ws[offs[4]:offs[4] + 2 * B * (tokens // 4) * d_out].view(torch.bfloat16)).reshape(
+        B, tokens // 4, d_out)
+    r_ref = U.max_pool_tokens(U.linear(xn, p["proj_w"], p["proj_b"]), qs)
+    assert rel_l2(r, r_ref) < 5e-3
+
+
+def test_repeat_is_deterministic_bf16():
+    args = CASES["stage1_transition"]
+    y1, _, desc, packed, p, x = run_case(*args, dtype="bf16", seed=8, affine="random")
+    y2 = host(hb.block_forward(desc, packed, dev(x)))
+    np.testing.assert_array_equal(y1, y2)

@@ -1,0 +1,30 @@
+"""Device-side bounded waits: a wait that nothing completes records HIERA_ERR_TIMEOUT and
+the kernel returns; the context stays usable."""
+
+import pytest
+import torch
+
+from mask_unit_windowed_b200 import binding as hb
+
+pytestmark = pytest.mark.gpu
+
+
+def test_timeout_probe_reports_and_recovers():
+    assert hb.device_status() == 0
+    hb.timeout_probe(2000)                 # 2 ms limit
+    assert hb.device_status() == 7         # HIERA_ERR_TIMEOUT, then cleared
+    assert hb.device_status() == 0
+    x = torch.randn(1, 64, 112, device="cuda").to(torch.bfloat16)
+    u = hb.unroll(x, 8, 3)
+    assert torch.equal(hb.reroll(u, 8, 3).reshape(1, 64, 112), x)
+    assert hb.device_status() == 0
+
+
+def test_workspace_too_small_rejected():
+    desc = hb.BlockDesc(B=1, tokens=256, dim_in=112, dim_out=112, heads=2)
+    x = torch.zeros(1, 256, 112, device="cuda", dtype=torch.bfloat16)
+    packed = torch.zeros(hb.block_packed_bytes(desc), dtype=torch.uint8, device="cuda")
+    ws = torch.empty(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(hb.HieraError) as e:
+        hb.block_forward(desc, packed, x, workspace=ws)
+    assert e.value.code == 5
