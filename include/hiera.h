@@ -240,6 +240,22 @@ HIERA_API hiera_status hiera_backbone_forward(const hiera_backbone_desc* desc, c
                                     size_t workspace_bytes, hiera_stream_t stream);
 
 /* --------------------------------------------------------------------------------
+ * Launch profiling (host-side bookkeeping only). Between hiera_profile_begin() and
+ * hiera_profile_end(), every kernel launch the library makes, on whatever stream the
+ * call was given, is preceded by cudaEventRecord(events[i], stream) and its kernel id is
+ * stored in kinds[i] (i counts launches from 0; launches beyond `capacity` are not
+ * marked). `events` are cudaEvent_t handles created by the caller with timing enabled.
+ * hiera_profile_end() records events[n] on `stream` (n = launches seen, if n <
+ * capacity) and returns n, so launch i took elapsed(events[i], events[i+1]) when all
+ * launches went to one stream. Works under CUDA-graph stream capture (the records
+ * become event nodes). Not thread-safe: one session at a time per process.
+ * hiera_kernel_name() names a kernel id (static string).
+ * -------------------------------------------------------------------------------- */
+HIERA_API hiera_status hiera_profile_begin(void* const* events, int capacity, int* kinds);
+HIERA_API int hiera_profile_end(hiera_stream_t stream);
+HIERA_API const char* hiera_kernel_name(int kind);
+
+/* --------------------------------------------------------------------------------
  * Self-test of the bounded-wait machinery: launches one kernel that waits on an
  * mbarrier nothing will complete, for at most limit_us microseconds; the wait records
  * HIERA_ERR_TIMEOUT in the device status word and the kernel returns normally.

@@ -99,6 +99,10 @@ def lib() -> ctypes.CDLL:
             "hiera_backbone_forward": ([ctypes.POINTER(BackboneDescC), P, P,
                                         ctypes.POINTER(ctypes.c_void_p), P, S, P], I),
             "hiera_debug_timeout_probe": ([I, P], I),
+            "hiera_profile_begin": ([ctypes.POINTER(ctypes.c_void_p), I,
+                                     ctypes.POINTER(ctypes.c_int)], I),
+            "hiera_profile_end": ([P], I),
+            "hiera_kernel_name": ([I], ctypes.c_char_p),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -346,3 +350,37 @@ def timeout_probe(limit_us: int, stream=None):
 
 def status_string(code: int) -> str:
     return lib().hiera_status_string(code).decode()
+
+
+def kernel_name(kind: int) -> str:
+    return lib().hiera_kernel_name(kind).decode()
+
+
+class LaunchProfile:
+    """Marks every library launch with a CUDA event (see hiera_profile_begin).
+
+    with LaunchProfile(capacity) as prof:  ... library calls on one stream ...
+    prof.durations_ms() -> list of (kernel name, ms) once the work has completed.
+    """
+
+    def __init__(self, capacity: int = 512, stream=None):
+        self.capacity = capacity
+        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(capacity)]
+        self._handles = (ctypes.c_void_p * capacity)(*[e.cuda_event for e in self.events])
+        self._kinds = (ctypes.c_int * capacity)()
+        self.stream = stream
+        self.count = 0
+
+    def __enter__(self):
+        _check(lib().hiera_profile_begin(self._handles, self.capacity, self._kinds),
+               "hiera_profile_begin")
+        return self
+
+    def __exit__(self, *exc):
+        self.count = lib().hiera_profile_end(_stream(self.stream))
+        return False
+
+    def durations_ms(self):
+        n = min(self.count, self.capacity - 1)
+        return [(kernel_name(self._kinds[i]), self.events[i].elapsed_time(self.events[i + 1]))
+                for i in range(n)]

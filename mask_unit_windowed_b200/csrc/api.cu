@@ -494,6 +494,25 @@ int g_num_sms() {
 
 unsigned int* g_status_ptr() { return dev_info().status; }
 
+namespace {
+struct ProfileSession {
+  void* const* events = nullptr;
+  int* kinds = nullptr;
+  int capacity = 0;
+  int count = 0;
+  bool open = false;
+} g_prof;
+}  // namespace
+
+void profile_mark(int kind, cudaStream_t stream) {
+  if (!g_prof.open) return;
+  if (g_prof.count < g_prof.capacity) {
+    cudaEventRecord(static_cast<cudaEvent_t>(g_prof.events[g_prof.count]), stream);
+    g_prof.kinds[g_prof.count] = kind;
+  }
+  ++g_prof.count;
+}
+
 uint64_t g_wait_limit_ns() {
   static uint64_t limit = [] {
     const char* e = getenv("HIERA_WAIT_LIMIT_MS");
@@ -774,9 +793,36 @@ hiera_status hiera_backbone_forward(const hiera_backbone_desc* desc, const void*
   return HIERA_OK;
 }
 
+hiera_status hiera_profile_begin(void* const* events, int capacity, int* kinds) {
+  if (events == nullptr || kinds == nullptr || capacity < 1) return HIERA_ERR_INVALID_ARG;
+  g_prof.events = events;
+  g_prof.kinds = kinds;
+  g_prof.capacity = capacity;
+  g_prof.count = 0;
+  g_prof.open = true;
+  return HIERA_OK;
+}
+
+int hiera_profile_end(hiera_stream_t stream) {
+  if (!g_prof.open) return 0;
+  g_prof.open = false;
+  if (g_prof.count < g_prof.capacity)
+    cudaEventRecord(static_cast<cudaEvent_t>(g_prof.events[g_prof.count]), (cudaStream_t)stream);
+  return g_prof.count;
+}
+
+const char* hiera_kernel_name(int kind) {
+  static const char* names[K_COUNT] = {
+      "patch_embed", "unroll_reroll", "gemm_qkv_lnfold", "gemm_fc1_lnfold_gelu",
+      "gemm_bias_residual", "attention_tiled", "attention_packed", "f32_gemm",
+      "f32_attention", "f32_row_stats", "pack", "timeout_probe"};
+  return (kind >= 0 && kind < K_COUNT) ? names[kind] : "unknown";
+}
+
 hiera_status hiera_debug_timeout_probe(int limit_us, hiera_stream_t stream) {
   if (limit_us < 1 || limit_us > 10000000) return HIERA_ERR_INVALID_ARG;
   HIERA_TRY(check_device());
+  profile_mark(K_PROBE, (cudaStream_t)stream);
   timeout_probe_kernel<<<1, 32, 0, (cudaStream_t)stream>>>((uint64_t)limit_us * 1000ull,
                                                            g_status_ptr());
   return cudaGetLastError() == cudaSuccess ? HIERA_OK : HIERA_ERR_CUDA;

@@ -305,6 +305,7 @@ hiera_status launch_attention_bf16(const AttnArgs& a, cudaStream_t stream) {
   p.d_out = a.d_out;
   p.sl2 = (float)(1.4426950408889634 / sqrt(56.0));
   if (p.units <= 0 || a.Tq <= 0 || a.Tkv <= 0) return HIERA_OK;
+  profile_mark(a.Tq <= 16 && a.Tkv <= 64 ? K_ATTN_PACKED : K_ATTN_TILED, stream);
   if (a.Tq <= 16 && a.Tkv <= 16) {
     attn_packed_kernel<16><<<(p.units + 3) / 4, 128, 4 * (2048 + 2 * 16 * 128), stream>>>(p);
   } else if (a.Tq <= 16 && a.Tkv <= 64) {

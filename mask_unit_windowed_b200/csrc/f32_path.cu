@@ -200,6 +200,7 @@ hiera_status launch_row_stats_f32(const float* x, int M, int K, float eps, float
                                   cudaStream_t stream) {
   if (M <= 0) return HIERA_OK;
   const long long threads = (long long)M * 32;
+  profile_mark(K_F32_STATS, stream);
   row_stats_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, stream>>>(x, M, K, eps, stats);
   return cudaGetLastError() == cudaSuccess ? HIERA_OK : HIERA_ERR_CUDA;
 }
@@ -208,6 +209,7 @@ hiera_status launch_gemm_f32(const F32GemmArgs& a, cudaStream_t stream) {
   if (a.M <= 0 || a.N <= 0) return HIERA_OK;
   dim3 grid((a.N + TB - 1) / TB, (a.M + TB - 1) / TB);
   if (grid.y > 65535) return HIERA_ERR_SHAPE;
+  profile_mark(K_F32_GEMM, stream);
   gemm_f32_kernel<<<grid, 256, 0, stream>>>(a);
   return cudaGetLastError() == cudaSuccess ? HIERA_OK : HIERA_ERR_CUDA;
 }
@@ -218,6 +220,7 @@ hiera_status launch_attention_f32(const F32AttnArgs& a, cudaStream_t stream) {
   if (units <= 0 || Tq <= 0) return HIERA_OK;
   dim3 grid(units, (Tq + QPB - 1) / QPB);
   if (grid.y > 65535) return HIERA_ERR_SHAPE;
+  profile_mark(K_F32_ATTN, stream);
   attention_f32_kernel<<<grid, 256, 0, stream>>>(a);
   return cudaGetLastError() == cudaSuccess ? HIERA_OK : HIERA_ERR_CUDA;
 }

@@ -544,6 +544,8 @@ hiera_status run(const TcGemmArgs& a, cudaStream_t stream) {
   if (tiles == 0) return HIERA_OK;
   int grid = g_num_sms();
   if (grid > tiles) grid = tiles;
+  profile_mark(EPI == EPI_QKV ? K_GEMM_QKV : (EPI == EPI_GELU ? K_GEMM_GELU : K_GEMM_STORE),
+               stream);
   kern<<<grid, FOLD ? 320 : 192, C::SMEM_BYTES, stream>>>(tmA, tmB, p);
   return cudaGetLastError() == cudaSuccess ? HIERA_OK : HIERA_ERR_CUDA;
 }

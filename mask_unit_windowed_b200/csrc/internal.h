@@ -13,6 +13,14 @@ int g_num_sms();                         // SM count of the current device (cach
 uint64_t g_wait_limit_ns();              // bound on every device-side wait
 unsigned int* g_status_ptr();            // device address of the status word (current device)
 
+// kernel ids reported by the launch profiler (hiera_profile_begin)
+enum KernelId {
+  K_PATCH_EMBED = 0, K_PERMUTE = 1, K_GEMM_QKV = 2, K_GEMM_GELU = 3, K_GEMM_STORE = 4,
+  K_ATTN_TILED = 5, K_ATTN_PACKED = 6, K_F32_GEMM = 7, K_F32_ATTN = 8, K_F32_STATS = 9,
+  K_PACK = 10, K_PROBE = 11, K_COUNT = 12
+};
+void profile_mark(int kind, cudaStream_t stream);  // no-op unless a session is open
+
 cudaError_t launch_permute(bool unroll, const void* x, void* y, int B, int G, int C, int L,
                            int elem_bytes, cudaStream_t stream);
 

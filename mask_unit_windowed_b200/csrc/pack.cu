@@ -93,6 +93,7 @@ hiera_status launch_patch_pack(const void* w, const void* bias, int dtype_bf16, 
                                float* bias_out, cudaStream_t stream) {
   const int cout = 112, ktot = 196;
   const unsigned blocks = (cout * ktot + 255) / 256;
+  profile_mark(K_PACK, stream);
   if (dtype_bf16)
     patch_pack_kernel<bf16><<<blocks, 256, 0, stream>>>(
         static_cast<const bf16*>(w), static_cast<const bf16*>(bias), cout, ktot, wt, bias_out);
@@ -107,6 +108,7 @@ hiera_status launch_fold_pack(const void* w, const void* gamma, const void* beta
                               float* colsum, float* colconst, cudaStream_t stream) {
   if (N <= 0 || K <= 0) return HIERA_OK;
   const unsigned blocks = (unsigned)(((long long)N * 32 + 255) / 256);
+  profile_mark(K_PACK, stream);
   if (dtype_bf16)
     fold_pack_kernel<bf16><<<blocks, 256, 0, stream>>>(
         static_cast<const bf16*>(w), static_cast<const bf16*>(gamma),
@@ -126,6 +128,7 @@ hiera_status launch_copy_pack(const void* w, const void* bias, int N, int K, int
   if (NK <= 0) return HIERA_OK;
   long long blocks = (NK + 255) / 256;
   if (blocks > 4096) blocks = 4096;
+  profile_mark(K_PACK, stream);
   if (dtype_bf16)
     copy_pack_kernel<bf16><<<(unsigned)blocks, 256, 0, stream>>>(
         static_cast<const bf16*>(w), static_cast<const bf16*>(bias), NK, N,

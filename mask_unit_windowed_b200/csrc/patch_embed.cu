@@ -126,6 +126,7 @@ hiera_status launch_patch_embed(const void* img, const void* w, const float* b, 
   static bool attr_done[2][64] = {{false}};
   int dev = 0;
   cudaGetDevice(&dev);
+  profile_mark(K_PATCH_EMBED, stream);
   if (dtype_bf16) {
     if (dev < 64 && !attr_done[1][dev]) {
       if (cudaFuncSetAttribute(patch_embed_kernel<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -40,6 +40,7 @@ cudaError_t launch_permute(bool unroll, const void* x, void* y, int B, int G, in
   long long blocks = (total + 255) / 256;
   const long long cap = (long long)g_num_sms() * 16;
   if (blocks > cap) blocks = cap;
+  profile_mark(K_PERMUTE, stream);
   if (unroll)
     permute_kernel<true><<<(int)blocks, 256, 0, stream>>>(
         static_cast<const uint4*>(x), static_cast<uint4*>(y), B, G, L, chunks, total);
