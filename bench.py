@@ -1,0 +1,439 @@
+"""Throughput of the Hiera-B+ backbone forward (512x512x4 images, bf16) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one forward of the whole backbone (patch embedding + pos_embed + Unroll,
+24 blocks, Reroll of the four stage features) over one batch of 8 synthetic images per
+GPU, replayed from a CUDA graph of the library's launches. Inputs are resident in HBM
+when a timed step starts; L2 is flushed (256 MiB write) before every step and the step
+is timed with CUDA events on the launching stream; the timed value sums the K step
+windows and takes the max over ranks. Multi-GPU runs are independent replicas (one
+batch per rank, no collective on the data path): value = all images / max time.
+
+Rank 0 prints one JSON line with the headline images/s, the roofline of the dominant
+kernel (per-launch CUDA events inside a separately captured graph of the same
+forward), the end-to-end number through the public API with host buffers, SM clocks
+sampled during the timed region, and the CPU oracle timed on a bounded sample.
+
+--impl reference times the CPU oracle (fp64 numpy, formulation U) on the same metric:
+each step is one 512^2 image through the whole backbone; the number of steps is capped
+so that the run ends within a few minutes.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "Hiera-B+ backbone images/s (512², bf16, 1 B200); attn+GEMM % of BF16 peak"
+UNIT = "images/s"
+IMG = 512
+BATCH = 8
+SEED = 3
+L2_FLUSH_BYTES = 256 << 20
+STAGE_DIMS = (112, 224, 448, 896)
+STAGE_HEADS = (2, 4, 8, 16)
+STAGE_DEPTHS = (2, 3, 16, 3)
+HD = 56
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return (float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]),
+                "measured")
+    except (OSError, KeyError, ValueError):
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def launch_flops(img: int, B: int):
+    """Algorithmic FLOPs of every library launch of one backbone forward, in launch order
+    (head_dim 56, not the padded 64). Returns list of (kind-class, flops, bytes_hint)."""
+    G0 = img // 4
+    out = [("patch_embed", 2.0 * B * G0 * G0 * 112 * 196)]
+    prev = STAGE_DIMS[0]
+    i = 0
+    for s, depth in enumerate(STAGE_DEPTHS):
+        Gs = G0 >> s
+        for j in range(depth):
+            trans = s > 0 and j == 0
+            d_in = prev if trans else STAGE_DIMS[s]
+            d = STAGE_DIMS[s]
+            n_in = (2 * Gs) ** 2 if trans else Gs * Gs
+            nq = Gs * Gs
+            mua = s < 2
+            flat_mu = 64 >> (2 * s)
+            window = flat_mu * (4 if trans else 1)
+            nW = n_in // window if mua else 1
+            tkv = n_in // nW
+            tq = tkv // (4 if trans else 1)
+            n1 = 3 * d + (d if trans else 0)
+            out.append(("gemm", 2.0 * B * n_in * d_in * n1))
+            out.append(("attention", 4.0 * B * STAGE_HEADS[s] * nW * tq * tkv * HD))
+            out.append(("gemm", 2.0 * B * nq * d * d))
+            out.append(("gemm", 2.0 * B * nq * d * 4 * d))
+            out.append(("gemm", 2.0 * B * nq * 4 * d * d))
+            if i in (1, 4, 20, 23):
+                out.append(("unroll_reroll", 0.0))
+            i += 1
+        prev = STAGE_DIMS[s]
+    return out
+
+
+KIND_CLASS = {"patch_embed": "patch_embed", "unroll_reroll": "unroll_reroll",
+              "gemm_qkv_lnfold": "gemm", "gemm_fc1_lnfold_gelu": "gemm",
+              "gemm_bias_residual": "gemm", "attention_tiled": "attention",
+              "attention_packed": "attention"}
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.02):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons = [], 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        self.ok = False
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # NVML missing: report no clock record
+            return self
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+        return False
+
+    def record(self):
+        if not self.ok or not self.samples:
+            return None
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "samples": len(self.samples),
+                "reasons": [n for bit, n in self.REASONS.items() if self.reasons & bit]}
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_images_per_s(budget_s: float, max_steps: int, warmup: int):
+    """Time the CPU oracle: each step one 512^2 image through the whole backbone."""
+    from mask_unit_windowed_b200 import synthetic as syn
+    from oracle import unrolled as U
+    p = syn.backbone_params(SEED, IMG, dtype="bf16")
+    img = syn.image(SEED, 1, IMG)
+    for _ in range(min(warmup, 1)):
+        U.backbone_forward(img, p)
+    times = []
+    t_start = time.perf_counter()
+    while len(times) < max_steps:
+        t0 = time.perf_counter()
+        U.backbone_forward(img, p)
+        times.append(time.perf_counter() - t0)
+        if time.perf_counter() - t_start + times[-1] > budget_s:
+            break
+    return len(times) / sum(times), len(times)
+
+
+def run_reference(args, rank: int):
+    if rank != 0:
+        return
+    value, steps = oracle_images_per_s(150.0, args.steps, args.warmup)
+    cores = blas_threads()
+    cpu = {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+           "sample": f"{steps} step(s) of one {IMG}x{IMG}x4 image through the full backbone "
+                     "(fp64 numpy oracle, unrolled formulation)"}
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": steps, "warmup": min(args.warmup, 1),
+            "ms_per_step": 1000.0 / value, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"Hiera-B+ backbone forward, {IMG}x{IMG}x4 image, batch 1 "
+                                   "per step, CPU oracle", "img": IMG},
+            "cpu_baseline": cpu,
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+
+    from mask_unit_windowed_b200 import binding as hb
+    from mask_unit_windowed_b200 import synthetic as syn
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    hbm_gbs, tf_burst, tf_sust, peak_src = peaks()
+    B = args.batch
+
+    # ---- weights and inputs (synthetic, seeded; random-init Hiera-B+)
+    params = syn.backbone_params(SEED, IMG, dtype="bf16")
+
+    def t(a):
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev, torch.bfloat16)
+
+    weights = {"patch_w": t(params["patch_w"]), "patch_b": t(params["patch_b"]),
+               "pos_embed": t(params["pos_embed"]),
+               "blocks": [{k: t(v) for k, v in blk.items()} for blk in params["blocks"]]}
+    desc = hb.BackboneDesc(B=B, img=IMG)
+    packed = hb.backbone_pack(desc, weights)
+    del weights
+    img_host = torch.from_numpy(syn.image(SEED + rank, B, IMG)).to(torch.bfloat16).pin_memory()
+    img = img_host.to(dev)
+    feats = [torch.empty(s, dtype=torch.bfloat16, device=dev) for s in desc.feature_shapes()]
+    ws = torch.empty(hb.backbone_workspace_bytes(desc), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def forward():
+        hb.backbone_forward(desc, packed, img, feats=feats, workspace=ws)
+
+    with torch.cuda.stream(stream):
+        forward()
+    torch.cuda.synchronize()
+    st = hb.device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {hb.status_string(st)}")
+
+    # ---- CUDA graph of one forward (the library's launches only)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        forward()
+    torch.cuda.synchronize()
+
+    # ---- instrumented graph: an event before every launch (kernel breakdown / roofline)
+    prof = hb.LaunchProfile(capacity=256, stream=stream)
+    pgraph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(pgraph, stream=stream):
+        with prof:
+            forward()
+    torch.cuda.synchronize()
+    n_launches = prof.count
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            graph.replay()
+    torch.cuda.synchronize()
+
+    # ---- timed region
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clocks:
+        with torch.cuda.stream(stream):
+            for k in range(args.steps):
+                flush.fill_(k & 0xFF)
+                starts[k].record(stream)
+                graph.replay()
+                ends[k].record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    st = hb.device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"device status after timing: {hb.status_string(st)}")
+    if world > 1:
+        tt = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    images = B * args.steps * world
+    value = images / (total_ms / 1000.0)
+    ms_per_step = total_ms / args.steps
+
+    # ---- per-kernel breakdown from the instrumented graph (same workload, L2 flushed)
+    reps = 5
+    per_launch = None
+    with torch.cuda.stream(stream):
+        for r in range(reps):
+            flush.fill_(r)
+            pgraph.replay()
+            torch.cuda.synchronize()
+            d = prof.durations_ms()
+            per_launch = [(n, ms) for n, ms in d] if per_launch is None else \
+                [(n, a + ms) for (n, a), (_, ms) in zip(per_launch, d)]
+    per_launch = [(n, ms / reps) for n, ms in per_launch]
+    flops = launch_flops(IMG, B)
+    classes = {}
+    if len(flops) == len(per_launch) and all(KIND_CLASS.get(n) == c for (n, _), (c, _) in
+                                             zip(per_launch, flops)):
+        for (n, ms), (c, fl) in zip(per_launch, flops):
+            e = classes.setdefault(c, {"launches": 0, "ms": 0.0, "gflop": 0.0})
+            e["launches"] += 1
+            e["ms"] += ms
+            e["gflop"] += fl / 1e9
+    else:
+        for n, ms in per_launch:
+            e = classes.setdefault(KIND_CLASS.get(n, n), {"launches": 0, "ms": 0.0, "gflop": 0.0})
+            e["launches"] += 1
+            e["ms"] += ms
+    step_ms_prof = sum(ms for _, ms in per_launch)
+    for c, e in classes.items():
+        e["share"] = e["ms"] / step_ms_prof if step_ms_prof > 0 else None
+        e["tflops"] = e["gflop"] / e["ms"] if e["ms"] > 0 else 0.0
+        e["frac_of_bf16_sustained"] = e["tflops"] / tf_sust
+    dominant = max((c for c in classes if c in ("gemm", "attention")),
+                   key=lambda c: classes[c]["ms"])
+    dom = classes[dominant]
+    attn_gemm_gflop = sum(fl for c, fl in flops if c in ("gemm", "attention")) / 1e9
+    roofline = {"bound": "tensor", "kernel": {"gemm": "tcgen05 GEMM (all Linear layers)",
+                                              "attention": "mask-unit / global attention"}
+                [dominant],
+                "achieved": dom["tflops"], "peak": tf_sust, "unit": "TFLOP/s",
+                "frac": dom["tflops"] / tf_sust, "traffic": None,
+                "peak_kind": f"bf16 dense sustained ({peak_src})",
+                "launches_per_step": dom["launches"],
+                "gflop_per_launch": dom["gflop"] / max(dom["launches"], 1),
+                "ms_per_launch": dom["ms"] / max(dom["launches"], 1)}
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        feats_host = [torch.empty(f.shape, dtype=f.dtype, pin_memory=True) for f in feats]
+        es = [torch.cuda.Event(enable_timing=True) for _ in range(args.e2e_steps)]
+        ee = [torch.cuda.Event(enable_timing=True) for _ in range(args.e2e_steps)]
+        with torch.cuda.stream(stream):
+            for k in range(args.e2e_steps + 2):
+                flush.fill_(k & 0xFF)
+                if k >= 2:
+                    es[k - 2].record(stream)
+                img.copy_(img_host, non_blocking=True)
+                hb.backbone_forward(desc, packed, img, feats=feats, workspace=ws, stream=stream)
+                for fh, f in zip(feats_host, feats):
+                    fh.copy_(f, non_blocking=True)
+                if k >= 2:
+                    ee[k - 2].record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = sum(s.elapsed_time(e) for s, e in zip(es, ee))
+        if world > 1:
+            tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e2e_ms = float(tt.item())
+        e2e = {"value": B * args.e2e_steps * world / (e2e_ms / 1000.0), "unit": UNIT,
+               "h2d_bytes_per_step": img.numel() * img.element_size(),
+               "d2h_bytes_per_step": sum(f.numel() * f.element_size() for f in feats),
+               "steps": args.e2e_steps,
+               "api": "hiera_backbone_forward (eager) + pinned H2D image / D2H features"}
+
+    del graph, pgraph
+    if rank != 0:
+        return
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        v, n = oracle_images_per_s(20.0, 3, 0)
+        cpu = {"value": v, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{n} image(s) of {IMG}x{IMG}x4 through the full backbone "
+                         "(fp64 numpy oracle, unrolled formulation)"}
+    gflop_per_image = sum(fl for _, fl in flops) / B / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"Hiera-B+ backbone forward, {IMG}x{IMG}x4 bf16 images, "
+                               f"batch {B} per GPU (random-init weights, seed {SEED})",
+                   "img": IMG, "batch_per_gpu": B, "global_batch": B * world,
+                   "parallelism": f"replicas x{world} (no data-path collective)",
+                   "l2": "flushed before every step (256 MiB write)",
+                   "timing": "CUDA-graph replay of the library launches, per-step CUDA events"},
+        "tflops": gflop_per_image * images / (total_ms * 1e-3) * 1e-3,
+        "attn_gemm_frac_of_bf16_peak": attn_gemm_gflop / (ms_per_step * 1e-3) / 1e3 / tf_sust,
+        "gflop_per_image": gflop_per_image,
+        "roofline": roofline,
+        "kernels": classes,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "clocks": clocks.record(),
+        "gpu_launches": n_launches * args.steps,
+        "launches_per_step": n_launches,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--batch", type=int, default=BATCH)
+    ap.add_argument("--e2e-steps", type=int, default=30)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

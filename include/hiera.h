@@ -262,6 +262,10 @@ HIERA_API const char* hiera_kernel_name(int kind);
  * -------------------------------------------------------------------------------- */
 HIERA_API hiera_status hiera_debug_timeout_probe(int limit_us, hiera_stream_t stream);
 
+/* Self-test of the tensor-core path's GELU: y[i] = GELU(x[i]) for n fp32 device values,
+ * computed exactly as the fc1 epilogue does (erf after Abramowitz & Stegun eq. 7.1.28). */
+HIERA_API hiera_status hiera_debug_gelu(const float* x, float* y, int n, hiera_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

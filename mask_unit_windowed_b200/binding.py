@@ -99,6 +99,7 @@ def lib() -> ctypes.CDLL:
             "hiera_backbone_forward": ([ctypes.POINTER(BackboneDescC), P, P,
                                         ctypes.POINTER(ctypes.c_void_p), P, S, P], I),
             "hiera_debug_timeout_probe": ([I, P], I),
+            "hiera_debug_gelu": ([P, P, I, P], I),
             "hiera_profile_begin": ([ctypes.POINTER(ctypes.c_void_p), I,
                                      ctypes.POINTER(ctypes.c_int)], I),
             "hiera_profile_end": ([P], I),
@@ -344,6 +345,14 @@ def device_status(stream=None) -> int:
     return lib().hiera_get_device_status(_stream(stream))
 
 
+def debug_gelu(x: torch.Tensor, stream=None) -> torch.Tensor:
+    _need(x, "x")
+    y = torch.empty_like(x)
+    _check(lib().hiera_debug_gelu(_ptr(x), _ptr(y), x.numel(), _stream(stream)),
+           "hiera_debug_gelu")
+    return y
+
+
 def timeout_probe(limit_us: int, stream=None):
     _check(lib().hiera_debug_timeout_probe(limit_us, _stream(stream)), "hiera_debug_timeout_probe")
 
@@ -366,6 +375,9 @@ class LaunchProfile:
     def __init__(self, capacity: int = 512, stream=None):
         self.capacity = capacity
         self.events = [torch.cuda.Event(enable_timing=True) for _ in range(capacity)]
+        for e in self.events:      # torch creates the CUDA event on first record
+            e.record()
+        torch.cuda.synchronize()
         self._handles = (ctypes.c_void_p * capacity)(*[e.cuda_event for e in self.events])
         self._kinds = (ctypes.c_int * capacity)()
         self.stream = stream

@@ -474,6 +474,11 @@ BackboneWs backbone_ws_layout(const hiera_backbone_desc* bd, const BlockPlan pla
   return L;
 }
 
+__global__ void gelu_probe_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) y[i] = gelu_fast(x[i]);
+}
+
 __global__ void timeout_probe_kernel(uint64_t limit_ns, unsigned int* status) {
   __shared__ uint64_t bar;
   if (threadIdx.x == 0) {
@@ -495,6 +500,17 @@ int g_num_sms() {
 unsigned int* g_status_ptr() { return dev_info().status; }
 
 namespace {
+// Under stream capture a plain cudaEventRecord only orders the capture; the external
+// flag makes it an event-record node that re-records on every graph replay.
+void record_profile_event(cudaEvent_t ev, cudaStream_t stream) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaStreamIsCapturing(stream, &cs);
+  if (cs == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(ev, stream, cudaEventRecordExternal);
+  else
+    cudaEventRecord(ev, stream);
+}
+
 struct ProfileSession {
   void* const* events = nullptr;
   int* kinds = nullptr;
@@ -507,7 +523,7 @@ struct ProfileSession {
 void profile_mark(int kind, cudaStream_t stream) {
   if (!g_prof.open) return;
   if (g_prof.count < g_prof.capacity) {
-    cudaEventRecord(static_cast<cudaEvent_t>(g_prof.events[g_prof.count]), stream);
+    record_profile_event(static_cast<cudaEvent_t>(g_prof.events[g_prof.count]), stream);
     g_prof.kinds[g_prof.count] = kind;
   }
   ++g_prof.count;
@@ -807,7 +823,8 @@ int hiera_profile_end(hiera_stream_t stream) {
   if (!g_prof.open) return 0;
   g_prof.open = false;
   if (g_prof.count < g_prof.capacity)
-    cudaEventRecord(static_cast<cudaEvent_t>(g_prof.events[g_prof.count]), (cudaStream_t)stream);
+    record_profile_event(static_cast<cudaEvent_t>(g_prof.events[g_prof.count]),
+                         (cudaStream_t)stream);
   return g_prof.count;
 }
 
@@ -817,6 +834,14 @@ const char* hiera_kernel_name(int kind) {
       "gemm_bias_residual", "attention_tiled", "attention_packed", "f32_gemm",
       "f32_attention", "f32_row_stats", "pack", "timeout_probe"};
   return (kind >= 0 && kind < K_COUNT) ? names[kind] : "unknown";
+}
+
+hiera_status hiera_debug_gelu(const float* x, float* y, int n, hiera_stream_t stream) {
+  if (x == nullptr || y == nullptr || n < 1) return HIERA_ERR_INVALID_ARG;
+  HIERA_TRY(check_device());
+  profile_mark(K_PROBE, (cudaStream_t)stream);
+  gelu_probe_kernel<<<(n + 255) / 256, 256, 0, (cudaStream_t)stream>>>(x, y, n);
+  return cudaGetLastError() == cudaSuccess ? HIERA_OK : HIERA_ERR_CUDA;
 }
 
 hiera_status hiera_debug_timeout_probe(int limit_us, hiera_stream_t stream) {

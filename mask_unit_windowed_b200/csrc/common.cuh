@@ -85,6 +85,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
   }
 }
 
+// Orders this thread's prior generic-proxy shared-memory accesses before later
+// async-proxy (TMA / tensor-core) accesses of the same memory.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -182,6 +188,19 @@ __device__ __forceinline__ void tc_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[1
       : "r"(taddr));
 }
 
+__device__ __forceinline__ void tc_ld_32x32b_x8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7])
+      : "r"(taddr));
+}
+
+// Named barrier among `count` threads (a multiple of 32) of the CTA.
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // Shared-memory matrix descriptor for a K-major operand tile stored with the 128-byte
 // swizzle: rows of 64 bf16 (128 B), 8-row core groups 1024 B apart. Fields: start
 // address >> 4 in bits 0-13, leading-dimension byte offset >> 4 in bits 16-29 (unused
@@ -216,6 +235,34 @@ __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v 
 
 __device__ __forceinline__ float gelu_erf(float x) {
   return 0.5f * x * (1.0f + erff(x * 0.70710678118654752440f));
+}
+
+// erf by Abramowitz & Stegun, Handbook of Mathematical Functions, eq. 7.1.28 (after
+// Hastings): for x >= 0, erf(x) = 1 - (1 + a1 x + ... + a6 x^6)^-16 with |error| <= 3e-7.
+// One approximate reciprocal (MUFU) and FMAs; the 16th power by four squarings, so large
+// x underflows cleanly to erf = 1. Odd extension for x < 0.
+__device__ __forceinline__ float erf_as7128(float x) {
+  const float ax = fabsf(x);
+  float p = fmaf(0.0000430638f, ax, 0.0002765672f);
+  p = fmaf(p, ax, 0.0001520143f);
+  p = fmaf(p, ax, 0.0092705272f);
+  p = fmaf(p, ax, 0.0422820123f);
+  p = fmaf(p, ax, 0.0705230784f);
+  p = fmaf(p, ax, 1.0f);
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(p));
+  r = r * r;
+  r = r * r;
+  r = r * r;
+  r = r * r;
+  return copysignf(1.0f - r, x);
+}
+
+// GELU(x) = x * Phi(x) = 0.5 x (1 + erf(x / sqrt 2)) with the erf above (|error| of the
+// result <= ~1e-6 |x|, far below bf16 resolution). Used by the bf16 tensor-core path.
+__device__ __forceinline__ float gelu_fast(float x) {
+  const float e = erf_as7128(x * 0.70710678118654752440f);
+  return fmaf(0.5f * x, e, 0.5f * x);
 }
 
 // ------------------------------------------------------------------ Unroll map

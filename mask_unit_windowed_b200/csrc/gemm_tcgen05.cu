@@ -32,7 +32,8 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int STAGES = 4;
+constexpr int EPI_WARPS = 8;              // 2 per TMEM lane quarter, each half the columns
+constexpr int EPI_THREADS = EPI_WARPS * 32;
 
 struct KParams {
   int M, N, K;
@@ -52,161 +53,85 @@ struct KParams {
   unsigned int* status;
 };
 
+constexpr int cmin(int a, int b) { return a < b ? a : b; }
+
 template <int BN>
 struct Cfg {
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = cmin(8, (184 * 1024) / STAGE_BYTES);
   static constexpr int ACC_STRIDE = BN <= 128 ? 128 : 256;
   static constexpr int TMEM_COLS = 2 * ACC_STRIDE;
+  static constexpr int HALF = BN / 2;                    // columns per epilogue thread
+  static constexpr int CH = (HALF % 56 == 0) ? 56 : cmin(HALF, 32);  // columns per chunk
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
-  static constexpr int STATS_OFF = BAR_OFF + 256;
+  static constexpr int CONST_OFF = BAR_OFF + 256;        // colsum[BN], colconst[BN] (fp32)
+  static constexpr int STATS_OFF = CONST_OFF + 2 * BN * 4;
   static constexpr int SMEM_BYTES = STATS_OFF + 2 * 128 * 8 + 1024;
   static_assert(B_BYTES % 1024 == 0, "W tile must keep 1024-byte alignment");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128");
+  static_assert(HALF % CH == 0 && CH % 8 == 0, "epilogue chunking");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
+// Every lane observes the barrier phase itself (so each has acquired the producer's
+// writes), then the warp agrees on the outcome so that it stays converged for the
+// .sync.aligned tcgen05 instructions that follow.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint64_t limit,
                                           unsigned int* status, volatile int* abort_flag) {
-  int ok = 1;
-  if ((threadIdx.x & 31) == 0) {
-    ok = mbar_wait(bar, parity, limit, status, abort_flag) ? 1 : 0;
-    if (!ok) *abort_flag = 1;
-  }
-  ok = __shfl_sync(0xffffffffu, ok, 0);
-  __syncwarp();  // order lane 0's acquire before the other lanes' reads
+  int ok = mbar_wait(bar, parity, limit, status, abort_flag) ? 1 : 0;
+  ok = __all_sync(0xffffffffu, ok);
+  if (!ok) *abort_flag = 1;
   return ok != 0;
 }
 
-__device__ __forceinline__ uint4 add_bf16x8(uint4 a, uint4 b) {
-  uint4 o;
-  o.x = pack_bf16x2(bf16_lo(a.x) + bf16_lo(b.x), bf16_hi(a.x) + bf16_hi(b.x));
-  o.y = pack_bf16x2(bf16_lo(a.y) + bf16_lo(b.y), bf16_hi(a.y) + bf16_hi(b.y));
-  o.z = pack_bf16x2(bf16_lo(a.z) + bf16_lo(b.z), bf16_hi(a.z) + bf16_hi(b.z));
-  o.w = pack_bf16x2(bf16_lo(a.w) + bf16_lo(b.w), bf16_hi(a.w) + bf16_hi(b.w));
-  return o;
-}
-
-// Epilogue of one 128 x BN tile for one thread (= one TMEM lane = one tile row).
-template <int BN, int EPI, bool FOLD, bool POOLED>
-__device__ __forceinline__ void epilogue_tile(const KParams& p, uint32_t tbase, int mt, int nt,
-                                              int rt, float mean, float rstd) {
-  const int n0 = nt * BN;
-  long long m;
-  int b = 0, tok = 0, np = 0;
-  if (POOLED) {
-    const int per = p.tokens >> 2;
-    const int pm = mt * 32 + (rt >> 2);
-    b = pm / per;
-    np = pm - b * per;
-    tok = (rt & 3) * per + np;
-    m = (long long)b * p.tokens + tok;
+// CH consecutive accumulator columns of this thread's TMEM lane, one wait.
+template <int CH>
+__device__ __forceinline__ void tmem_load(uint32_t taddr, uint32_t (&r)[CH]) {
+  if constexpr (CH == 56) {
+    tc_ld_32x32b_x32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+    tc_ld_32x32b_x16(taddr + 32, *reinterpret_cast<uint32_t(*)[16]>(&r[32]));
+    tc_ld_32x32b_x8(taddr + 48, *reinterpret_cast<uint32_t(*)[8]>(&r[48]));
+  } else if constexpr (CH == 32) {
+    tc_ld_32x32b_x32(taddr, r);
+  } else if constexpr (CH == 16) {
+    tc_ld_32x32b_x16(taddr, r);
   } else {
-    m = (long long)mt * BM + rt;
-    if (EPI == EPI_QKV) {
-      b = (int)(m / p.tokens);
-      tok = (int)(m - (long long)b * p.tokens);
-    }
+    static_assert(CH == 8, "chunk");
+    tc_ld_32x32b_x8(taddr, r);
   }
-  const bool row_ok = m < p.M;
-  const int which = (EPI == EPI_QKV) ? n0 / p.d_out : 0;
-  const bool pool_this = POOLED && (which == 0 || which == 3);
-  const bool writer = row_ok && (!pool_this || (rt & 3) == 0);
-  const int colw0 = (EPI == EPI_QKV) ? n0 - which * p.d_out : 0;
+  tc_wait_ld();
+  // tcgen05.ld fills its registers asynchronously; only after tcgen05.wait::ld are they
+  // valid. Re-define each one after the wait so no use can be scheduled above it.
+#pragma unroll
+  for (int i = 0; i < CH; ++i) asm volatile("" : "+r"(r[i]));
+}
 
-#pragma unroll 1
-  for (int c0 = 0; c0 < BN; c0 += 16) {
-    uint32_t r[16];
-    tc_ld_32x32b_x16(tbase + (uint32_t)c0, r);
-    tc_wait_ld();
-    float v[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int n = n0 + c0 + i;
-      const float acc = __uint_as_float(r[i]);
-      const float cc = p.colconst != nullptr ? __ldg(p.colconst + n)
-                       : (p.bias16 != nullptr ? __bfloat162float(p.bias16[n]) : 0.f);
-      float x;
-      if (FOLD) {
-        x = rstd * (acc - mean * __ldg(p.colsum + n)) + cc;
-      } else {
-        x = acc + cc;
-      }
-      if (EPI == EPI_GELU) x = gelu_erf(x);
-      v[i] = x;
-    }
-    if (EPI == EPI_QKV) {
-      if (pool_this) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          v[i] = fmaxf(v[i], __shfl_xor_sync(0xffffffffu, v[i], 1));
-          v[i] = fmaxf(v[i], __shfl_xor_sync(0xffffffffu, v[i], 2));
-        }
-      }
-#pragma unroll
-      for (int g = 0; g < 2; ++g) {
-        const int colw = colw0 + c0 + 8 * g;
-        uint4 pk;
-        pk.x = pack_bf16x2(v[8 * g + 0], v[8 * g + 1]);
-        pk.y = pack_bf16x2(v[8 * g + 2], v[8 * g + 3]);
-        pk.z = pack_bf16x2(v[8 * g + 4], v[8 * g + 5]);
-        pk.w = pack_bf16x2(v[8 * g + 6], v[8 * g + 7]);
-        if (!writer) continue;
-        bf16* dst;
-        if (which == 3) {
-          const int nq = POOLED ? (p.tokens >> 2) : p.tokens;
-          const int tq = POOLED ? np : tok;
-          dst = p.r + ((long long)b * nq + tq) * p.d_out + colw;
-        } else {
-          const int h = colw / 56, e = colw - h * 56;
-          const int tt = pool_this ? np : tok;
-          const int w = tt % p.nW, j = tt / p.nW;
-          const int T = which == 0 ? p.Tq : p.Tkv;
-          bf16* base = which == 0 ? p.q : (which == 1 ? p.k : p.v);
-          dst = base + ((((long long)b * p.nW + w) * p.heads + h) * T + j) * 64 + e;
-        }
-        *reinterpret_cast<uint4*>(dst) = pk;
-      }
-    } else {
-#pragma unroll
-      for (int g = 0; g < 2; ++g) {
-        uint4 pk;
-        pk.x = pack_bf16x2(v[8 * g + 0], v[8 * g + 1]);
-        pk.y = pack_bf16x2(v[8 * g + 2], v[8 * g + 3]);
-        pk.z = pack_bf16x2(v[8 * g + 4], v[8 * g + 5]);
-        pk.w = pack_bf16x2(v[8 * g + 6], v[8 * g + 7]);
-        if (!row_ok) continue;
-        const long long off = m * p.ldo + n0 + c0 + 8 * g;
-        if (p.residual != nullptr) {
-          // residual added in fp32 before the single rounding to bf16
-          const uint4 rr = __ldg(reinterpret_cast<const uint4*>(p.residual + off));
-          pk.x = pack_bf16x2(v[8 * g + 0] + bf16_lo(rr.x), v[8 * g + 1] + bf16_hi(rr.x));
-          pk.y = pack_bf16x2(v[8 * g + 2] + bf16_lo(rr.y), v[8 * g + 3] + bf16_hi(rr.y));
-          pk.z = pack_bf16x2(v[8 * g + 4] + bf16_lo(rr.z), v[8 * g + 5] + bf16_hi(rr.z));
-          pk.w = pack_bf16x2(v[8 * g + 6] + bf16_lo(rr.w), v[8 * g + 7] + bf16_hi(rr.w));
-        }
-        *reinterpret_cast<uint4*>(p.out + off) = pk;
-      }
-    }
-  }
-  // channels 56..63 of every q/k/v head row written above are zero padding
-  if (EPI == EPI_QKV && which != 3 && writer) {
-    const int tt = pool_this ? np : tok;
-    const int w = tt % p.nW, j = tt / p.nW;
-    const int T = which == 0 ? p.Tq : p.Tkv;
-    bf16* base = which == 0 ? p.q : (which == 1 ? p.k : p.v);
-    for (int h = colw0 / 56; h < (colw0 + BN) / 56; ++h) {
-      bf16* dst = base + ((((long long)b * p.nW + w) * p.heads + h) * T + j) * 64 + 56;
-      *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
-    }
-  }
+__device__ __forceinline__ uint4 pack8(const float* v) {
+  uint4 pk;
+  pk.x = pack_bf16x2(v[0], v[1]);
+  pk.y = pack_bf16x2(v[2], v[3]);
+  pk.z = pack_bf16x2(v[4], v[5]);
+  pk.w = pack_bf16x2(v[6], v[7]);
+  return pk;
+}
+
+__device__ __forceinline__ uint4 pack8_add(const float* v, uint4 rr) {
+  uint4 pk;
+  pk.x = pack_bf16x2(v[0] + bf16_lo(rr.x), v[1] + bf16_hi(rr.x));
+  pk.y = pack_bf16x2(v[2] + bf16_lo(rr.y), v[3] + bf16_hi(rr.y));
+  pk.z = pack_bf16x2(v[4] + bf16_lo(rr.z), v[5] + bf16_hi(rr.z));
+  pk.w = pack_bf16x2(v[6] + bf16_lo(rr.w), v[7] + bf16_hi(rr.w));
+  return pk;
 }
 
 template <int BN, int EPI, bool FOLD, bool POOLED>
-__global__ void __launch_bounds__(FOLD ? 320 : 192, 1)
+__global__ void __launch_bounds__(FOLD ? 448 : 320, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const KParams p) {
   using C = Cfg<BN>;
+  constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t* smem = smem_raw + pad;
@@ -220,6 +145,8 @@ __global__ void __launch_bounds__(FOLD ? 320 : 192, 1)
   uint64_t* drain = st_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* col_sum = reinterpret_cast<float*>(smem + C::CONST_OFF);
+  float* col_const = col_sum + BN;
   float2* stats = reinterpret_cast<float2*>(smem + C::STATS_OFF);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -235,9 +162,9 @@ __global__ void __launch_bounds__(FOLD ? 320 : 192, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 128);
+      mbar_init(&acc_empty[a], EPI_THREADS);
       mbar_init(&st_full[a], 128);
-      mbar_init(&st_empty[a], 128);
+      mbar_init(&st_empty[a], EPI_THREADS);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -346,26 +273,129 @@ __global__ void __launch_bounds__(FOLD ? 320 : 192, 1)
       tc_commit(drain);
       mbar_wait(drain, 0, p.limit_ns, p.status);
     }
-  } else if (warp < 6) {
+  } else if (warp < 2 + EPI_WARPS) {
     // ------------------------------------------------------------ epilogue
-    const int quarter = warp & 3;
-    const int rt = quarter * 32 + lane;
+    constexpr int HALF = C::HALF, CH = C::CH;
+    const int ew = warp - 2;
+    const int quarter = warp & 3;          // TMEM lanes 32*quarter .. +31
+    const int c_begin = (ew >> 2) * HALF;  // this warp's half of the tile's columns
+    const int rt = quarter * 32 + lane;    // tile row == TMEM lane
+    const int etid = ew * 32 + lane;
     int acc = 0;
     uint32_t aph = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       const int mt = tile / n_tiles, nt = tile - (tile / n_tiles) * n_tiles;
+      const int n0 = nt * BN;
+      // row bookkeeping
+      long long m;
+      int b = 0, tok = 0, np = 0;
+      if (POOLED) {
+        const int per = p.tokens >> 2;
+        const int pm = mt * 32 + (rt >> 2);
+        b = pm / per;
+        np = pm - b * per;
+        tok = (rt & 3) * per + np;
+        m = (long long)b * p.tokens + tok;
+      } else {
+        m = (long long)mt * BM + rt;
+        if (EPI == EPI_QKV) {
+          b = (int)(m / p.tokens);
+          tok = (int)(m - (long long)b * p.tokens);
+        }
+      }
+      const bool row_ok = m < p.M;
+      // residual of this row / half, in flight while the mainloop runs
+      constexpr int NV = (EPI == EPI_STORE) ? HALF / 8 : 1;
+      uint4 res[NV];
+      const bool has_res = (EPI == EPI_STORE) && p.residual != nullptr && row_ok;
+      if (EPI == EPI_STORE) {
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+          res[i] = has_res ? __ldg(reinterpret_cast<const uint4*>(
+                                 p.residual + m * p.ldo + n0 + c_begin + 8 * i))
+                           : make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      // per-column constants of this tile into shared memory
+      named_bar_sync(1, EPI_THREADS);  // every epilogue thread is done with the last tile's
+      for (int i = etid; i < BN; i += EPI_THREADS) {
+        col_sum[i] = FOLD ? __ldg(p.colsum + n0 + i) : 0.f;
+        col_const[i] = p.colconst != nullptr ? __ldg(p.colconst + n0 + i)
+                       : (p.bias16 != nullptr ? __bfloat162float(p.bias16[n0 + i]) : 0.f);
+      }
+      named_bar_sync(1, EPI_THREADS);
       if (!warp_wait(&acc_full[acc], aph, p.limit_ns, p.status, abort_flag)) break;
-      float mean = 0.f, rstd = 1.f;
+      float fa = 1.f, fb = 0.f;  // v = fa * acc + fb * colsum + colconst
       if (FOLD) {
         if (!warp_wait(&st_full[acc], aph, p.limit_ns, p.status, abort_flag)) break;
         const float2 st = stats[acc * 128 + rt];
-        mean = st.x;
-        rstd = st.y;
         mbar_arrive(&st_empty[acc]);
+        fa = st.y;
+        fb = -st.x * st.y;
       }
       tc_fence_after();
-      const uint32_t tbase = tmem + (uint32_t)(acc * C::ACC_STRIDE) + ((uint32_t)(quarter * 32) << 16);
-      epilogue_tile<BN, EPI, FOLD, POOLED>(p, tbase, mt, nt, rt, mean, rstd);
+      const uint32_t tbase = tmem + (uint32_t)(acc * C::ACC_STRIDE) +
+                             ((uint32_t)(quarter * 32) << 16) + (uint32_t)c_begin;
+      const int which = (EPI == EPI_QKV) ? n0 / p.d_out : 0;
+      const bool pool_this = POOLED && (which == 0 || which == 3);
+      const bool writer = row_ok && (!pool_this || (rt & 3) == 0);
+#pragma unroll
+      for (int c = 0; c < HALF; c += CH) {
+        uint32_t r[CH];
+        tmem_load<CH>(tbase + (uint32_t)c, r);
+        float v[CH];
+#pragma unroll
+        for (int i = 0; i < CH; ++i) {
+          const int cl = c_begin + c + i;
+          float x = FOLD ? fmaf(fa, __uint_as_float(r[i]), fmaf(fb, col_sum[cl], col_const[cl]))
+                         : __uint_as_float(r[i]) + col_const[cl];
+          if (EPI == EPI_GELU) x = gelu_fast(x);
+          v[i] = x;
+        }
+        if (EPI == EPI_QKV) {
+          static_assert(EPI != EPI_QKV || CH == 56, "q/k/v chunks are whole heads");
+          if (pool_this) {
+#pragma unroll
+            for (int i = 0; i < CH; ++i) {
+              v[i] = fmaxf(v[i], __shfl_xor_sync(0xffffffffu, v[i], 1));
+              v[i] = fmaxf(v[i], __shfl_xor_sync(0xffffffffu, v[i], 2));
+            }
+          }
+          if (writer) {
+            const int colw = n0 - which * p.d_out + c_begin + c;  // multiple of 56
+            if (which == 3) {
+              const int nq = POOLED ? (p.tokens >> 2) : p.tokens;
+              const int tq = POOLED ? np : tok;
+              bf16* dst = p.r + ((long long)b * nq + tq) * p.d_out + colw;
+#pragma unroll
+              for (int g = 0; g < CH / 8; ++g)
+                *reinterpret_cast<uint4*>(dst + 8 * g) = pack8(&v[8 * g]);
+            } else {
+              const int h = colw / 56;
+              const int tt = pool_this ? np : tok;
+              const int w = tt % p.nW, j = tt / p.nW;
+              const int T = which == 0 ? p.Tq : p.Tkv;
+              bf16* base = which == 0 ? p.q : (which == 1 ? p.k : p.v);
+              bf16* dst = base + ((((long long)b * p.nW + w) * p.heads + h) * T + j) * 64;
+#pragma unroll
+              for (int g = 0; g < 7; ++g)
+                *reinterpret_cast<uint4*>(dst + 8 * g) = pack8(&v[8 * g]);
+              *reinterpret_cast<uint4*>(dst + 56) = make_uint4(0u, 0u, 0u, 0u);
+            }
+          }
+        } else if (row_ok) {
+          bf16* dst = p.out + m * p.ldo + n0 + c_begin + c;
+#pragma unroll
+          for (int g = 0; g < CH / 8; ++g) {
+            uint4 pk;
+            if (EPI == EPI_STORE && has_res)
+              pk = pack8_add(&v[8 * g], res[(c / 8 + g) < NV ? (c / 8 + g) : 0]);
+            else
+              pk = pack8(&v[8 * g]);
+            *reinterpret_cast<uint4*>(dst + 8 * g) = pk;
+          }
+        }
+      }
       tc_fence_before();
       mbar_arrive(&acc_empty[acc]);
       if (++acc == 2) {
@@ -375,7 +405,7 @@ __global__ void __launch_bounds__(FOLD ? 320 : 192, 1)
     }
   } else if (FOLD) {
     // ------------------------------------------------------------ LayerNorm row statistics
-    const int t = (warp - 6) * 32 + lane;
+    const int t = (warp - 2 - EPI_WARPS) * 32 + lane;
     int s = 0, acc = 0;
     uint32_t ph = 0, aph = 0;
     bool ok = true;
@@ -392,7 +422,6 @@ __global__ void __launch_bounds__(FOLD ? 320 : 192, 1)
         uint4 ch[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) ch[c] = row[c];
-        mbar_arrive(&empty[s]);
         const int kvalid = min(BK, p.K - kb * BK);
         // physical 16-byte chunk c of this 128-byte row holds logical chunk c ^ (row & 7)
         float sum = 0.f;
@@ -414,11 +443,17 @@ __global__ void __launch_bounds__(FOLD ? 320 : 192, 1)
           const uint32_t wv[4] = {ch[c].x, ch[c].y, ch[c].z, ch[c].w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            float d0 = bf16_lo(wv[e]) - bmean, d1 = bf16_hi(wv[e]) - bmean;
+            const float d0 = bf16_lo(wv[e]) - bmean, d1 = bf16_hi(wv[e]) - bmean;
             if (k0 + 2 * e < kvalid) bm2 += d0 * d0;
             if (k0 + 2 * e + 1 < kvalid) bm2 += d1 * d1;
           }
         }
+        // The stage may be refilled by TMA (async proxy) as soon as every consumer has
+        // arrived: consume the loaded values first, order these generic-proxy reads before
+        // the async-proxy writes that follow the release, then arrive.
+        asm volatile("" ::"f"(bmean), "f"(bm2) : "memory");
+        fence_proxy_async_smem();
+        mbar_arrive(&empty[s]);
         // Chan et al. pairwise update of (count, mean, M2)
         const int tot = cnt + kvalid;
         const float delta = bmean - mean;
@@ -546,7 +581,7 @@ hiera_status run(const TcGemmArgs& a, cudaStream_t stream) {
   if (grid > tiles) grid = tiles;
   profile_mark(EPI == EPI_QKV ? K_GEMM_QKV : (EPI == EPI_GELU ? K_GEMM_GELU : K_GEMM_STORE),
                stream);
-  kern<<<grid, FOLD ? 320 : 192, C::SMEM_BYTES, stream>>>(tmA, tmB, p);
+  kern<<<grid, FOLD ? 448 : 320, C::SMEM_BYTES, stream>>>(tmA, tmB, p);
   return cudaGetLastError() == cudaSuccess ? HIERA_OK : HIERA_ERR_CUDA;
 }
 

@@ -69,6 +69,7 @@ __global__ void __launch_bounds__(256) copy_pack_kernel(const T* __restrict__ w,
   const long long stride = (long long)gridDim.x * blockDim.x;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < NK; i += stride)
     w_out[i] = w[i];
+  if (bias_out == nullptr) return;  // plain copy (no bias vector to convert)
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < N; i += stride)
     bias_out[i] = bias != nullptr ? ld(bias, i) : 0.f;
 }

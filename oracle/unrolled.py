@@ -251,3 +251,49 @@ def backbone_forward(img_nhwc, params, mask_unit_attn_override=None):
             Gs = G >> s
             feats.append(reroll(x, Gs, UNROLL_LEVELS - s))
     return feats
+
+
+def block_forward_rows(x, p, heads, q_stride, window_tokens, mask_unit_attn, rows,
+                       eps=LN_EPS, head_dim=HEAD_DIM):
+    """Output of block_forward for selected output tokens only (for sizes where the full
+    attention matrix is too large for the host). `rows` is a list of (b, n_out) pairs with
+    n_out indexing the block's output tokens. Same definition as block_forward, evaluated
+    one query row at a time: keys and values of the query's window are projected for the
+    whole window, the query is max-pooled over the q_stride outermost chunks of the
+    window, softmax runs over that window's keys."""
+    x = _f64(x)
+    B, N, dim_in = x.shape
+    d_out = p["attn_proj_w"].shape[0]
+    nW = N // window_tokens if mask_unit_attn else 1
+    T = N // nW
+    Tq = T // q_stride
+    out = np.empty((len(rows), d_out))
+    cache = {}
+    for r, (b, n_out) in enumerate(rows):
+        w, jq = n_out % nW, n_out // nW
+        key = (b, w)
+        if key not in cache:
+            toks = np.arange(T) * nW + w                       # window members, j = 0..T-1
+            xn = layer_norm(x[b, toks], p["norm1_w"], p["norm1_b"], eps)
+            qkv = linear(xn, p["qkv_w"], p["qkv_b"]).reshape(T, 3, heads, head_dim)
+            resid = None
+            if dim_in != d_out:
+                resid = linear(xn, p["proj_w"], p["proj_b"])  # [T, d_out]
+            cache = {key: (qkv, resid, toks)}
+        qkv, resid, toks = cache[key]
+        members = [c * Tq + jq for c in range(q_stride)]      # in-window indices pooled
+        q = qkv[members, 0].max(axis=0)                       # [heads, hd]
+        k, v = qkv[:, 1], qkv[:, 2]                            # [T, heads, hd]
+        o = np.empty((heads, head_dim))
+        for h in range(heads):
+            s = (k[:, h] @ q[h]) / math.sqrt(head_dim)
+            o[h] = softmax_rows(s[None])[0] @ v[:, h]
+        a = linear(o.reshape(1, d_out), p["attn_proj_w"], p["attn_proj_b"])[0]
+        if dim_in != d_out:
+            res = resid[members].max(axis=0)
+        else:
+            res = x[b, toks[jq]]
+        x1 = res + a
+        h2 = layer_norm(x1[None], p["norm2_w"], p["norm2_b"], eps)
+        out[r] = x1 + mlp(h2, p["fc1_w"], p["fc1_b"], p["fc2_w"], p["fc2_b"])[0]
+    return out

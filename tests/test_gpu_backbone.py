@@ -1,0 +1,159 @@
+"""Hiera-B+ backbone through the C ABI against the fp64 oracle.
+
+bf16 mode: rel-L2 <= 3e-2 per feature after the full backbone; fp32 mode: max-abs
+<= 1e-4 relative to the feature scale. At 2048^2 the oracle cannot evaluate the global
+stages; mask-unit-local stages 0-1 are checked exactly on sampled mask units (each one's
+receptive field is its own 32x32-pixel patch plus the 3-pixel convolution halo).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from mask_unit_windowed_b200 import binding as hb
+from mask_unit_windowed_b200 import synthetic as syn
+from oracle import unrolled as U
+
+from helpers import TORCH_DT, dev, host, max_abs, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+BF16_REL_L2 = 3e-2
+
+
+def weights_dev(p, dtype):
+    return {"patch_w": dev(p["patch_w"], dtype), "patch_b": dev(p["patch_b"], dtype),
+            "pos_embed": dev(p["pos_embed"], dtype),
+            "blocks": [{k: dev(v, dtype) for k, v in b.items()} for b in p["blocks"]]}
+
+
+def run_backbone(img, B, dtype, seed, affine, lagged=False):
+    p = syn.backbone_params(seed, img, dtype=dtype, affine=affine)
+    x = syn.image(seed, B, img, dtype=dtype)
+    desc = hb.BackboneDesc(B=B, img=img, dtype=TORCH_DT[dtype],
+                           mask_unit_attn_stage2_first=lagged)
+    packed = hb.backbone_pack(desc, weights_dev(p, dtype))
+    feats = hb.backbone_forward(desc, packed, dev(x, dtype))
+    assert hb.device_status() == 0
+    return [host(f) for f in feats], p, x, desc, packed
+
+
+@pytest.mark.parametrize("img,B", [(64, 2), (128, 1)])
+def test_backbone_bf16_small(img, B):
+    feats, p, x, *_ = run_backbone(img, B, "bf16", 31, "random")
+    ref = U.backbone_forward(x, p)
+    for s, (f, r) in enumerate(zip(feats, ref)):
+        assert f.shape == r.shape
+        assert rel_l2(f, r) <= BF16_REL_L2, (s, rel_l2(f, r))
+
+
+def test_backbone_bf16_lagged_mask_unit_flag():
+    feats, p, x, *_ = run_backbone(64, 2, "bf16", 32, "random", lagged=True)
+    flags = [True] * 6 + [False] * 18
+    ref = U.backbone_forward(x, p, mask_unit_attn_override=flags)
+    for s, (f, r) in enumerate(zip(feats, ref)):
+        assert rel_l2(f, r) <= BF16_REL_L2, (s, rel_l2(f, r))
+
+
+def test_backbone_f32_small():
+    feats, p, x, *_ = run_backbone(64, 1, "f32", 33, "random")
+    ref = U.backbone_forward(x, p)
+    for s, (f, r) in enumerate(zip(feats, ref)):
+        assert max_abs(f, r) <= 1e-4 * max(1.0, np.abs(r).max()), (s, max_abs(f, r))
+
+
+def test_cfg4_backbone_512_bf16():
+    """Full Hiera-B+ at 512x512x4 ~ U(-1,1), bf16, batch 1: features 128^2x112, 64^2x224,
+    32^2x448, 16^2x896 against the oracle."""
+    feats, p, x, desc, packed = run_backbone(512, 1, "bf16", 3, "init")
+    ref = U.backbone_forward(x, p)
+    shapes = [(1, 128, 128, 112), (1, 64, 64, 224), (1, 32, 32, 448), (1, 16, 16, 896)]
+    for s, (f, r) in enumerate(zip(feats, ref)):
+        assert f.shape == shapes[s]
+        assert rel_l2(f, r) <= BF16_REL_L2, (s, rel_l2(f, r))
+
+
+def test_batch_rows_independent_bitwise():
+    """Image i of a batch of 8 gives bit-identical features to the same image alone."""
+    p = syn.backbone_params(3, 512, dtype="bf16")
+    x = syn.image(3, 8, 512)
+    w = weights_dev(p, "bf16")
+    d8 = hb.BackboneDesc(B=8, img=512)
+    d1 = hb.BackboneDesc(B=1, img=512)
+    f8 = hb.backbone_forward(d8, hb.backbone_pack(d8, w), dev(x))
+    for i in (0, 5):
+        f1 = hb.backbone_forward(d1, hb.backbone_pack(d1, w), dev(x[i:i + 1]))
+        for s, (a, b) in enumerate(zip(f8, f1)):
+            diff = (a[i:i + 1].float() - b.float()).abs().max().item()
+            assert torch.equal(a[i:i + 1], b), (i, s, diff)
+
+
+def _oracle_mask_unit_stages01(x_img, p, my, mx, G0):
+    """Stages 0-1 of one mask unit (8x8 stage-0 tokens) from its padded pixel patch."""
+    img = x_img.shape[1]
+    pad = np.zeros((1, img + 6, img + 6, 4))
+    pad[:, 3:3 + img, 3:3 + img] = x_img
+    crop = pad[:, 32 * my:32 * my + 38, 32 * mx:32 * mx + 38]       # halo included
+    tok = U.patch_embed(crop, p["patch_w"], p["patch_b"], pad=0)    # [1, 64, 112] raster 8x8
+    ys, xs = np.meshgrid(np.arange(8) + 8 * my, np.arange(8) + 8 * mx, indexing="ij")
+    tok = tok + np.asarray(p["pos_embed"], np.float64)[(ys * G0 + xs).reshape(-1)][None]
+    t = U.unroll(tok, 8, 3)
+    sched = U.block_schedule()
+    feats = []
+    for i in range(5):
+        c = sched[i]
+        window = (64 >> (2 * c["stage"])) * c["q_stride"]
+        t = U.block_forward(t, p["blocks"][i], c["heads"], c["q_stride"], window, True)
+        if i == 1:
+            feats.append(U.reroll(t, 8, 3)[0])
+        if i == 4:
+            feats.append(U.reroll(t, 4, 2)[0])
+    return feats
+
+
+def test_cfg5_backbone_2048_sampled_mask_units():
+    """Hiera-B+ at 2048x2048x4, bf16, batch 1 (262144 stage-0 tokens, 4096 mask units,
+    global attention over 16384 tokens in stage 2): stage 0 and 1 features of sampled
+    mask units against the oracle; stage 2 and 3 features finite."""
+    feats, p, x, *_ = run_backbone(2048, 1, "bf16", 4, "init")
+    G0 = 512
+    x64 = np.asarray(x, np.float64)
+    for my, mx in [(0, 0), (63, 63), (0, 63), (17, 41), (40, 3)]:
+        f0, f1 = _oracle_mask_unit_stages01(x64, p, my, mx, G0)
+        g0 = feats[0][0, 8 * my:8 * my + 8, 8 * mx:8 * mx + 8]
+        g1 = feats[1][0, 4 * my:4 * my + 4, 4 * mx:4 * mx + 4]
+        assert rel_l2(g0, f0) <= BF16_REL_L2, rel_l2(g0, f0)
+        assert rel_l2(g1, f1) <= BF16_REL_L2, rel_l2(g1, f1)
+    assert np.isfinite(feats[2]).all() and np.isfinite(feats[3]).all()
+    assert feats[2].shape == (1, 128, 128, 448) and feats[3].shape == (1, 64, 64, 896)
+
+
+def test_global_block_16384_tokens_sampled_rows():
+    """A stage-2 global block at the 2048^2 token count (16384 tokens, 8 heads, bf16):
+    sampled output rows against the oracle evaluated one query row at a time."""
+    B, N, d = 1, 16384, 448
+    p = syn.block_params(41, d, d, False, dtype="bf16", affine="random")
+    x = syn.activations(41, (B, N, d), dtype="bf16")
+    desc = hb.BlockDesc(B=B, tokens=N, dim_in=d, dim_out=d, heads=8, mask_unit_attn=False)
+    y = host(hb.block_forward(desc, hb.block_pack(desc, {k: dev(v) for k, v in p.items()}),
+                              dev(x)))
+    rows = [(0, n) for n in np.random.default_rng(0).choice(N, 24, replace=False)]
+    ref = U.block_forward_rows(x, p, 8, 1, 1, False, rows)
+    got = np.stack([y[b, n] for b, n in rows])
+    assert rel_l2(got, ref) <= 1e-2
+
+
+def test_transition_block_65536_tokens_sampled_rows():
+    """Block 5 at 2048^2: 65536 stage-1 tokens (224) -> 16384 (448), pooled queries,
+    global attention over 65536 keys; sampled rows against the per-row oracle."""
+    B, N = 1, 65536
+    p = syn.block_params(42, 224, 448, True, dtype="bf16", affine="random")
+    x = syn.activations(42, (B, N, 224), dtype="bf16")
+    desc = hb.BlockDesc(B=B, tokens=N, dim_in=224, dim_out=448, heads=8, q_stride=4,
+                        window_tokens=16, mask_unit_attn=False)
+    y = host(hb.block_forward(desc, hb.block_pack(desc, {k: dev(v) for k, v in p.items()}),
+                              dev(x)))
+    rows = [(0, n) for n in np.random.default_rng(1).choice(N // 4, 12, replace=False)]
+    ref = U.block_forward_rows(x, p, 8, 4, 16, False, rows)
+    got = np.stack([y[b, n] for b, n in rows])
+    assert rel_l2(got, ref) <= 1e-2

@@ -124,3 +124,54 @@ def test_repeat_is_deterministic_bf16():
     y1, _, desc, packed, p, x = run_case(*args, dtype="bf16", seed=8, affine="random")
     y2 = host(hb.block_forward(desc, packed, dev(x)))
     np.testing.assert_array_equal(y1, y2)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_block_batch_independent_bitwise(name):
+    """Image 0 of a batch gives bit-identical output to the same image alone."""
+    B, tokens, d_in, d_out, heads, qs, window, mua = CASES[name]
+    p = syn.block_params(9, d_in, d_out, d_in != d_out, dtype="bf16", affine="random")
+    x = syn.activations(9, (B, tokens, d_in), dtype="bf16")
+    w = block_weights_dev(p, "bf16")
+    dB = hb.BlockDesc(B=B, tokens=tokens, dim_in=d_in, dim_out=d_out, heads=heads,
+                      q_stride=qs, window_tokens=window, mask_unit_attn=mua)
+    d1 = hb.BlockDesc(B=1, tokens=tokens, dim_in=d_in, dim_out=d_out, heads=heads,
+                      q_stride=qs, window_tokens=window, mask_unit_attn=mua)
+    yB = hb.block_forward(dB, hb.block_pack(dB, w), dev(x))
+    y1 = hb.block_forward(d1, hb.block_pack(d1, w), dev(x[:1]))
+    diff = (yB[:1].float() - y1.float()).abs().max().item()
+    assert torch.equal(yB[:1], y1), diff
+
+
+@pytest.mark.parametrize("name", ["global_ragged", "stage3_global", "stage1_transition",
+                                  "stage0_windowed"])
+def test_block_intermediates_deterministic(name):
+    """Race check: five forwards of the same block into workspaces pre-filled with
+    different garbage give bit-identical q/k/v, attention output, residual, x1, MLP hidden
+    and y."""
+    B, tokens, d_in, d_out, heads, qs, window, mua = CASES[name]
+    p = syn.block_params(10, d_in, d_out, d_in != d_out, dtype="bf16", affine="random")
+    x = dev(syn.activations(10, (B, tokens, d_in), dtype="bf16"))
+    desc = hb.BlockDesc(B=B, tokens=tokens, dim_in=d_in, dim_out=d_out, heads=heads,
+                        q_stride=qs, window_tokens=window, mask_unit_attn=mua)
+    packed = hb.block_pack(desc, block_weights_dev(p, "bf16"))
+    offs = hb.block_workspace_layout(desc)
+    nW = tokens // window if mua else 1
+    Tkv = tokens // nW
+    Tq, Nq = Tkv // qs, tokens // qs
+    sizes = [B * nW * heads * Tq * 64 * 2, B * nW * heads * Tkv * 64 * 2,
+             B * nW * heads * Tkv * 64 * 2, B * Nq * d_out * 2, B * Nq * d_out * 2,
+             B * Nq * d_out * 2, B * Nq * 4 * d_out * 2]
+    nbytes = hb.block_workspace_bytes(desc)
+    ref = None
+    for rep in range(5):
+        ws = torch.full((nbytes,), (rep * 53 + 7) % 256, dtype=torch.uint8, device="cuda")
+        y = hb.block_forward(desc, packed, x, workspace=ws)
+        torch.cuda.synchronize()
+        parts = [ws[o:o + n].clone() for o, n in zip(offs, sizes) if o >= 0] + [y.clone()]
+        if ref is None:
+            ref = parts
+        else:
+            for i, (a, b) in enumerate(zip(parts, ref)):
+                assert torch.equal(a, b), f"buffer {i} differs in repeat {rep}"
+    assert hb.device_status() == 0

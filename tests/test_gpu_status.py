@@ -28,3 +28,15 @@ def test_workspace_too_small_rejected():
     with pytest.raises(hb.HieraError) as e:
         hb.block_forward(desc, packed, x, workspace=ws)
     assert e.value.code == 5
+
+
+def test_tensor_core_path_gelu_within_error_bound():
+    """The fc1 epilogue's GELU (erf by Abramowitz & Stegun 7.1.28, |erf error| <= 3e-7)
+    against the fp64 definition x * Phi(x)."""
+    import numpy as np
+    from oracle import unrolled as U
+    x = np.linspace(-12, 12, 200001).astype(np.float32)
+    y = hb.debug_gelu(torch.from_numpy(x).cuda()).cpu().numpy().astype(np.float64)
+    ref = U.gelu(x.astype(np.float64))
+    err = np.abs(y - ref)
+    assert np.all(err <= 1e-6 + 1e-6 * np.abs(x)), float(err.max())

@@ -352,3 +352,18 @@ def test_in_window_permutation_equivariance():
     np.testing.assert_allclose(y2, y[:, perm], rtol=1e-12, atol=1e-12)
     # and a token of another window is unaffected by that permutation
     np.testing.assert_allclose(y2[:, 0], y[:, 0], rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("case", [
+    (2, 64, 8, 8, 2, 1, 16, True), (2, 64, 6, 8, 2, 4, 16, True), (1, 64, 8, 8, 2, 1, 64, False),
+    (2, 64, 6, 8, 2, 4, 64, False)])
+def test_block_rows_matches_full_block(case):
+    """The per-row evaluation used for large sampled checks equals the full block."""
+    B, N, d_in, d_out, heads, qs, window, mua = case
+    p = _tiny_block(14, d_in, d_out, d_in != d_out)
+    x = np.random.default_rng(15).standard_normal((B, N, d_in))
+    full = U.block_forward(x, p, heads, qs, window, mua, head_dim=4)
+    rows = [(b, n) for b in range(B) for n in range(0, N // qs, 3)]
+    part = U.block_forward_rows(x, p, heads, qs, window, mua, rows, head_dim=4)
+    for r, (b, n) in enumerate(rows):
+        np.testing.assert_allclose(part[r], full[b, n], rtol=1e-12, atol=1e-12)
