@@ -191,6 +191,34 @@ HIERA_API hiera_status hiera_block_forward(const hiera_block_desc* desc, const v
 HIERA_API hiera_status hiera_block_workspace_layout(const hiera_block_desc* desc, long long offsets[7]);
 
 /* --------------------------------------------------------------------------------
+ * Allocation-free variant of hiera_block_forward (no counterpart on the pages: it exists
+ * for callers, not for the method).
+ *
+ * Some callers cannot provide a workspace because they cannot allocate device memory at
+ * all: a plug-in running inside a host framework that owns every device allocation and
+ * hands the plug-in only its input and output buffers, or a real-time loop whose policy
+ * forbids cudaMalloc once it has started. hiera_block_forward_noalloc() computes exactly
+ * what hiera_block_forward() computes, but its intermediates live in one library-owned
+ * device array of HIERA_STATIC_SCRATCH_BYTES bytes (32 MiB), declared statically in the
+ * library: every GPU that loads the library holds that array until the process exits.
+ * The call itself allocates and frees nothing.
+ *
+ * The caller still passes the packed weights, the input x and the output y (as for
+ * hiera_block_forward). A block whose hiera_block_workspace_bytes() exceeds
+ * HIERA_STATIC_SCRATCH_BYTES is rejected with HIERA_ERR_WORKSPACE before anything runs.
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress,
+ * with that device current) and caches it; make that first call before any stream
+ * capture. All calls share the one array, which keeps the last call's contents: calls
+ * whose GPU work overlaps (different streams, or different host threads) race on it and
+ * must be serialised by the caller. Nothing in the array needs to start at zero: every
+ * byte a call reads was written earlier in the same call.
+ * -------------------------------------------------------------------------------- */
+#define HIERA_STATIC_SCRATCH_BYTES ((size_t)32 << 20)
+HIERA_API hiera_status hiera_block_forward_noalloc(const hiera_block_desc* desc,
+                                                   const void* packed, const void* x, void* y,
+                                                   hiera_stream_t stream);
+
+/* --------------------------------------------------------------------------------
  * PatchEmbed + pos_embed + Unroll ("Architecture Summary": Conv2d(4 -> 112, 7x7,
  * stride 4) reshaped to [B, N, C]; learned pos_embed (1, N, 112) added; Unroll).
  *

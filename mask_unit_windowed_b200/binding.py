@@ -100,6 +100,7 @@ def lib() -> ctypes.CDLL:
                                         ctypes.POINTER(ctypes.c_void_p), P, S, P], I),
             "hiera_debug_timeout_probe": ([I, P], I),
             "hiera_debug_gelu": ([P, P, I, P], I),
+            "hiera_block_forward_noalloc": ([ctypes.POINTER(BlockDescC), P, P, P, P], I),
             "hiera_profile_begin": ([ctypes.POINTER(ctypes.c_void_p), I,
                                      ctypes.POINTER(ctypes.c_int)], I),
             "hiera_profile_end": ([P], I),
@@ -252,6 +253,23 @@ def block_forward(desc: BlockDesc, packed: torch.Tensor, x: torch.Tensor, out=No
     _check(lib().hiera_block_forward(ctypes.byref(d), _ptr(packed), _ptr(x), _ptr(out),
                                      _ptr(workspace), workspace.numel(), _stream(stream)),
            "hiera_block_forward")
+    return out
+
+
+STATIC_SCRATCH_BYTES = 32 << 20
+
+
+def block_forward_noalloc(desc: BlockDesc, packed: torch.Tensor, x: torch.Tensor, out=None,
+                          stream=None) -> torch.Tensor:
+    """hiera_block_forward_noalloc: the block forward with the library's static scratch
+    (for callers that cannot allocate a workspace); `out` may be preallocated."""
+    _need(x, "x")
+    d = desc.c()
+    if out is None:
+        out = torch.empty((desc.B, desc.out_tokens, desc.dim_out), dtype=x.dtype,
+                          device=x.device)
+    _check(lib().hiera_block_forward_noalloc(ctypes.byref(d), _ptr(packed), _ptr(x), _ptr(out),
+                                             _stream(stream)), "hiera_block_forward_noalloc")
     return out
 
 

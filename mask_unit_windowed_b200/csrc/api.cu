@@ -474,6 +474,27 @@ BackboneWs backbone_ws_layout(const hiera_backbone_desc* bd, const BlockPlan pla
   return L;
 }
 
+// Library-owned scratch for hiera_block_forward_noalloc (see include/hiera.h): a static
+// device array, so calls through that entry point allocate nothing. Host code needs the
+// array's device address, looked up once per device with that device current.
+static __device__ __align__(256) unsigned char g_static_scratch[HIERA_STATIC_SCRATCH_BYTES];
+void* g_static_scratch_addr[kMaxDev] = {};
+std::mutex g_static_scratch_mu;
+
+hiera_status static_scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return HIERA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_static_scratch_mu);
+  if (g_static_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr)
+      return HIERA_ERR_CUDA;
+    g_static_scratch_addr[dev] = p;
+  }
+  *out = g_static_scratch_addr[dev];
+  return HIERA_OK;
+}
+
 __global__ void gelu_probe_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) y[i] = gelu_fast(x[i]);
@@ -685,6 +706,21 @@ hiera_status hiera_block_forward(const hiera_block_desc* desc, const void* packe
   const cudaStream_t st = (cudaStream_t)stream;
   return g.bf16 ? forward_bf16(g, (const uint8_t*)packed, x, y, (uint8_t*)workspace, st)
                 : forward_f32(g, (const uint8_t*)packed, x, y, (uint8_t*)workspace, st);
+}
+
+hiera_status hiera_block_forward_noalloc(const hiera_block_desc* desc, const void* packed,
+                                         const void* x, void* y, hiera_stream_t stream) {
+  Geom g;
+  HIERA_TRY(make_geom(desc, &g));
+  if (packed == nullptr || x == nullptr || y == nullptr) return HIERA_ERR_INVALID_ARG;
+  if (!aligned16(packed) || !aligned16(x) || !aligned16(y)) return HIERA_ERR_ALIGNMENT;
+  if (ws_layout(g).total > HIERA_STATIC_SCRATCH_BYTES) return HIERA_ERR_WORKSPACE;
+  HIERA_TRY(check_device());
+  void* scratch = nullptr;
+  HIERA_TRY(static_scratch_address(&scratch));
+  const cudaStream_t st = (cudaStream_t)stream;
+  return g.bf16 ? forward_bf16(g, (const uint8_t*)packed, x, y, (uint8_t*)scratch, st)
+                : forward_f32(g, (const uint8_t*)packed, x, y, (uint8_t*)scratch, st);
 }
 
 hiera_status hiera_patch_pack(const void* patch_w, const void* patch_b, void* packed,

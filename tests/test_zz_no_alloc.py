@@ -1,0 +1,60 @@
+"""The allocation-free block entry point (hiera_block_forward_noalloc).
+
+It serves callers that cannot allocate device memory (a plug-in whose host framework owns
+all device allocations, a real-time loop that forbids cudaMalloc after start-up): the
+intermediates live in the library's static scratch array instead of a caller workspace.
+Its output must match hiera_block_forward on the same inputs, on consecutive calls that
+reuse the array with the previous call's contents still in it.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from mask_unit_windowed_b200 import binding as hb
+from mask_unit_windowed_b200 import synthetic as syn
+
+pytestmark = pytest.mark.gpu
+
+
+def _case(dtype, B, tokens, d_in, d_out, heads, q_stride, window, mua, seed):
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    p = syn.block_params(seed, d_in, d_out, d_in != d_out, dtype=dtype, affine="random")
+    x = torch.from_numpy(syn.activations(seed, (B, tokens, d_in), dtype=dtype)).to("cuda", tdt)
+    desc = hb.BlockDesc(B=B, tokens=tokens, dim_in=d_in, dim_out=d_out, heads=heads,
+                        q_stride=q_stride, window_tokens=window, mask_unit_attn=mua, dtype=tdt)
+    packed = hb.block_pack(desc, {k: torch.from_numpy(v).to("cuda", tdt) for k, v in p.items()})
+    return desc, packed, x
+
+
+def _rel_l2(a, b):
+    a, b = a.double(), b.double()
+    return float((a - b).norm() / b.norm())
+
+
+@pytest.mark.parametrize("dtype,args", [
+    ("bf16", (2, 256, 112, 224, 4, 4, 64, True, 51)),     # stage-1 transition, pooled
+    ("bf16", (2, 1024, 448, 448, 8, 1, 1, False, 52)),    # stage-2 global
+    ("f32", (1, 1024, 112, 112, 2, 1, 64, True, 53)),     # stage-0 block in fp32
+])
+def test_noalloc_matches_workspace_entry_point_twice(dtype, args):
+    desc, packed, x = _case(dtype, *args)
+    assert hb.block_workspace_bytes(desc) <= hb.STATIC_SCRATCH_BYTES
+    ref = hb.block_forward(desc, packed, x)
+    for _ in range(2):   # the second call finds the first call's data in the scratch
+        y = hb.block_forward_noalloc(desc, packed, x)
+        torch.cuda.synchronize()
+        assert hb.device_status() == 0
+        if dtype == "bf16":
+            assert _rel_l2(y, ref) <= 1e-2
+        else:
+            assert float((y - ref).abs().max()) <= 1e-4
+        assert torch.equal(y, ref)
+
+
+def test_noalloc_rejects_blocks_larger_than_the_static_scratch():
+    desc, packed, x = _case("bf16", 8, 1024, 448, 448, 8, 1, 1, False, 54)
+    assert hb.block_workspace_bytes(desc) > hb.STATIC_SCRATCH_BYTES
+    with pytest.raises(hb.HieraError) as e:
+        hb.block_forward_noalloc(desc, packed, x)
+    assert e.value.code == 5   # HIERA_ERR_WORKSPACE
