@@ -158,7 +158,10 @@ WsLayout ws_layout(const Geom& g) {
     }
     L.x1 = o; o = up256(o + (size_t)qrows * g.d_out * 2);
     L.h = o; o = up256(o + (size_t)qrows * g.hid * 2);
-    L.st1 = L.st2 = -1;
+    // LayerNorm statistics: norm1's (one partial per row, from a statistics pass when the
+    // caller's x did not come with partials) and norm2's (written by the proj epilogue)
+    L.st1 = o; o = up256(o + (size_t)rows * 8);
+    L.st2 = o; o = up256(o + (size_t)qrows * store_stats_parts(g.d_out) * 8);
   } else {
     L.q = o; o = up256(o + (size_t)rows * g.N1 * 4);
     L.k = L.v = -1;
@@ -214,11 +217,21 @@ bool weights_aligned(const hiera_block_weights* w) {
   return true;
 }
 
+// stats_x: partial (mean, M2) of x's rows from x's producer ([rows][parts_x]), or nullptr
+// to compute them here; stats_y: where to write y's partials for the next LayerNorm
+// ([qrows][store_stats_parts(d_out)]), or nullptr.
 hiera_status forward_bf16(const Geom& g, const uint8_t* packed, const void* x, void* y,
-                          uint8_t* ws, cudaStream_t st) {
+                          uint8_t* ws, cudaStream_t st, const float2* stats_x = nullptr,
+                          int parts_x = 0, float2* stats_y = nullptr) {
   const PackLayout P = pack_layout(g);
   const WsLayout W = ws_layout(g);
   const long long rows = (long long)g.B * g.tokens, qrows = (long long)g.B * g.Nq;
+  if (stats_x == nullptr) {
+    HIERA_TRY(launch_row_partials_bf16(x, (int)rows, g.d_in, (float2*)(ws + W.st1), st));
+    stats_x = (const float2*)(ws + W.st1);
+    parts_x = 1;
+  }
+  const int parts_out = store_stats_parts(g.d_out);
   // (a3-a6, a8 folded) norm1 + qkv (+ transition proj) with window scatter and q / r pooling
   TcGemmArgs a{};
   a.M = (int)rows;
@@ -230,6 +243,8 @@ hiera_status forward_bf16(const Geom& g, const uint8_t* packed, const void* x, v
   a.colconst = (const float*)(packed + P.c1);
   a.ln_eps = g.eps;
   a.ln_fold = 1;
+  a.stats_in = stats_x;
+  a.stats_parts = parts_x;
   a.q = ws + W.q;
   a.k = ws + W.k;
   a.v = ws + W.v;
@@ -266,6 +281,8 @@ hiera_status forward_bf16(const Geom& g, const uint8_t* packed, const void* x, v
   pj.out = ws + W.x1;
   pj.residual = g.transition ? (const void*)(ws + W.r) : x;
   pj.ldo = g.d_out;
+  pj.stats_out = ws + W.st2;
+  pj.stats_out_parts = parts_out;
   HIERA_TRY(launch_tc_gemm(EPI_STORE, pj, st));
   // (a10, a11) norm2 + fc1 + GELU
   TcGemmArgs f1{};
@@ -278,6 +295,8 @@ hiera_status forward_bf16(const Geom& g, const uint8_t* packed, const void* x, v
   f1.colconst = (const float*)(packed + P.c2);
   f1.ln_eps = g.eps;
   f1.ln_fold = 1;
+  f1.stats_in = ws + W.st2;
+  f1.stats_parts = parts_out;
   f1.out = ws + W.h;
   f1.ldo = g.hid;
   HIERA_TRY(launch_tc_gemm(EPI_GELU, f1, st));
@@ -292,6 +311,8 @@ hiera_status forward_bf16(const Geom& g, const uint8_t* packed, const void* x, v
   f2.out = y;
   f2.residual = ws + W.x1;
   f2.ldo = g.d_out;
+  f2.stats_out = stats_y;
+  f2.stats_out_parts = stats_y != nullptr ? parts_out : 0;
   return launch_tc_gemm(EPI_STORE, f2, st);
 }
 
@@ -453,7 +474,7 @@ BackbonePack backbone_pack_layout(const hiera_backbone_desc* bd, const BlockPlan
 }
 
 struct BackboneWs {
-  size_t act0, act1, block, total;
+  size_t act0, act1, st0, st1, block, total;
 };
 
 BackboneWs backbone_ws_layout(const hiera_backbone_desc* bd, const BlockPlan plan[kDepth]) {
@@ -467,9 +488,13 @@ BackboneWs backbone_ws_layout(const hiera_backbone_desc* bd, const BlockPlan pla
     make_geom(&plan[i].d, &g);
     blk = std::max(blk, ws_layout(g).total);
   }
+  // LayerNorm partials passed from block to block: at most 2 per stage-0 token
+  const size_t stb = (size_t)bd->B * G0 * G0 * 2 * 8;
   L.act0 = 0;
   L.act1 = up256(act);
-  L.block = L.act1 + up256(act);
+  L.st0 = L.act1 + up256(act);
+  L.st1 = L.st0 + up256(stb);
+  L.block = L.st1 + up256(stb);
   L.total = L.block + blk;
   return L;
 }
@@ -747,7 +772,7 @@ hiera_status hiera_patch_embed(const void* img, const void* packed_patch, const 
     return HIERA_ERR_ALIGNMENT;
   HIERA_TRY(check_device());
   const float* p = static_cast<const float*>(packed_patch);
-  return launch_patch_embed(img, p, p + 196 * 112, pos_embed, out, B, img_side,
+  return launch_patch_embed(img, p, p + 196 * 112, pos_embed, out, nullptr, B, img_side,
                             dtype == HIERA_BF16 ? 1 : 0, (cudaStream_t)stream);
 }
 
@@ -820,17 +845,22 @@ hiera_status hiera_backbone_forward(const hiera_backbone_desc* desc, const void*
   const int es = bf ? 2 : 4;
   const int G0 = desc->img / 4;
   uint8_t* act[2] = {ws + W.act0, ws + W.act1};
-  // (a0-a2) patch embedding + pos_embed + Unroll, fused
+  float2* stp[2] = {(float2*)(ws + W.st0), (float2*)(ws + W.st1)};
+  // (a0-a2) patch embedding + pos_embed + Unroll, fused; in bf16 it also emits the LayerNorm
+  // partials of its output (two 56-channel halves per token) for block 0's norm1
   HIERA_TRY(launch_patch_embed(img_nhwc, pk + P.patch_w, (const float*)(pk + P.patch_b),
-                               pk + P.pos, act[0], desc->B, desc->img, bf, st));
-  int cur = 0, s_idx = 0;
+                               pk + P.pos, act[0], bf ? stp[0] : nullptr, desc->B, desc->img,
+                               bf, st));
+  int cur = 0, s_idx = 0, parts = 2;
   for (int i = 0; i < kDepth; ++i) {
     Geom g;
     make_geom(&plan[i].d, &g);
     const uint8_t* bp = pk + P.blocks[i];
     uint8_t* out = act[cur ^ 1];
-    HIERA_TRY(g.bf16 ? forward_bf16(g, bp, act[cur], out, ws + W.block, st)
+    HIERA_TRY(g.bf16 ? forward_bf16(g, bp, act[cur], out, ws + W.block, st, stp[cur], parts,
+                                    stp[cur ^ 1])
                      : forward_f32(g, bp, act[cur], out, ws + W.block, st));
+    parts = store_stats_parts(g.d_out);
     cur ^= 1;
     if (s_idx < 4 && i == kStageEnds[s_idx]) {
       // (a13) Reroll the stage output to NHWC
@@ -868,7 +898,7 @@ const char* hiera_kernel_name(int kind) {
   static const char* names[K_COUNT] = {
       "patch_embed", "unroll_reroll", "gemm_qkv_lnfold", "gemm_fc1_lnfold_gelu",
       "gemm_bias_residual", "attention_tiled", "attention_packed", "f32_gemm",
-      "f32_attention", "f32_row_stats", "pack", "timeout_probe"};
+      "f32_attention", "f32_row_stats", "pack", "timeout_probe", "row_stats"};
   return (kind >= 0 && kind < K_COUNT) ? names[kind] : "unknown";
 }
 

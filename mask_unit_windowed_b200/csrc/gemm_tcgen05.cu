@@ -10,15 +10,19 @@
 //               swizzle, STAGES-deep ring guarded by full/empty mbarriers.
 //   warp 1      owns TMEM (2 accumulators of BN fp32 columns) and issues tcgen05.mma
 //               (M = 128, N = BN, K = 16 per instruction) from one thread.
-//   warps 2-5   epilogue: tcgen05.ld of the accumulator (TMEM lane = tile row), the
-//               LayerNorm fold / bias / GELU / residual, and the store or the scatter
-//               into head-major q/k/v with the q_stride max-pool.
-//   warps 6-9   (LayerNorm-fold GEMMs only) row statistics of A read from the same
-//               shared-memory stages as they stream past: per-64-column mean and M2,
-//               merged with Chan's parallel update, so LayerNorm costs no extra pass.
+//   warps 2-9   epilogue, two warps per TMEM lane quarter (each half of the columns):
+//               tcgen05.ld of the accumulator (TMEM lane = tile row), the LayerNorm fold /
+//               bias / GELU / residual, and the store or the scatter into head-major
+//               q/k/v with the q_stride max-pool.
 //
 // LayerNorm fold: with W' = W diag(gamma) (packed once), s_n = sum_k W'_nk and
 // c_n = sum_k beta_k W_nk + b_n,  LN(x) W^T + b = rstd * (x W'^T - mean * s) + c.
+// The row statistics arrive as P partial (mean, M2) pairs per row, each over K/P
+// columns, written by whichever kernel produced x (the epilogue of the previous GEMM,
+// the patch embedding, or a statistics pass); the epilogue merges them with Chan's
+// formula, so LayerNorm costs no extra pass over x. A STORE epilogue can itself emit
+// such partials of the values it writes (after rounding to bf16), one per (row, column
+// half of its tile).
 // Transition pooling: a 4-D tensor map loads, for 32 pooled tokens n, the four rows
 // n + c*T/4 (c = 0..3) interleaved, so the four pooling candidates are adjacent TMEM
 // lanes and the max is two warp shuffles.
@@ -51,6 +55,10 @@ struct KParams {
   int tokens, nW, heads, d_out, Tq, Tkv;
   uint64_t limit_ns;
   unsigned int* status;
+  const float2* stats_in;  // FOLD: [M][stats_parts] partial (mean, M2) of A's rows
+  int stats_parts;
+  float2* stats_out;       // STORE: [M][stats_out_parts] partials of the output, or nullptr
+  int stats_out_parts;
 };
 
 constexpr int cmin(int a, int b) { return a < b ? a : b; }
@@ -67,8 +75,7 @@ struct Cfg {
   static constexpr int CH = (HALF % 56 == 0) ? 56 : cmin(HALF, 32);  // columns per chunk
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
   static constexpr int CONST_OFF = BAR_OFF + 256;        // colsum[BN], colconst[BN] (fp32)
-  static constexpr int STATS_OFF = CONST_OFF + 2 * BN * 4;
-  static constexpr int SMEM_BYTES = STATS_OFF + 2 * 128 * 8 + 1024;
+  static constexpr int SMEM_BYTES = CONST_OFF + 2 * BN * 4 + 1024;
   static_assert(B_BYTES % 1024 == 0, "W tile must keep 1024-byte alignment");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128");
   static_assert(HALF % CH == 0 && CH % 8 == 0, "epilogue chunking");
@@ -117,17 +124,8 @@ __device__ __forceinline__ uint4 pack8(const float* v) {
   return pk;
 }
 
-__device__ __forceinline__ uint4 pack8_add(const float* v, uint4 rr) {
-  uint4 pk;
-  pk.x = pack_bf16x2(v[0] + bf16_lo(rr.x), v[1] + bf16_hi(rr.x));
-  pk.y = pack_bf16x2(v[2] + bf16_lo(rr.y), v[3] + bf16_hi(rr.y));
-  pk.z = pack_bf16x2(v[4] + bf16_lo(rr.z), v[5] + bf16_hi(rr.z));
-  pk.w = pack_bf16x2(v[6] + bf16_lo(rr.w), v[7] + bf16_hi(rr.w));
-  return pk;
-}
-
 template <int BN, int EPI, bool FOLD, bool POOLED>
-__global__ void __launch_bounds__(FOLD ? 448 : 320, 1)
+__global__ void __launch_bounds__(320, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const KParams p) {
   using C = Cfg<BN>;
@@ -140,14 +138,11 @@ __global__ void __launch_bounds__(FOLD ? 448 : 320, 1)
   uint64_t* empty = bars + STAGES;
   uint64_t* acc_full = bars + 2 * STAGES;
   uint64_t* acc_empty = acc_full + 2;
-  uint64_t* st_full = acc_empty + 2;
-  uint64_t* st_empty = st_full + 2;
-  uint64_t* drain = st_empty + 2;
+  uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* col_sum = reinterpret_cast<float*>(smem + C::CONST_OFF);
   float* col_const = col_sum + BN;
-  float2* stats = reinterpret_cast<float2*>(smem + C::STATS_OFF);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m_tiles = POOLED ? ((p.M >> 2) + 31) / 32 : (p.M + BM - 1) / BM;
@@ -158,13 +153,11 @@ __global__ void __launch_bounds__(FOLD ? 448 : 320, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + (FOLD ? 128 : 0));
+      mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
       mbar_init(&acc_empty[a], EPI_THREADS);
-      mbar_init(&st_full[a], 128);
-      mbar_init(&st_empty[a], EPI_THREADS);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -316,6 +309,31 @@ __global__ void __launch_bounds__(FOLD ? 448 : 320, 1)
                            : make_uint4(0u, 0u, 0u, 0u);
         }
       }
+      // LayerNorm statistics of this row, merged from the producer's partials
+      float fa = 1.f, fb = 0.f;  // v = fa * acc + fb * colsum + colconst
+      if (FOLD && row_ok) {
+        const int P = p.stats_parts;
+        const float2* sp = p.stats_in + m * P;
+        float2 part[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) part[j] = j < P ? __ldg(sp + j) : make_float2(0.f, 0.f);
+        float mean = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) mean += part[j].x;
+        mean /= (float)P;
+        float m2 = 0.f, dev2 = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (j < P) {
+            const float dlt = part[j].x - mean;
+            m2 += part[j].y;
+            dev2 = fmaf(dlt, dlt, dev2);
+          }
+        }
+        m2 = fmaf((float)(p.K / P), dev2, m2);   // Chan et al., equal counts K / P
+        fa = rsqrtf(m2 / (float)p.K + p.ln_eps);
+        fb = -mean * fa;
+      }
       // per-column constants of this tile into shared memory
       named_bar_sync(1, EPI_THREADS);  // every epilogue thread is done with the last tile's
       for (int i = etid; i < BN; i += EPI_THREADS) {
@@ -325,20 +343,13 @@ __global__ void __launch_bounds__(FOLD ? 448 : 320, 1)
       }
       named_bar_sync(1, EPI_THREADS);
       if (!warp_wait(&acc_full[acc], aph, p.limit_ns, p.status, abort_flag)) break;
-      float fa = 1.f, fb = 0.f;  // v = fa * acc + fb * colsum + colconst
-      if (FOLD) {
-        if (!warp_wait(&st_full[acc], aph, p.limit_ns, p.status, abort_flag)) break;
-        const float2 st = stats[acc * 128 + rt];
-        mbar_arrive(&st_empty[acc]);
-        fa = st.y;
-        fb = -st.x * st.y;
-      }
       tc_fence_after();
       const uint32_t tbase = tmem + (uint32_t)(acc * C::ACC_STRIDE) +
                              ((uint32_t)(quarter * 32) << 16) + (uint32_t)c_begin;
       const int which = (EPI == EPI_QKV) ? n0 / p.d_out : 0;
       const bool pool_this = POOLED && (which == 0 || which == 3);
       const bool writer = row_ok && (!pool_this || (rt & 3) == 0);
+      float st_mean = 0.f, st_m2 = 0.f;  // running statistics of the stored half row
 #pragma unroll
       for (int c = 0; c < HALF; c += CH) {
         uint32_t r[CH];
@@ -385,89 +396,56 @@ __global__ void __launch_bounds__(FOLD ? 448 : 320, 1)
           }
         } else if (row_ok) {
           bf16* dst = p.out + m * p.ldo + n0 + c_begin + c;
+          if (EPI == EPI_STORE && has_res) {
+#pragma unroll
+            for (int g = 0; g < CH / 8; ++g) {
+              const uint4 rr = res[(c / 8 + g) < NV ? (c / 8 + g) : 0];
+              v[8 * g + 0] += bf16_lo(rr.x);
+              v[8 * g + 1] += bf16_hi(rr.x);
+              v[8 * g + 2] += bf16_lo(rr.y);
+              v[8 * g + 3] += bf16_hi(rr.y);
+              v[8 * g + 4] += bf16_lo(rr.z);
+              v[8 * g + 5] += bf16_hi(rr.z);
+              v[8 * g + 6] += bf16_lo(rr.w);
+              v[8 * g + 7] += bf16_hi(rr.w);
+            }
+          }
 #pragma unroll
           for (int g = 0; g < CH / 8; ++g) {
-            uint4 pk;
-            if (EPI == EPI_STORE && has_res)
-              pk = pack8_add(&v[8 * g], res[(c / 8 + g) < NV ? (c / 8 + g) : 0]);
-            else
-              pk = pack8(&v[8 * g]);
+            const uint4 pk = pack8(&v[8 * g]);
             *reinterpret_cast<uint4*>(dst + 8 * g) = pk;
+            if (EPI == EPI_STORE && p.stats_out != nullptr) {
+              // statistics of the values as stored (bf16)
+              v[8 * g + 0] = bf16_lo(pk.x);
+              v[8 * g + 1] = bf16_hi(pk.x);
+              v[8 * g + 2] = bf16_lo(pk.y);
+              v[8 * g + 3] = bf16_hi(pk.y);
+              v[8 * g + 4] = bf16_lo(pk.z);
+              v[8 * g + 5] = bf16_hi(pk.z);
+              v[8 * g + 6] = bf16_lo(pk.w);
+              v[8 * g + 7] = bf16_hi(pk.w);
+            }
+          }
+          if (EPI == EPI_STORE && p.stats_out != nullptr) {
+            float s = 0.f;
+#pragma unroll
+            for (int i = 0; i < CH; ++i) s += v[i];
+            const float cmean = s * (1.f / (float)CH);
+            float cm2 = 0.f;
+#pragma unroll
+            for (int i = 0; i < CH; ++i) cm2 = fmaf(v[i] - cmean, v[i] - cmean, cm2);
+            // Chan et al. merge of this chunk into the running (count, mean, M2)
+            const float na = (float)c, nb = (float)CH, nt_ = na + nb;
+            const float dlt = cmean - st_mean;
+            st_mean = fmaf(dlt, nb / nt_, st_mean);
+            st_m2 = st_m2 + cm2 + dlt * dlt * (na * nb / nt_);
           }
         }
       }
+      if (EPI == EPI_STORE && p.stats_out != nullptr && row_ok)
+        p.stats_out[m * p.stats_out_parts + nt * 2 + (ew >> 2)] = make_float2(st_mean, st_m2);
       tc_fence_before();
       mbar_arrive(&acc_empty[acc]);
-      if (++acc == 2) {
-        acc = 0;
-        aph ^= 1u;
-      }
-    }
-  } else if (FOLD) {
-    // ------------------------------------------------------------ LayerNorm row statistics
-    const int t = (warp - 2 - EPI_WARPS) * 32 + lane;
-    int s = 0, acc = 0;
-    uint32_t ph = 0, aph = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-      if (!warp_wait(&st_empty[acc], aph ^ 1u, p.limit_ns, p.status, abort_flag)) break;
-      float mean = 0.f, m2 = 0.f;
-      int cnt = 0;
-      for (int kb = 0; kb < kblocks; ++kb) {
-        if (!warp_wait(&full[s], ph, p.limit_ns, p.status, abort_flag)) {
-          ok = false;
-          break;
-        }
-        const uint4* row = reinterpret_cast<const uint4*>(smem + s * C::STAGE_BYTES + t * 128);
-        uint4 ch[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) ch[c] = row[c];
-        const int kvalid = min(BK, p.K - kb * BK);
-        // physical 16-byte chunk c of this 128-byte row holds logical chunk c ^ (row & 7)
-        float sum = 0.f;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const int k0 = ((c ^ (t & 7)) << 3);
-          const uint32_t wv[4] = {ch[c].x, ch[c].y, ch[c].z, ch[c].w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            if (k0 + 2 * e < kvalid) sum += bf16_lo(wv[e]);
-            if (k0 + 2 * e + 1 < kvalid) sum += bf16_hi(wv[e]);
-          }
-        }
-        const float bmean = sum / (float)kvalid;
-        float bm2 = 0.f;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const int k0 = ((c ^ (t & 7)) << 3);
-          const uint32_t wv[4] = {ch[c].x, ch[c].y, ch[c].z, ch[c].w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float d0 = bf16_lo(wv[e]) - bmean, d1 = bf16_hi(wv[e]) - bmean;
-            if (k0 + 2 * e < kvalid) bm2 += d0 * d0;
-            if (k0 + 2 * e + 1 < kvalid) bm2 += d1 * d1;
-          }
-        }
-        // The stage may be refilled by TMA (async proxy) as soon as every consumer has
-        // arrived: consume the loaded values first, order these generic-proxy reads before
-        // the async-proxy writes that follow the release, then arrive.
-        asm volatile("" ::"f"(bmean), "f"(bm2) : "memory");
-        fence_proxy_async_smem();
-        mbar_arrive(&empty[s]);
-        // Chan et al. pairwise update of (count, mean, M2)
-        const int tot = cnt + kvalid;
-        const float delta = bmean - mean;
-        mean += delta * ((float)kvalid / (float)tot);
-        m2 += bm2 + delta * delta * ((float)cnt * (float)kvalid / (float)tot);
-        cnt = tot;
-        if (++s == STAGES) {
-          s = 0;
-          ph ^= 1u;
-        }
-      }
-      if (!ok) break;
-      stats[acc * 128 + t] = make_float2(mean, rsqrtf(m2 / (float)p.K + p.ln_eps));
-      mbar_arrive(&st_full[acc]);
       if (++acc == 2) {
         acc = 0;
         aph ^= 1u;
@@ -563,6 +541,10 @@ hiera_status run(const TcGemmArgs& a, cudaStream_t stream) {
   p.Tkv = a.Tkv;
   p.limit_ns = g_wait_limit_ns();
   p.status = g_status_ptr();
+  p.stats_in = static_cast<const float2*>(a.stats_in);
+  p.stats_parts = a.stats_parts;
+  p.stats_out = static_cast<float2*>(a.stats_out);
+  p.stats_out_parts = a.stats_out_parts;
 
   auto kern = tc_gemm_kernel<BN, EPI, FOLD, POOLED>;
   static bool attr_done[64] = {false};  // per device
@@ -581,7 +563,7 @@ hiera_status run(const TcGemmArgs& a, cudaStream_t stream) {
   if (grid > tiles) grid = tiles;
   profile_mark(EPI == EPI_QKV ? K_GEMM_QKV : (EPI == EPI_GELU ? K_GEMM_GELU : K_GEMM_STORE),
                stream);
-  kern<<<grid, FOLD ? 448 : 320, C::SMEM_BYTES, stream>>>(tmA, tmB, p);
+  kern<<<grid, 320, C::SMEM_BYTES, stream>>>(tmA, tmB, p);
   return cudaGetLastError() == cudaSuccess ? HIERA_OK : HIERA_ERR_CUDA;
 }
 
@@ -590,6 +572,12 @@ hiera_status run(const TcGemmArgs& a, cudaStream_t stream) {
 hiera_status launch_tc_gemm(int epi, const TcGemmArgs& a, cudaStream_t stream) {
   if (a.M <= 0 || a.N <= 0 || a.K <= 0) return HIERA_OK;
   if (a.N % 16 != 0 || a.K % 8 != 0) return HIERA_ERR_SHAPE;
+  if (a.ln_fold && (a.stats_in == nullptr || a.stats_parts < 1 || a.stats_parts > 8 ||
+                    a.K % a.stats_parts != 0))
+    return HIERA_ERR_INVALID_ARG;
+  if (a.stats_out != nullptr &&
+      (epi != EPI_STORE || a.stats_out_parts != 2 * (a.N / store_bn(a.N))))
+    return HIERA_ERR_INVALID_ARG;
   if (epi == EPI_QKV) {
     if (!a.ln_fold) return HIERA_ERR_INVALID_ARG;
     const bool pooled = a.pooled != 0;
@@ -614,12 +602,14 @@ hiera_status launch_tc_gemm(int epi, const TcGemmArgs& a, cudaStream_t stream) {
     return HIERA_ERR_SHAPE;
   }
   if (a.ln_fold) return HIERA_ERR_INVALID_ARG;
-  if (a.N % 224 == 0) return run<224, EPI_STORE, false, false>(a, stream);
-  if (a.N % 128 == 0) return run<128, EPI_STORE, false, false>(a, stream);
-  if (a.N % 112 == 0) return run<112, EPI_STORE, false, false>(a, stream);
-  if (a.N % 64 == 0) return run<64, EPI_STORE, false, false>(a, stream);
-  if (a.N % 32 == 0) return run<32, EPI_STORE, false, false>(a, stream);
-  return run<16, EPI_STORE, false, false>(a, stream);
+  switch (store_bn(a.N)) {
+    case 224: return run<224, EPI_STORE, false, false>(a, stream);
+    case 128: return run<128, EPI_STORE, false, false>(a, stream);
+    case 112: return run<112, EPI_STORE, false, false>(a, stream);
+    case 64: return run<64, EPI_STORE, false, false>(a, stream);
+    case 32: return run<32, EPI_STORE, false, false>(a, stream);
+    default: return run<16, EPI_STORE, false, false>(a, stream);
+  }
 }
 
 }  // namespace hiera

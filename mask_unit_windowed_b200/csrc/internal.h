@@ -17,7 +17,7 @@ unsigned int* g_status_ptr();            // device address of the status word (c
 enum KernelId {
   K_PATCH_EMBED = 0, K_PERMUTE = 1, K_GEMM_QKV = 2, K_GEMM_GELU = 3, K_GEMM_STORE = 4,
   K_ATTN_TILED = 5, K_ATTN_PACKED = 6, K_F32_GEMM = 7, K_F32_ATTN = 8, K_F32_STATS = 9,
-  K_PACK = 10, K_PROBE = 11, K_COUNT = 12
+  K_PACK = 10, K_PROBE = 11, K_ROW_STATS = 12, K_COUNT = 13
 };
 void profile_mark(int kind, cudaStream_t stream);  // no-op unless a session is open
 
@@ -37,6 +37,10 @@ struct TcGemmArgs {
   const void* bias_bf16;  // [N] bf16 bias used when colconst is nullptr (may be nullptr)
   float ln_eps;
   int ln_fold;            // 1: LayerNorm of A's rows folded into the epilogue
+  const void* stats_in;   // ln_fold: float2 [M][stats_parts] partial (mean, M2) of A's rows,
+  int stats_parts;        //          each over K / stats_parts columns (1..8 parts)
+  void* stats_out;        // EPI_STORE: float2 [M][stats_out_parts] partials of the output
+  int stats_out_parts;    //          (= 2 * N / store_bn(N)), or nullptr
   // EPI_STORE / EPI_GELU: out[m * ldo + n] (+ residual[m * ldo + n])
   void* out;
   const void* residual;
@@ -52,6 +56,18 @@ struct TcGemmArgs {
 };
 
 hiera_status launch_tc_gemm(int epi, const TcGemmArgs& a, cudaStream_t stream);
+
+// N-tile width the plain-store GEMM uses for N output columns (N a multiple of 16).
+inline int store_bn(int N) {
+  return N % 224 == 0 ? 224 : N % 128 == 0 ? 128 : N % 112 == 0 ? 112 : N % 64 == 0 ? 64
+         : N % 32 == 0 ? 32 : 16;
+}
+// Partial statistics per row written by a plain-store GEMM with N columns.
+inline int store_stats_parts(int N) { return 2 * (N / store_bn(N)); }
+
+// Per-row (mean, M2) of a bf16 [M, K] matrix as one partial per row.
+hiera_status launch_row_partials_bf16(const void* x, int M, int K, float2* out,
+                                      cudaStream_t stream);
 
 // ---------------------------------------------------------------- attention (bf16, mma.sync)
 struct AttnArgs {
@@ -96,8 +112,10 @@ hiera_status launch_copy_pack(const void* w, const void* bias, int N, int K, int
                               void* w_out, float* bias_out, cudaStream_t stream);
 hiera_status launch_patch_pack(const void* w, const void* bias, int dtype_bf16, float* wt,
                                float* bias_out, cudaStream_t stream);
+// stats_out (bf16 only, may be nullptr): float2 [B*N][2] partial (mean, M2) of each output
+// token's two 56-channel halves.
 hiera_status launch_patch_embed(const void* img, const void* w, const float* b,
-                                const void* pos, void* out, int B, int img_side,
-                                int dtype_bf16, cudaStream_t stream);
+                                const void* pos, void* out, float2* stats_out, int B,
+                                int img_side, int dtype_bf16, cudaStream_t stream);
 
 }  // namespace hiera

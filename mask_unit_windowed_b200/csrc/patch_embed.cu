@@ -40,7 +40,9 @@ __global__ void __launch_bounds__(256, 1) patch_embed_kernel(const T* __restrict
                                                              const float* __restrict__ wt,
                                                              const float* __restrict__ bias,
                                                              const T* __restrict__ pos,
-                                                             T* __restrict__ out, int img_side) {
+                                                             T* __restrict__ out,
+                                                             float2* __restrict__ stats_out,
+                                                             int img_side) {
   extern __shared__ __align__(16) float smem_f[];
   float* sW = smem_f;                 // [196][112]
   float* sIn = smem_f + KTOT * COUT;  // [7][4][XPITCH]
@@ -106,10 +108,23 @@ __global__ void __launch_bounds__(256, 1) patch_embed_kernel(const T* __restrict
       for (int j = 0; j < 56; ++j) {
         const float v = acc[j] + __ldg(bias + half * 56 + j) + to_f(pr[j]);
         if constexpr (sizeof(T) == 2) {
-          dst[j] = __float2bfloat16_rn(v);
+          const bf16 rv = __float2bfloat16_rn(v);
+          dst[j] = rv;
+          acc[j] = __bfloat162float(rv);  // the value as stored, for the statistics below
         } else {
           dst[j] = v;
         }
+      }
+      if (stats_out != nullptr) {
+        // partial (mean, M2) of this half of the token, for the first block's norm1
+        float s = 0.f;
+#pragma unroll
+        for (int j = 0; j < 56; ++j) s += acc[j];
+        const float mean = s * (1.f / 56.f);
+        float m2 = 0.f;
+#pragma unroll
+        for (int j = 0; j < 56; ++j) m2 = fmaf(acc[j] - mean, acc[j] - mean, m2);
+        stats_out[((long long)b * N + u) * 2 + half] = make_float2(mean, m2);
       }
     }
   }
@@ -118,8 +133,8 @@ __global__ void __launch_bounds__(256, 1) patch_embed_kernel(const T* __restrict
 }  // namespace
 
 hiera_status launch_patch_embed(const void* img, const void* w, const float* b, const void* pos,
-                                void* out, int B, int img_side, int dtype_bf16,
-                                cudaStream_t stream) {
+                                void* out, float2* stats_out, int B, int img_side,
+                                int dtype_bf16, cudaStream_t stream) {
   const int G = img_side / 4;
   dim3 grid((G + SEG - 1) / SEG, (G + ROWS - 1) / ROWS, B);
   if (grid.y > 65535 || grid.z > 65535) return HIERA_ERR_SHAPE;
@@ -136,7 +151,7 @@ hiera_status launch_patch_embed(const void* img, const void* w, const float* b, 
     }
     patch_embed_kernel<bf16><<<grid, 256, SMEM_TOTAL, stream>>>(
         static_cast<const bf16*>(img), static_cast<const float*>(w), b,
-        static_cast<const bf16*>(pos), static_cast<bf16*>(out), img_side);
+        static_cast<const bf16*>(pos), static_cast<bf16*>(out), stats_out, img_side);
   } else {
     if (dev < 64 && !attr_done[0][dev]) {
       if (cudaFuncSetAttribute(patch_embed_kernel<float>,
@@ -147,7 +162,7 @@ hiera_status launch_patch_embed(const void* img, const void* w, const float* b, 
     }
     patch_embed_kernel<float><<<grid, 256, SMEM_TOTAL, stream>>>(
         static_cast<const float*>(img), static_cast<const float*>(w), b,
-        static_cast<const float*>(pos), static_cast<float*>(out), img_side);
+        static_cast<const float*>(pos), static_cast<float*>(out), nullptr, img_side);
   }
   return cudaGetLastError() == cudaSuccess ? HIERA_OK : HIERA_ERR_CUDA;
 }
