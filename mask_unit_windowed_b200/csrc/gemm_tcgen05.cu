@@ -68,14 +68,17 @@ struct Cfg {
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = cmin(8, (184 * 1024) / STAGE_BYTES);
+  static constexpr int STG_BYTES = 8 * 32 * 128;  // per epilogue warp: 32 rows x 128 B staging
+  static constexpr int STAGES =
+      cmin(8, (227 * 1024 - 1024 - 256 - 2 * BN * 4 - 128 - STG_BYTES) / STAGE_BYTES);
   static constexpr int ACC_STRIDE = BN <= 128 ? 128 : 256;
   static constexpr int TMEM_COLS = 2 * ACC_STRIDE;
   static constexpr int HALF = BN / 2;                    // columns per epilogue thread
   static constexpr int CH = (HALF % 56 == 0) ? 56 : cmin(HALF, 32);  // columns per chunk
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
   static constexpr int CONST_OFF = BAR_OFF + 256;        // colsum[BN], colconst[BN] (fp32)
-  static constexpr int SMEM_BYTES = CONST_OFF + 2 * BN * 4 + 1024;
+  static constexpr int STG_OFF = (CONST_OFF + 2 * BN * 4 + 127) / 128 * 128;
+  static constexpr int SMEM_BYTES = STG_OFF + STG_BYTES + 1024;
   static_assert(B_BYTES % 1024 == 0, "W tile must keep 1024-byte alignment");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128");
   static_assert(HALF % CH == 0 && CH % 8 == 0, "epilogue chunking");
@@ -143,6 +146,7 @@ __global__ void __launch_bounds__(320, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* col_sum = reinterpret_cast<float*>(smem + C::CONST_OFF);
   float* col_const = col_sum + BN;
+  uint8_t* stg_all = smem + C::STG_OFF;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m_tiles = POOLED ? ((p.M >> 2) + 31) / 32 : (p.M + BM - 1) / BM;
@@ -363,6 +367,7 @@ __global__ void __launch_bounds__(320, 1)
           if (EPI == EPI_GELU) x = gelu_fast(x);
           v[i] = x;
         }
+        // ---- finish the values of this chunk (pooling / residual)
         if (EPI == EPI_QKV) {
           static_assert(EPI != EPI_QKV || CH == 56, "q/k/v chunks are whole heads");
           if (pool_this) {
@@ -372,75 +377,93 @@ __global__ void __launch_bounds__(320, 1)
               v[i] = fmaxf(v[i], __shfl_xor_sync(0xffffffffu, v[i], 2));
             }
           }
-          if (writer) {
-            const int colw = n0 - which * p.d_out + c_begin + c;  // multiple of 56
-            if (which == 3) {
-              const int nq = POOLED ? (p.tokens >> 2) : p.tokens;
-              const int tq = POOLED ? np : tok;
-              bf16* dst = p.r + ((long long)b * nq + tq) * p.d_out + colw;
-#pragma unroll
-              for (int g = 0; g < CH / 8; ++g)
-                *reinterpret_cast<uint4*>(dst + 8 * g) = pack8(&v[8 * g]);
-            } else {
-              const int h = colw / 56;
-              const int tt = pool_this ? np : tok;
-              const int w = tt % p.nW, j = tt / p.nW;
-              const int T = which == 0 ? p.Tq : p.Tkv;
-              bf16* base = which == 0 ? p.q : (which == 1 ? p.k : p.v);
-              bf16* dst = base + ((((long long)b * p.nW + w) * p.heads + h) * T + j) * 64;
-#pragma unroll
-              for (int g = 0; g < 7; ++g)
-                *reinterpret_cast<uint4*>(dst + 8 * g) = pack8(&v[8 * g]);
-              *reinterpret_cast<uint4*>(dst + 56) = make_uint4(0u, 0u, 0u, 0u);
-            }
-          }
-        } else if (row_ok) {
-          bf16* dst = p.out + m * p.ldo + n0 + c_begin + c;
-          if (EPI == EPI_STORE && has_res) {
-#pragma unroll
-            for (int g = 0; g < CH / 8; ++g) {
-              const uint4 rr = res[(c / 8 + g) < NV ? (c / 8 + g) : 0];
-              v[8 * g + 0] += bf16_lo(rr.x);
-              v[8 * g + 1] += bf16_hi(rr.x);
-              v[8 * g + 2] += bf16_lo(rr.y);
-              v[8 * g + 3] += bf16_hi(rr.y);
-              v[8 * g + 4] += bf16_lo(rr.z);
-              v[8 * g + 5] += bf16_hi(rr.z);
-              v[8 * g + 6] += bf16_lo(rr.w);
-              v[8 * g + 7] += bf16_hi(rr.w);
-            }
-          }
+        } else if (EPI == EPI_STORE && has_res) {
 #pragma unroll
           for (int g = 0; g < CH / 8; ++g) {
-            const uint4 pk = pack8(&v[8 * g]);
-            *reinterpret_cast<uint4*>(dst + 8 * g) = pk;
-            if (EPI == EPI_STORE && p.stats_out != nullptr) {
-              // statistics of the values as stored (bf16)
-              v[8 * g + 0] = bf16_lo(pk.x);
-              v[8 * g + 1] = bf16_hi(pk.x);
-              v[8 * g + 2] = bf16_lo(pk.y);
-              v[8 * g + 3] = bf16_hi(pk.y);
-              v[8 * g + 4] = bf16_lo(pk.z);
-              v[8 * g + 5] = bf16_hi(pk.z);
-              v[8 * g + 6] = bf16_lo(pk.w);
-              v[8 * g + 7] = bf16_hi(pk.w);
-            }
-          }
-          if (EPI == EPI_STORE && p.stats_out != nullptr) {
-            float s = 0.f;
-#pragma unroll
-            for (int i = 0; i < CH; ++i) s += v[i];
-            const float cmean = s * (1.f / (float)CH);
-            float cm2 = 0.f;
-#pragma unroll
-            for (int i = 0; i < CH; ++i) cm2 = fmaf(v[i] - cmean, v[i] - cmean, cm2);
-            // Chan et al. merge of this chunk into the running (count, mean, M2)
-            const float na = (float)c, nb = (float)CH, nt_ = na + nb;
-            const float dlt = cmean - st_mean;
-            st_mean = fmaf(dlt, nb / nt_, st_mean);
-            st_m2 = st_m2 + cm2 + dlt * dlt * (na * nb / nt_);
+            const uint4 rr = res[(c / 8 + g) < NV ? (c / 8 + g) : 0];
+            v[8 * g + 0] += bf16_lo(rr.x);
+            v[8 * g + 1] += bf16_hi(rr.x);
+            v[8 * g + 2] += bf16_lo(rr.y);
+            v[8 * g + 3] += bf16_hi(rr.y);
+            v[8 * g + 4] += bf16_lo(rr.z);
+            v[8 * g + 5] += bf16_hi(rr.z);
+            v[8 * g + 6] += bf16_lo(rr.w);
+            v[8 * g + 7] += bf16_hi(rr.w);
           }
         }
+        // ---- destination of this lane's row for this chunk
+        bf16* dst_row = nullptr;
+        bool valid = row_ok;
+        int nchunk = CH / 8;  // 16-byte chunks per row written
+        if (EPI == EPI_QKV) {
+          valid = writer;
+          const int colw = n0 - which * p.d_out + c_begin + c;  // multiple of 56
+          if (which == 3) {
+            const int nq = POOLED ? (p.tokens >> 2) : p.tokens;
+            const int tq = POOLED ? np : tok;
+            dst_row = p.r + ((long long)b * nq + tq) * p.d_out + colw;
+          } else {
+            const int h = colw / 56;
+            const int tt = pool_this ? np : tok;
+            const int w = tt % p.nW, j = tt / p.nW;
+            const int T = which == 0 ? p.Tq : p.Tkv;
+            bf16* base = which == 0 ? p.q : (which == 1 ? p.k : p.v);
+            dst_row = base + ((((long long)b * p.nW + w) * p.heads + h) * T + j) * 64;
+            nchunk = 8;  // channels 56..63 of every head row are zero padding
+          }
+        } else {
+          dst_row = p.out + m * p.ldo + n0 + c_begin + c;
+        }
+        // ---- stage the packed row in shared memory (XOR-swizzled 16-byte chunks)
+        uint8_t* stg = stg_all + (ew << 12);
+#pragma unroll
+        for (int g = 0; g < CH / 8; ++g) {
+          const uint4 pk = pack8(&v[8 * g]);
+          *reinterpret_cast<uint4*>(stg + (lane << 7) + ((g ^ (lane & 7)) << 4)) = pk;
+          if (EPI == EPI_STORE && p.stats_out != nullptr) {
+            // statistics of the values as stored (bf16)
+            v[8 * g + 0] = bf16_lo(pk.x);
+            v[8 * g + 1] = bf16_hi(pk.x);
+            v[8 * g + 2] = bf16_lo(pk.y);
+            v[8 * g + 3] = bf16_hi(pk.y);
+            v[8 * g + 4] = bf16_lo(pk.z);
+            v[8 * g + 5] = bf16_hi(pk.z);
+            v[8 * g + 6] = bf16_lo(pk.w);
+            v[8 * g + 7] = bf16_hi(pk.w);
+          }
+        }
+        if (EPI == EPI_QKV && CH == 56)
+          *reinterpret_cast<uint4*>(stg + (lane << 7) + ((7 ^ (lane & 7)) << 4)) =
+              make_uint4(0u, 0u, 0u, 0u);
+        if (EPI == EPI_STORE && p.stats_out != nullptr && row_ok) {
+          float s = 0.f;
+#pragma unroll
+          for (int i = 0; i < CH; ++i) s += v[i];
+          const float cmean = s * (1.f / (float)CH);
+          float cm2 = 0.f;
+#pragma unroll
+          for (int i = 0; i < CH; ++i) cm2 = fmaf(v[i] - cmean, v[i] - cmean, cm2);
+          // Chan et al. merge of this chunk into the running (count, mean, M2)
+          const float na = (float)c, nb = (float)CH, nt_ = na + nb;
+          const float dlt = cmean - st_mean;
+          st_mean = fmaf(dlt, nb / nt_, st_mean);
+          st_m2 = st_m2 + cm2 + dlt * dlt * (na * nb / nt_);
+        }
+        __syncwarp();
+        // ---- copy out: 8 lanes per row, 4 rows per instruction, whole row segments
+        const unsigned long long my_dst = reinterpret_cast<unsigned long long>(dst_row);
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+          const int row = it * 4 + (lane >> 3), ch = lane & 7;
+          const unsigned long long d = __shfl_sync(0xffffffffu, my_dst, row);
+          const int ok = __shfl_sync(0xffffffffu, valid ? 1 : 0, row);
+          if (ok && ch < nchunk) {
+            const uint4 val =
+                *reinterpret_cast<const uint4*>(stg + (row << 7) + ((ch ^ (row & 7)) << 4));
+            *reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(d) + ch * 8) = val;
+          }
+        }
+        __syncwarp();
       }
       if (EPI == EPI_STORE && p.stats_out != nullptr && row_ok)
         p.stats_out[m * p.stats_out_parts + nt * 2 + (ew >> 2)] = make_float2(st_mean, st_m2);
