@@ -97,7 +97,7 @@ def launch_flops(img: int, B: int):
 KIND_CLASS = {"patch_embed": "patch_embed", "unroll_reroll": "unroll_reroll",
               "gemm_qkv_lnfold": "gemm", "gemm_fc1_lnfold_gelu": "gemm",
               "gemm_bias_residual": "gemm", "attention_tiled": "attention",
-              "attention_packed": "attention"}
+              "attention_packed": "attention", "attention_tcgen05": "attention"}
 
 
 class ClockSampler:

@@ -184,10 +184,12 @@ HIERA_API hiera_status hiera_block_forward(const hiera_block_desc* desc, const v
 
 /* Byte offsets of the block's intermediates inside its workspace, for inspection:
  * [0] q, [1] k, [2] v (head-major: bf16 [B][windows][heads][T][64] with channels 56..63
- * zero; f32 token-major [B, tokens, 4*dim_out] holding q|k|v|proj in [0] and -1 in
- * [1],[2]), [3] merged attention output [B, tokens/q_stride, dim_out], [4] transition
- * residual (or -1), [5] x after the attention residual, [6] MLP hidden
- * [B, tokens/q_stride, 4*dim_out]. Returns HIERA_ERR_SHAPE on a bad desc. */
+ * zero, except that v is stored transposed, [B][windows][heads][64][T], when the block's
+ * attention runs on the tensor-core kernel: T_q >= 128 and T_kv >= 128; f32 token-major
+ * [B, tokens, 4*dim_out] holding q|k|v|proj in [0] and -1 in [1],[2]), [3] merged
+ * attention output [B, tokens/q_stride, dim_out], [4] transition residual (or -1), [5] x
+ * after the attention residual, [6] MLP hidden [B, tokens/q_stride, 4*dim_out]. Returns
+ * HIERA_ERR_SHAPE on a bad desc. */
 HIERA_API hiera_status hiera_block_workspace_layout(const hiera_block_desc* desc, long long offsets[7]);
 
 /* --------------------------------------------------------------------------------

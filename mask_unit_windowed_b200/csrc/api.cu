@@ -256,6 +256,8 @@ hiera_status forward_bf16(const Geom& g, const uint8_t* packed, const void* x, v
   a.Tq = g.Tq;
   a.Tkv = g.Tkv;
   a.pooled = g.qs == 4;
+  const bool tc_attn = attention_tc_supported(g.Tq, g.Tkv);
+  a.vt = tc_attn ? 1 : 0;
   HIERA_TRY(launch_tc_gemm(EPI_QKV, a, st));
   // (a7, a8) attention core, heads merged
   AttnArgs at{};
@@ -269,7 +271,7 @@ hiera_status forward_bf16(const Geom& g, const uint8_t* packed, const void* x, v
   at.Tq = g.Tq;
   at.Tkv = g.Tkv;
   at.d_out = g.d_out;
-  HIERA_TRY(launch_attention_bf16(at, st));
+  HIERA_TRY(tc_attn ? launch_attention_tc(at, st) : launch_attention_bf16(at, st));
   // (a9) attention proj + residual
   TcGemmArgs pj{};
   pj.M = (int)qrows;
@@ -898,7 +900,8 @@ const char* hiera_kernel_name(int kind) {
   static const char* names[K_COUNT] = {
       "patch_embed", "unroll_reroll", "gemm_qkv_lnfold", "gemm_fc1_lnfold_gelu",
       "gemm_bias_residual", "attention_tiled", "attention_packed", "f32_gemm",
-      "f32_attention", "f32_row_stats", "pack", "timeout_probe", "row_stats"};
+      "f32_attention", "f32_row_stats", "pack", "timeout_probe", "row_stats",
+      "attention_tcgen05"};
   return (kind >= 0 && kind < K_COUNT) ? names[kind] : "unknown";
 }
 

@@ -1,0 +1,395 @@
+// Tensor-core (tcgen05) attention core for the global-attention blocks ("Phase 4: Hiera
+// Backbone MLX Port", Architecture Summary, MaskUnitAttention with mask_unit_attn=False:
+// scaled dot-product attention over all tokens, heads merged before proj).
+//
+// One CTA = two 128-row query tiles (A and B) of one (image, window, head) unit:
+//   warp 0      TMA: both Q tiles once, then K (128 keys x 64) and V^T (64 x 128 keys) tiles
+//               through a KV_STAGES-deep ring shared by the two query tiles.
+//   warp 1      TMEM owner and MMA issuer: S_t = Q_t K_j^T (M=128, N=128, K=64) and
+//               O_t += P_t V_j (M=128, N=64, K=128) for t = A, B, interleaved so that the
+//               tensor core works on one tile while the other tile's softmax runs.
+//   warps 2-5   softmax of tile A, warps 6-9 of tile B, one query row per thread (TMEM lane
+//               = row): row max, then the weights P = 2^(s log2(e)/sqrt(56) - m) on the
+//               MUFU unit, rounded to bf16 with integer operations (the conversion unit
+//               shares the MUFU pipe) into the PV's A operand in shared memory. The running
+//               max is raised, and O rescaled in TMEM, only when a tile's max exceeds it by
+//               more than 2^8, so P entries stay below 256.
+// head_dim 56 is padded to 64: q/k channels 56..63 are zero; v^T padding row 56 is one, so
+// column 56 of O accumulates the softmax denominator from the very P values the tensor core
+// used; the output is O[:, :56] / O[:, 56].
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace hiera {
+namespace {
+
+constexpr int QT = 128;          // query rows per tile, two tiles per CTA
+constexpr int KT = 128;          // keys per tile
+constexpr int KV_STAGES = 4;
+constexpr int Q_BYTES = QT * 128;                // [128 q][64 ch] bf16
+constexpr int K_BYTES = KT * 128;                // [128 keys][64 ch]
+constexpr int V_BYTES = 2 * 64 * 128;            // two [64 ch][64 keys] blocks of V^T
+constexpr int KV_BYTES = K_BYTES + V_BYTES;
+constexpr int P_BYTES = 2 * QT * 128;            // two [128 q][64 keys] blocks
+constexpr int OFF_Q = 0;                         // Q_A, Q_B
+constexpr int OFF_KV = OFF_Q + 2 * Q_BYTES;
+constexpr int OFF_P = OFF_KV + KV_STAGES * KV_BYTES;  // P_A, P_B
+constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
+constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;
+constexpr uint32_t TMEM_COLS = 512;              // S_A, S_B [0,256), O_A, O_B [256,384)
+constexpr uint32_t O_COL = 256;
+constexpr float RESCALE_LOG2 = 8.f;              // raise the running max past 2^8 only
+
+struct AParams {
+  int Tq, Tkv, nW, heads, d_out;
+  float sl2;  // log2(e) / sqrt(56)
+  bf16* o;
+  uint64_t limit_ns;
+  unsigned int* status;
+};
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const AParams& p,
+                                          volatile int* abort_flag) {
+  int ok = mbar_wait(bar, parity, p.limit_ns, p.status, abort_flag) ? 1 : 0;
+  ok = __all_sync(0xffffffffu, ok);
+  if (!ok) *abort_flag = 1;
+  return ok != 0;
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  tc_ld_32x32b_x32(taddr, r);
+}
+
+__global__ void __launch_bounds__(320, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const AParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  uint8_t* smem = smem_raw + pad;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = kv_full + KV_STAGES;
+  uint64_t* s_full = kv_empty + KV_STAGES;  // [2]: one per query tile
+  uint64_t* s_free = s_full + 2;
+  uint64_t* p_full = s_free + 2;
+  uint64_t* p_free = p_full + 2;
+  uint64_t* o_done = p_free + 2;
+  uint64_t* drain = o_done + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int unit = blockIdx.y;
+  const int q0 = blockIdx.x * 2 * QT;
+  const int n_tiles = (p.Tkv + KT - 1) / KT;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < KV_STAGES; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&s_free[t], 128);
+      mbar_init(&p_full[t], 128);
+      mbar_init(&p_free[t], 1);
+      mbar_init(&o_done[t], 1);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == 1) {
+    tc_alloc(tmem_slot, TMEM_COLS);
+    tc_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, 2 * Q_BYTES);
+      tma_load_3d(smem + OFF_Q, &tmQ, q_full, 0, q0, unit);
+      tma_load_3d(smem + OFF_Q + Q_BYTES, &tmQ, q_full, 0, q0 + QT, unit);
+      long long issued = 0;
+      bool ok = true;
+      for (int j = 0; j < n_tiles; ++j) {
+        const int s = j % KV_STAGES;
+        if (!mbar_wait(&kv_empty[s], (uint32_t)(((j / KV_STAGES) & 1) ^ 1), p.limit_ns, p.status,
+                       abort_flag)) {
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        uint8_t* st = smem + OFF_KV + s * KV_BYTES;
+        mbar_arrive_expect_tx(&kv_full[s], KV_BYTES);
+        tma_load_3d(st, &tmK, &kv_full[s], 0, j * KT, unit);
+        tma_load_3d(st + K_BYTES, &tmV, &kv_full[s], j * KT, 0, unit);
+        tma_load_3d(st + K_BYTES + 64 * 128, &tmV, &kv_full[s], j * KT + 64, 0, unit);
+        ++issued;
+      }
+      mbar_wait(q_full, 0, p.limit_ns, p.status);
+      if (!ok) {
+        for (long long i = issued > KV_STAGES ? issued - KV_STAGES : 0; i < issued; ++i)
+          mbar_wait(&kv_full[i % KV_STAGES], (uint32_t)((i / KV_STAGES) & 1), p.limit_ns,
+                    p.status);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC_S = idesc_bf16_f32(128, KT);
+      constexpr uint32_t IDESC_O = idesc_bf16_f32(128, 64);
+      bool ok = mbar_wait(q_full, 0, p.limit_ns, p.status, abort_flag);
+      tc_fence_after();
+      for (int j = 0; ok && j <= n_tiles; ++j) {
+        if (j < n_tiles) {
+          const int s = j % KV_STAGES;
+          if (!mbar_wait(&kv_full[s], (uint32_t)((j / KV_STAGES) & 1), p.limit_ns, p.status,
+                         abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint64_t kdesc = smem_desc_sw128(smem_u32(smem + OFF_KV + s * KV_BYTES));
+          for (int t = 0; t < 2 && ok; ++t) {
+            // the softmax of tile t has read S_t(j-1) out of TMEM
+            if (j >= 1 && !mbar_wait(&s_free[t], (uint32_t)((j - 1) & 1), p.limit_ns, p.status,
+                                     abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t qdesc = smem_desc_sw128(smem_u32(smem + OFF_Q + t * Q_BYTES));
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              tc_mma_bf16(tmem + (uint32_t)(t * KT), qdesc + (uint64_t)(2 * kk),
+                          kdesc + (uint64_t)(2 * kk), IDESC_S, kk > 0 ? 1u : 0u);
+            tc_commit(&s_full[t]);
+          }
+          if (!ok) break;
+        }
+        if (j >= 1) {
+          const int jj = j - 1, s2 = jj % KV_STAGES;
+          const uint32_t vbase = smem_u32(smem + OFF_KV + s2 * KV_BYTES + K_BYTES);
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (!mbar_wait(&p_full[t], (uint32_t)(jj & 1), p.limit_ns, p.status, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t pbase = smem_u32(smem + OFF_P + t * P_BYTES);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const int blk = kk >> 2, k4 = kk & 3;
+              const uint64_t pd = smem_desc_sw128(pbase + blk * (QT * 128)) + (uint64_t)(2 * k4);
+              const uint64_t vd = smem_desc_sw128(vbase + blk * (64 * 128)) + (uint64_t)(2 * k4);
+              tc_mma_bf16(tmem + O_COL + (uint32_t)(t * 64), pd, vd, IDESC_O,
+                          (jj > 0 || kk > 0) ? 1u : 0u);
+            }
+            tc_commit(&o_done[t]);
+            tc_commit(&p_free[t]);
+          }
+          if (!ok) break;
+          tc_commit(&kv_empty[s2]);
+        }
+      }
+      if (!ok) *abort_flag = 1;
+      tc_commit(drain);
+      mbar_wait(drain, 0, p.limit_ns, p.status);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax (row per thread)
+    const int t = (warp - 2) >> 2;  // query tile of this warpgroup
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t s_col = (uint32_t)(t * KT), o_col = O_COL + (uint32_t)(t * 64);
+    const float sl2 = p.sl2;
+    const float thr = RESCALE_LOG2 / sl2;  // in raw score units
+    float m_run = -INFINITY;
+    bool ok = true;
+    uint8_t* pb = smem + OFF_P + t * P_BYTES + r * 128;
+    for (int j = 0; j < n_tiles; ++j) {
+      if (!warp_wait(&s_full[t], (uint32_t)(j & 1), p, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sr[KT];
+#pragma unroll
+      for (int c = 0; c < KT / 32; ++c)
+        tmem_ld32(lane_base + s_col + (uint32_t)(32 * c),
+                  *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
+      tc_wait_ld();
+#pragma unroll
+      for (int i = 0; i < KT; ++i) asm volatile("" : "+r"(sr[i]));
+      tc_fence_before();
+      mbar_arrive(&s_free[t]);  // S_t may be overwritten from here on
+      const int kv_valid = min(KT, p.Tkv - j * KT);
+      if (kv_valid < KT) {  // ragged last tile: masked keys take no part
+#pragma unroll
+        for (int i = 0; i < KT; ++i)
+          if (i >= kv_valid) sr[i] = __float_as_uint(-INFINITY);
+      }
+      // row max with 8 independent chains
+      float mx[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) mx[u] = __uint_as_float(sr[u]);
+#pragma unroll
+      for (int i = 8; i < KT; i += 8)
+#pragma unroll
+        for (int u = 0; u < 8; ++u) mx[u] = fmaxf(mx[u], __uint_as_float(sr[i + u]));
+      const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      float alpha = 1.f;
+      bool resc = false;
+      if (mt > m_run + thr) {
+        alpha = (m_run == -INFINITY) ? 0.f : ex2_approx((m_run - mt) * sl2);
+        m_run = mt;
+        resc = j > 0;
+      }
+      const float ms = m_run * sl2;
+      // P_t and O_t are free once the PV of tile j-1 has completed
+      if (j >= 1 && !warp_wait(&p_free[t], (uint32_t)((j - 1) & 1), p, abort_flag)) {
+        ok = false;
+        break;
+      }
+#pragma unroll
+      for (int c = 0; c < KT / 8; ++c) {
+        uint4 pk;
+        uint32_t* w4 = reinterpret_cast<uint32_t*>(&pk);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float x0 = fmaf(__uint_as_float(sr[8 * c + 2 * u]), sl2, -ms);   // -inf -> 0
+          const float x1 = fmaf(__uint_as_float(sr[8 * c + 2 * u + 1]), sl2, -ms);
+          w4[u] = pack_bf16x2_int(ex2_approx(x0), ex2_approx(x1));
+        }
+        const int blk = c >> 3, cc = c & 7;
+        *reinterpret_cast<uint4*>(pb + blk * (QT * 128) + ((cc ^ (r & 7)) << 4)) = pk;
+      }
+      if (__any_sync(0xffffffffu, resc)) {
+        // O_t holds the sum through tile j-1 (its PV completed above): rescale these rows
+        tc_fence_after();
+        const float f = resc ? alpha : 1.f;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t ov[32];
+          tmem_ld32(lane_base + o_col + (uint32_t)(32 * c), ov);
+          tc_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            asm volatile("" : "+r"(ov[i]));
+            ov[i] = __float_as_uint(__uint_as_float(ov[i]) * f);
+          }
+          tc_st_32x32b_x32(lane_base + o_col + (uint32_t)(32 * c), ov);
+        }
+        tc_wait_st();
+      }
+      fence_proxy_async_smem();  // P (generic stores) before the tensor core reads it
+      tc_fence_before();
+      mbar_arrive(&p_full[t]);
+    }
+    // ---- normalise and store this row: merged head layout, token j*nW + w. The PV of tile
+    // n-2 is complete (p_free above), so o_done's phase n-1 is the one pending.
+    if (ok && warp_wait(&o_done[t], (uint32_t)((n_tiles - 1) & 1), p, abort_flag)) {
+      tc_fence_after();
+      uint32_t ov[64];
+      tmem_ld32(lane_base + o_col, *reinterpret_cast<uint32_t(*)[32]>(&ov[0]));
+      tmem_ld32(lane_base + o_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&ov[32]));
+      tc_wait_ld();
+#pragma unroll
+      for (int i = 0; i < 64; ++i) asm volatile("" : "+r"(ov[i]));
+      const int qrow = q0 + t * QT + r;
+      if (qrow < p.Tq) {
+        const float inv = 1.f / __uint_as_float(ov[56]);  // softmax denominator (ones row of v)
+        const int h = unit % p.heads;
+        const int w = (unit / p.heads) % p.nW;
+        const int bimg = unit / (p.heads * p.nW);
+        const long long Nq = (long long)p.Tq * p.nW;
+        bf16* dst = p.o + ((long long)bimg * Nq + (long long)qrow * p.nW + w) * p.d_out + h * 56;
+#pragma unroll
+        for (int c = 0; c < 7; ++c) {
+          uint4 pk;
+          pk.x = pack_bf16x2(__uint_as_float(ov[8 * c + 0]) * inv, __uint_as_float(ov[8 * c + 1]) * inv);
+          pk.y = pack_bf16x2(__uint_as_float(ov[8 * c + 2]) * inv, __uint_as_float(ov[8 * c + 3]) * inv);
+          pk.z = pack_bf16x2(__uint_as_float(ov[8 * c + 4]) * inv, __uint_as_float(ov[8 * c + 5]) * inv);
+          pk.w = pack_bf16x2(__uint_as_float(ov[8 * c + 6]) * inv, __uint_as_float(ov[8 * c + 7]) * inv);
+          *reinterpret_cast<uint4*>(dst + 8 * c) = pk;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tc_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+bool attention_tc_supported(int Tq, int Tkv) { return Tq >= 128 && Tkv >= 128 && Tkv % 8 == 0; }
+
+hiera_status launch_attention_tc(const AttnArgs& a, cudaStream_t stream) {
+  const int units = a.B * a.nW * a.heads;
+  if (units <= 0) return HIERA_OK;
+  if (!attention_tc_supported(a.Tq, a.Tkv)) return HIERA_ERR_SHAPE;
+  CUtensorMap tmQ, tmK, tmV;
+  {
+    cuuint64_t dims[3] = {64, (cuuint64_t)a.Tq, (cuuint64_t)units};
+    cuuint64_t str[2] = {128, (cuuint64_t)a.Tq * 128};
+    cuuint32_t box[3] = {64, QT, 1};
+    if (!encode_tmap_bf16_sw128(&tmQ, a.q, 3, dims, str, box)) return HIERA_ERR_CUDA;
+  }
+  {
+    cuuint64_t dims[3] = {64, (cuuint64_t)a.Tkv, (cuuint64_t)units};
+    cuuint64_t str[2] = {128, (cuuint64_t)a.Tkv * 128};
+    cuuint32_t box[3] = {64, KT, 1};
+    if (!encode_tmap_bf16_sw128(&tmK, a.k, 3, dims, str, box)) return HIERA_ERR_CUDA;
+  }
+  {
+    cuuint64_t dims[3] = {(cuuint64_t)a.Tkv, 64, (cuuint64_t)units};
+    cuuint64_t str[2] = {(cuuint64_t)a.Tkv * 2, (cuuint64_t)a.Tkv * 128};
+    cuuint32_t box[3] = {64, 64, 1};
+    if (!encode_tmap_bf16_sw128(&tmV, a.v, 3, dims, str, box)) return HIERA_ERR_CUDA;
+  }
+  AParams p;
+  p.Tq = a.Tq;
+  p.Tkv = a.Tkv;
+  p.nW = a.nW;
+  p.heads = a.heads;
+  p.d_out = a.d_out;
+  p.sl2 = (float)(1.4426950408889634 / sqrt(56.0));
+  p.o = static_cast<bf16*>(a.o);
+  p.limit_ns = g_wait_limit_ns();
+  p.status = g_status_ptr();
+  static bool attr_done[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_done[dev]) {
+    if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SMEM_BYTES) != cudaSuccess)
+      return HIERA_ERR_CUDA;
+    attr_done[dev] = true;
+  }
+  dim3 grid((a.Tq + 2 * QT - 1) / (2 * QT), units);
+  if (grid.y > 65535) return HIERA_ERR_SHAPE;
+  profile_mark(K_ATTN_TC, stream);
+  attn_tc_kernel<<<grid, 320, SMEM_BYTES, stream>>>(tmQ, tmK, tmV, p);
+  return cudaGetLastError() == cudaSuccess ? HIERA_OK : HIERA_ERR_CUDA;
+}
+
+}  // namespace hiera

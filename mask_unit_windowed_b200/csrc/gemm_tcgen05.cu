@@ -53,6 +53,7 @@ struct KParams {
   bf16* v;
   bf16* r;
   int tokens, nW, heads, d_out, Tq, Tkv;
+  int vt;  // 1: v written transposed, [B][nW][heads][64][Tkv]
   uint64_t limit_ns;
   unsigned int* status;
   const float2* stats_in;  // FOLD: [M][stats_parts] partial (mean, M2) of A's rows
@@ -391,6 +392,23 @@ __global__ void __launch_bounds__(320, 1)
             v[8 * g + 7] += bf16_hi(rr.w);
           }
         }
+        if (EPI == EPI_QKV && which == 2 && p.vt) {
+          // v for the tensor-core attention, transposed: channel-major rows of Tkv keys.
+          // Padding row 56 holds ones, so the P V product also yields each query row's
+          // softmax denominator; rows 57..63 are zero. Lanes hold consecutive tokens, so
+          // each store instruction covers a run of keys.
+          if (writer) {
+            const int h = (n0 - 2 * p.d_out + c_begin + c) / 56;
+            const int w = tok % p.nW, j = tok / p.nW;
+            bf16* base = p.v + (((long long)b * p.nW + w) * p.heads + h) * 64 * (long long)p.Tkv + j;
+#pragma unroll
+            for (int e = 0; e < 56; ++e) base[(long long)e * p.Tkv] = __float2bfloat16_rn(v[e]);
+            base[56LL * p.Tkv] = __float2bfloat16_rn(1.f);
+#pragma unroll
+            for (int e = 57; e < 64; ++e) base[(long long)e * p.Tkv] = __float2bfloat16_rn(0.f);
+          }
+          continue;
+        }
         // ---- destination of this lane's row for this chunk
         bf16* dst_row = nullptr;
         bool valid = row_ok;
@@ -507,14 +525,7 @@ EncodeTiledFn get_encode_fn() {
 
 bool encode_bf16(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
                  const cuuint64_t* strides_bytes, const cuuint32_t* box) {
-  EncodeTiledFn fn = get_encode_fn();
-  if (fn == nullptr) return false;
-  cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base),
-                  dims, strides_bytes, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  return encode_tmap_bf16_sw128(map, base, rank, dims, strides_bytes, box);
 }
 
 template <int BN, int EPI, bool FOLD, bool POOLED>
@@ -562,6 +573,7 @@ hiera_status run(const TcGemmArgs& a, cudaStream_t stream) {
   p.d_out = a.d_out;
   p.Tq = a.Tq;
   p.Tkv = a.Tkv;
+  p.vt = a.vt;
   p.limit_ns = g_wait_limit_ns();
   p.status = g_status_ptr();
   p.stats_in = static_cast<const float2*>(a.stats_in);
@@ -591,6 +603,18 @@ hiera_status run(const TcGemmArgs& a, cudaStream_t stream) {
 }
 
 }  // namespace
+
+bool encode_tmap_bf16_sw128(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
+                            const cuuint64_t* strides_bytes, const cuuint32_t* box) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (fn == nullptr) return false;
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base),
+                  dims, strides_bytes, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
 
 hiera_status launch_tc_gemm(int epi, const TcGemmArgs& a, cudaStream_t stream) {
   if (a.M <= 0 || a.N <= 0 || a.K <= 0) return HIERA_OK;

@@ -17,7 +17,7 @@ unsigned int* g_status_ptr();            // device address of the status word (c
 enum KernelId {
   K_PATCH_EMBED = 0, K_PERMUTE = 1, K_GEMM_QKV = 2, K_GEMM_GELU = 3, K_GEMM_STORE = 4,
   K_ATTN_TILED = 5, K_ATTN_PACKED = 6, K_F32_GEMM = 7, K_F32_ATTN = 8, K_F32_STATS = 9,
-  K_PACK = 10, K_PROBE = 11, K_ROW_STATS = 12, K_COUNT = 13
+  K_PACK = 10, K_PROBE = 11, K_ROW_STATS = 12, K_ATTN_TC = 13, K_COUNT = 14
 };
 void profile_mark(int kind, cudaStream_t stream);  // no-op unless a session is open
 
@@ -51,6 +51,8 @@ struct TcGemmArgs {
   void* v;
   void* r;                // transition residual [B, tokens/4, d_out] (columns 3*d_out..)
   int tokens, nW, heads, d_out, Tq, Tkv;
+  int vt;                 // 1: write v transposed, [B][nW][heads][64][Tkv] with padding row
+                          //    56 = 1 (tensor-core attention)
   int pooled;             // 1: rows n, n+T/4, n+T/2, n+3T/4 of each image loaded together and
                           //    q / r columns max-pooled over them (q_stride 4)
 };
@@ -78,6 +80,14 @@ struct AttnArgs {
   int B, nW, heads, Tq, Tkv, d_out;
 };
 hiera_status launch_attention_bf16(const AttnArgs& a, cudaStream_t stream);
+// Tensor-core (tcgen05) attention for Tq >= 128 and Tkv >= 128: q/k as above, v transposed
+// [B][nW][heads][64][Tkv] with row 56 = 1 (a.v), Tkv a multiple of 8.
+bool attention_tc_supported(int Tq, int Tkv);
+hiera_status launch_attention_tc(const AttnArgs& a, cudaStream_t stream);
+
+// TMA descriptor of a bf16 tensor with 128-byte swizzle (cuTensorMapEncodeTiled).
+bool encode_tmap_bf16_sw128(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
+                            const cuuint64_t* strides_bytes, const cuuint32_t* box);
 
 // ---------------------------------------------------------------- fp32 SIMT path
 hiera_status launch_row_stats_f32(const float* x, int M, int K, float eps, float2* stats,
