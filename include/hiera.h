@@ -226,12 +226,13 @@ HIERA_API hiera_status hiera_block_forward_noalloc(const hiera_block_desc* desc,
  *
  * hiera_patch_pack(): patch_w OHWI [112, 7, 7, 4] and patch_b [112] (may be NULL = 0) of
  * `dtype` -> `packed` (caller memory of HIERA_PATCH_PACKED_BYTES bytes): fp32 [196][112]
- * with k = (ky*7 + kx)*4 + c, followed at byte 87808 by the fp32 bias [112].
+ * with k = (ky*7 + kx)*4 + c, then at byte 87808 the fp32 bias [112], then at byte 88256
+ * the weight as bf16 [112][208] (k fastest, zero for k >= 196) for the tensor-core path.
  * hiera_patch_embed(): img NHWC [B, img, img, 4]; pos_embed [(img/4)^2, 112] in raster
  * order; out [B, (img/4)^2, 112] in the unrolled order of hiera_unroll with levels = 3.
  * Padding 3, bias included; img a multiple of 32. fp32 accumulation in both dtypes.
  * -------------------------------------------------------------------------------- */
-#define HIERA_PATCH_PACKED_BYTES ((196 * 112 + 112) * 4)
+#define HIERA_PATCH_PACKED_BYTES ((196 * 112 + 112) * 4 + 112 * 208 * 2)
 HIERA_API hiera_status hiera_patch_pack(const void* patch_w, const void* patch_b, void* packed,
                               hiera_dtype dtype, hiera_stream_t stream);
 HIERA_API hiera_status hiera_patch_embed(const void* img, const void* packed_patch, const void* pos_embed,

@@ -24,7 +24,7 @@ HIERA_F32, HIERA_BF16 = 0, 1
 STATUS = {0: "HIERA_OK", 1: "HIERA_ERR_INVALID_ARG", 2: "HIERA_ERR_SHAPE", 3: "HIERA_ERR_DTYPE",
           4: "HIERA_ERR_ALIGNMENT", 5: "HIERA_ERR_WORKSPACE", 6: "HIERA_ERR_CUDA",
           7: "HIERA_ERR_TIMEOUT", 8: "HIERA_ERR_DEVICE"}
-PATCH_PACKED_BYTES = (196 * 112 + 112) * 4
+PATCH_PACKED_BYTES = (196 * 112 + 112) * 4 + 112 * 208 * 2
 
 
 class HieraError(RuntimeError):

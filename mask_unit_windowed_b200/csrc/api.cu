@@ -462,7 +462,7 @@ BackbonePack backbone_pack_layout(const hiera_backbone_desc* bd, const BlockPlan
   const size_t G0 = bd->img / 4;
   size_t o = 0;
   L.patch_w = o;
-  L.patch_b = o + 196 * 112 * 4;
+  L.patch_b = o + PATCH_OFF_BIAS;
   o = up256(o + HIERA_PATCH_PACKED_BYTES);
   L.pos = o; o = up256(o + G0 * G0 * 112 * es);
   for (int i = 0; i < kDepth; ++i) {
@@ -757,8 +757,7 @@ hiera_status hiera_patch_pack(const void* patch_w, const void* patch_b, void* pa
   if (!aligned16(patch_w) || !aligned16(packed) || (patch_b != nullptr && !aligned16(patch_b)))
     return HIERA_ERR_ALIGNMENT;
   HIERA_TRY(check_device());
-  float* p = static_cast<float*>(packed);
-  return launch_patch_pack(patch_w, patch_b, dtype == HIERA_BF16 ? 1 : 0, p, p + 196 * 112,
+  return launch_patch_pack(patch_w, patch_b, dtype == HIERA_BF16 ? 1 : 0, packed,
                            (cudaStream_t)stream);
 }
 
@@ -773,8 +772,7 @@ hiera_status hiera_patch_embed(const void* img, const void* packed_patch, const 
   if (!aligned16(img) || !aligned16(packed_patch) || !aligned16(pos_embed) || !aligned16(out))
     return HIERA_ERR_ALIGNMENT;
   HIERA_TRY(check_device());
-  const float* p = static_cast<const float*>(packed_patch);
-  return launch_patch_embed(img, p, p + 196 * 112, pos_embed, out, nullptr, B, img_side,
+  return launch_patch_embed(img, packed_patch, pos_embed, out, nullptr, B, img_side,
                             dtype == HIERA_BF16 ? 1 : 0, (cudaStream_t)stream);
 }
 
@@ -805,8 +803,7 @@ hiera_status hiera_backbone_pack(const hiera_backbone_desc* desc, const hiera_ba
   const cudaStream_t st = (cudaStream_t)stream;
   uint8_t* p = static_cast<uint8_t*>(packed);
   const int bf = desc->dtype == HIERA_BF16 ? 1 : 0;
-  HIERA_TRY(launch_patch_pack(w->patch_w, w->patch_b, bf, (float*)(p + L.patch_w),
-                              (float*)(p + L.patch_b), st));
+  HIERA_TRY(launch_patch_pack(w->patch_w, w->patch_b, bf, p + L.patch_w, st));
   const int G0 = desc->img / 4;
   HIERA_TRY(launch_copy_pack(w->pos_embed, nullptr, G0 * G0, 112, bf, p + L.pos, nullptr, st));
   for (int i = 0; i < kDepth; ++i) {
@@ -850,9 +847,8 @@ hiera_status hiera_backbone_forward(const hiera_backbone_desc* desc, const void*
   float2* stp[2] = {(float2*)(ws + W.st0), (float2*)(ws + W.st1)};
   // (a0-a2) patch embedding + pos_embed + Unroll, fused; in bf16 it also emits the LayerNorm
   // partials of its output (two 56-channel halves per token) for block 0's norm1
-  HIERA_TRY(launch_patch_embed(img_nhwc, pk + P.patch_w, (const float*)(pk + P.patch_b),
-                               pk + P.pos, act[0], bf ? stp[0] : nullptr, desc->B, desc->img,
-                               bf, st));
+  HIERA_TRY(launch_patch_embed(img_nhwc, pk + P.patch_w, pk + P.pos, act[0],
+                               bf ? stp[0] : nullptr, desc->B, desc->img, bf, st));
   int cur = 0, s_idx = 0, parts = 2;
   for (int i = 0; i < kDepth; ++i) {
     Geom g;

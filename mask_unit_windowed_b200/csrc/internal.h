@@ -120,12 +120,17 @@ hiera_status launch_fold_pack(const void* w, const void* gamma, const void* beta
                               float* colsum, float* colconst, cudaStream_t stream);
 hiera_status launch_copy_pack(const void* w, const void* bias, int N, int K, int dtype_bf16,
                               void* w_out, float* bias_out, cudaStream_t stream);
-hiera_status launch_patch_pack(const void* w, const void* bias, int dtype_bf16, float* wt,
-                               float* bias_out, cudaStream_t stream);
+// Packed patch-embedding weights (HIERA_PATCH_PACKED_BYTES): fp32 [196][112] (k-major), fp32
+// bias [112], bf16 [112][208] (co-major, k zero-padded to 208).
+constexpr int PATCH_K = 196, PATCH_KP = 208, PATCH_CO = 112;
+constexpr int PATCH_OFF_BIAS = PATCH_K * PATCH_CO * 4;
+constexpr int PATCH_OFF_W16 = PATCH_OFF_BIAS + PATCH_CO * 4;
+hiera_status launch_patch_pack(const void* w, const void* bias, int dtype_bf16, void* packed,
+                               cudaStream_t stream);
 // stats_out (bf16 only, may be nullptr): float2 [B*N][2] partial (mean, M2) of each output
 // token's two 56-channel halves.
-hiera_status launch_patch_embed(const void* img, const void* w, const float* b,
-                                const void* pos, void* out, float2* stats_out, int B,
-                                int img_side, int dtype_bf16, cudaStream_t stream);
+hiera_status launch_patch_embed(const void* img, const void* packed, const void* pos, void* out,
+                                float2* stats_out, int B, int img_side, int dtype_bf16,
+                                cudaStream_t stream);
 
 }  // namespace hiera

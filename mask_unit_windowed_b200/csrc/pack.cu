@@ -74,33 +74,44 @@ __global__ void __launch_bounds__(256) copy_pack_kernel(const T* __restrict__ w,
     bias_out[i] = bias != nullptr ? ld(bias, i) : 0.f;
 }
 
-// OHWI [112][7][7][4] kernel -> fp32 [196][112] (k = (ky*7 + kx)*4 + c), bias -> fp32
+// OHWI [112][7][7][4] kernel -> fp32 [196][112] (k = (ky*7 + kx)*4 + c), bias -> fp32, and
+// a bf16 [112][208] copy (k fastest, zero-padded) for the tensor-core patch embedding
 template <typename T>
 __global__ void __launch_bounds__(256) patch_pack_kernel(const T* __restrict__ w,
-                                                         const T* __restrict__ bias, int cout,
-                                                         int ktot, float* __restrict__ wt,
-                                                         float* __restrict__ bias_out) {
+                                                         const T* __restrict__ bias,
+                                                         float* __restrict__ wt,
+                                                         float* __restrict__ bias_out,
+                                                         bf16* __restrict__ w16) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < cout * ktot) {
-    const int k = i / cout, co = i - (i / cout) * cout;
-    wt[i] = ld(w, (long long)co * ktot + k);
+  if (i < PATCH_CO * PATCH_K) {
+    const int k = i / PATCH_CO, co = i - (i / PATCH_CO) * PATCH_CO;
+    wt[i] = ld(w, (long long)co * PATCH_K + k);
   }
-  if (i < cout) bias_out[i] = bias != nullptr ? ld(bias, i) : 0.f;
+  if (i < PATCH_CO * PATCH_KP) {
+    const int co = i / PATCH_KP, k = i - (i / PATCH_KP) * PATCH_KP;
+    w16[i] = __float2bfloat16_rn(k < PATCH_K ? ld(w, (long long)co * PATCH_K + k) : 0.f);
+  }
+  if (i < PATCH_CO) bias_out[i] = bias != nullptr ? ld(bias, i) : 0.f;
 }
 
 }  // namespace
 
-hiera_status launch_patch_pack(const void* w, const void* bias, int dtype_bf16, float* wt,
-                               float* bias_out, cudaStream_t stream) {
-  const int cout = 112, ktot = 196;
-  const unsigned blocks = (cout * ktot + 255) / 256;
+hiera_status launch_patch_pack(const void* w, const void* bias, int dtype_bf16, void* packed,
+                               cudaStream_t stream) {
+  uint8_t* pk = static_cast<uint8_t*>(packed);
+  float* wt = reinterpret_cast<float*>(pk);
+  float* bias_out = reinterpret_cast<float*>(pk + PATCH_OFF_BIAS);
+  bf16* w16 = reinterpret_cast<bf16*>(pk + PATCH_OFF_W16);
+  const unsigned blocks = (PATCH_CO * PATCH_KP + 255) / 256;
   profile_mark(K_PACK, stream);
   if (dtype_bf16)
-    patch_pack_kernel<bf16><<<blocks, 256, 0, stream>>>(
-        static_cast<const bf16*>(w), static_cast<const bf16*>(bias), cout, ktot, wt, bias_out);
+    patch_pack_kernel<bf16><<<blocks, 256, 0, stream>>>(static_cast<const bf16*>(w),
+                                                        static_cast<const bf16*>(bias), wt,
+                                                        bias_out, w16);
   else
-    patch_pack_kernel<float><<<blocks, 256, 0, stream>>>(
-        static_cast<const float*>(w), static_cast<const float*>(bias), cout, ktot, wt, bias_out);
+    patch_pack_kernel<float><<<blocks, 256, 0, stream>>>(static_cast<const float*>(w),
+                                                         static_cast<const float*>(bias), wt,
+                                                         bias_out, w16);
   return cudaGetLastError() == cudaSuccess ? HIERA_OK : HIERA_ERR_CUDA;
 }
 

@@ -3,12 +3,17 @@
 // [B, N, C]; a learned pos_embed (1, N, 112) is added; Unroll permutes the tokens).
 // Padding 3, so an img x img image gives a (img/4) x (img/4) token grid.
 //
-// A CTA computes ROWS output rows x 128 output columns of one image. Per output row the
-// 7 input rows it needs (x range of the 128 outputs plus the 3-pixel halo) are staged in
-// shared memory as fp32 channel planes; the kernel weights live in shared memory as fp32
-// [196][112] (k = (ky*7 + kx)*4 + c). Thread = (output pixel, half of the 112 channels):
-// 56 fp32 accumulators, weights read as warp-wide broadcasts. The epilogue adds bias and
-// pos_embed[raster token] and stores the row at its unrolled position (3 unroll levels).
+// bf16: an implicit GEMM on the tensor cores (mma.sync m16n8k16, fp32 accumulation): a CTA
+// holds the weight as bf16 [112][208] in shared memory and, per output row, the 7 input rows
+// its 128 output columns need (3-pixel halo, zero outside the image); each warp computes 16
+// output pixels x 112 channels over K = 196 (padded to 208) with A fragments gathered
+// straight from the staged input (the (ky, kx, c) ordering keeps every fragment pair in one
+// 4-byte word). The epilogue stages fp32 results per warp in shared memory; a lane per
+// (pixel, 56-channel half) adds bias and pos_embed[raster token], rounds once to bf16,
+// stores the half row at its unrolled position (3 unroll levels) and, when asked, the
+// LayerNorm partial (mean, M2) of the half for block 0's norm1.
+// fp32: the same computation in fp32 SIMT (weights fp32 [196][112] in shared memory, 56
+// accumulators per thread).
 #include "common.cuh"
 #include "internal.h"
 
@@ -24,24 +29,11 @@ constexpr int SMEM_W = KTOT * COUT * 4;                   // 87808
 constexpr int SMEM_IN = KSZ * CIN * XPITCH * 4;           // 57792
 constexpr int SMEM_TOTAL = SMEM_W + SMEM_IN;
 
-template <typename T>
-__device__ __forceinline__ float to_f(T v);
-template <>
-__device__ __forceinline__ float to_f<float>(float v) {
-  return v;
-}
-template <>
-__device__ __forceinline__ float to_f<bf16>(bf16 v) {
-  return __bfloat162float(v);
-}
-
-template <typename T>
-__global__ void __launch_bounds__(256, 1) patch_embed_kernel(const T* __restrict__ img,
+__global__ void __launch_bounds__(256, 1) patch_embed_kernel(const float* __restrict__ img,
                                                              const float* __restrict__ wt,
                                                              const float* __restrict__ bias,
-                                                             const T* __restrict__ pos,
-                                                             T* __restrict__ out,
-                                                             float2* __restrict__ stats_out,
+                                                             const float* __restrict__ pos,
+                                                             float* __restrict__ out,
                                                              int img_side) {
   extern __shared__ __align__(16) float smem_f[];
   float* sW = smem_f;                 // [196][112]
@@ -66,9 +58,9 @@ __global__ void __launch_bounds__(256, 1) patch_embed_kernel(const T* __restrict
       const int iy = 4 * oy - 3 + ky, ix = 4 * ox0 - 3 + xi;
       float v[CIN] = {0.f, 0.f, 0.f, 0.f};
       if (iy >= 0 && iy < img_side && ix >= 0 && ix < img_side) {
-        const T* src = img + (((long long)b * img_side + iy) * img_side + ix) * CIN;
+        const float* src = img + (((long long)b * img_side + iy) * img_side + ix) * CIN;
 #pragma unroll
-        for (int c = 0; c < CIN; ++c) v[c] = to_f(src[c]);
+        for (int c = 0; c < CIN; ++c) v[c] = src[c];
       }
 #pragma unroll
       for (int c = 0; c < CIN; ++c) sIn[(ky * CIN + c) * XPITCH + xi] = v[c];
@@ -102,67 +94,196 @@ __global__ void __launch_bounds__(256, 1) patch_embed_kernel(const T* __restrict
     if (ox < G) {
       const int t = oy * G + ox;
       const int u = unrolled_of_spatial(oy, ox, 3, M);
-      const T* pr = pos + (long long)t * COUT + half * 56;
-      T* dst = out + ((long long)b * N + u) * COUT + half * 56;
+      const float* pr = pos + (long long)t * COUT + half * 56;
+      float* dst = out + ((long long)b * N + u) * COUT + half * 56;
 #pragma unroll
-      for (int j = 0; j < 56; ++j) {
-        const float v = acc[j] + __ldg(bias + half * 56 + j) + to_f(pr[j]);
-        if constexpr (sizeof(T) == 2) {
-          const bf16 rv = __float2bfloat16_rn(v);
-          dst[j] = rv;
-          acc[j] = __bfloat162float(rv);  // the value as stored, for the statistics below
-        } else {
-          dst[j] = v;
-        }
+      for (int j = 0; j < 56; ++j) dst[j] = acc[j] + __ldg(bias + half * 56 + j) + pr[j];
+    }
+  }
+}
+
+// ---------------------------------------------------------------- bf16 tensor-core path
+constexpr int KP = 208;                 // K padded to 13 k-steps of 16
+constexpr int WPITCH = 216;             // bf16 per weight row in smem (conflict-free fragments)
+constexpr int IN_PITCH = 516;           // pixels per staged input row
+constexpr int OPITCH = 116;             // fp32 per staged output pixel (29 x 16 B: odd)
+constexpr int MMA_ROWS = 4;             // output rows per CTA (weights loaded once)
+constexpr int MMA_SMEM = PATCH_CO * WPITCH * 2 + KSZ * IN_PITCH * CIN * 2 + 8 * 16 * OPITCH * 4;
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1,
+                                               uint32_t a2, uint32_t a3, uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// element offset of (k, local pixel px) in the staged input [ky][x][c]; k even
+__device__ __forceinline__ int in_off(int k, int px) {
+  const int ky = k / 28, rem = k - 28 * ky;
+  return (ky * IN_PITCH + 4 * px + (rem >> 2)) * CIN + (rem & 3);
+}
+
+__global__ void __launch_bounds__(256, 1) patch_embed_mma_kernel(
+    const bf16* __restrict__ img, const bf16* __restrict__ w16, const float* __restrict__ bias,
+    const bf16* __restrict__ pos, bf16* __restrict__ out, float2* __restrict__ stats_out,
+    int img_side) {
+  extern __shared__ __align__(16) uint8_t smem_pe[];
+  bf16* sW = reinterpret_cast<bf16*>(smem_pe);                       // [112][WPITCH]
+  bf16* sIn = sW + PATCH_CO * WPITCH;                                // [7][IN_PITCH][4]
+  float* sOut = reinterpret_cast<float*>(sIn + KSZ * IN_PITCH * CIN);  // [8 warps][16][OPITCH]
+  const int G = img_side / 4;
+  const int M = G / 8;
+  const int N = G * G;
+  const int b = blockIdx.z;
+  const int ox0 = blockIdx.x * SEG;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t4 = lane & 3;
+
+  for (int i = tid; i < PATCH_CO * (KP / 8); i += 256) {
+    const int co = i / (KP / 8), c8 = i - co * (KP / 8);
+    *reinterpret_cast<uint4*>(sW + co * WPITCH + c8 * 8) =
+        __ldg(reinterpret_cast<const uint4*>(w16 + co * KP) + c8);
+  }
+  float* so = sOut + warp * 16 * OPITCH;
+  for (int rr = 0; rr < MMA_ROWS; ++rr) {
+    const int oy = blockIdx.y * MMA_ROWS + rr;
+    if (oy >= G) break;
+    __syncthreads();  // previous row's readers are done with sIn
+    for (int i = tid; i < KSZ * XSPAN; i += 256) {
+      const int ky = i / XSPAN, xi = i - ky * XSPAN;
+      const int iy = 4 * oy - 3 + ky, ix = 4 * ox0 - 3 + xi;
+      uint2 v = make_uint2(0u, 0u);
+      if (iy >= 0 && iy < img_side && ix >= 0 && ix < img_side)
+        v = __ldg(reinterpret_cast<const uint2*>(img + (((long long)b * img_side + iy) * img_side + ix) * CIN));
+      *reinterpret_cast<uint2*>(sIn + (ky * IN_PITCH + xi) * CIN) = v;
+    }
+    __syncthreads();
+    const int px = warp * 16 + g;  // fragment rows g and g + 8
+    float acc[14][4];
+#pragma unroll
+    for (int nt = 0; nt < 14; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll 1
+    for (int ks = 0; ks < KP / 16; ++ks) {
+      const int kA = 16 * ks + 2 * t4, kB = kA + 8;
+      uint32_t a0 = 0, a1 = 0, a2 = 0, a3 = 0;
+      if (kA < PATCH_K) {
+        a0 = *reinterpret_cast<const uint32_t*>(sIn + in_off(kA, px));
+        a1 = *reinterpret_cast<const uint32_t*>(sIn + in_off(kA, px + 8));
       }
-      if (stats_out != nullptr) {
-        // partial (mean, M2) of this half of the token, for the first block's norm1
-        float s = 0.f;
+      if (kB < PATCH_K) {
+        a2 = *reinterpret_cast<const uint32_t*>(sIn + in_off(kB, px));
+        a3 = *reinterpret_cast<const uint32_t*>(sIn + in_off(kB, px + 8));
+      }
 #pragma unroll
-        for (int j = 0; j < 56; ++j) s += acc[j];
-        const float mean = s * (1.f / 56.f);
-        float m2 = 0.f;
-#pragma unroll
-        for (int j = 0; j < 56; ++j) m2 = fmaf(acc[j] - mean, acc[j] - mean, m2);
-        stats_out[((long long)b * N + u) * 2 + half] = make_float2(mean, m2);
+      for (int nt = 0; nt < 14; ++nt) {
+        const bf16* wr = sW + (nt * 8 + g) * WPITCH;
+        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(wr + kA);
+        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(wr + kB);
+        mma_bf16_16816(acc[nt], a0, a1, a2, a3, b0, b1);
       }
     }
+    // stage fp32 (+ bias) per warp: pixel rows g, g + 8; channels 8 nt + 2 t4, +1
+#pragma unroll
+    for (int nt = 0; nt < 14; ++nt) {
+      const int co = nt * 8 + 2 * t4;
+      const float b0 = __ldg(bias + co), b1 = __ldg(bias + co + 1);
+      *reinterpret_cast<float2*>(so + g * OPITCH + co) = make_float2(acc[nt][0] + b0, acc[nt][1] + b1);
+      *reinterpret_cast<float2*>(so + (g + 8) * OPITCH + co) =
+          make_float2(acc[nt][2] + b0, acc[nt][3] + b1);
+    }
+    __syncwarp();
+    // lane = (pixel, half): + pos_embed, one rounding, unrolled store, LayerNorm partial
+    {
+      const int lp = lane >> 1, half = lane & 1;
+      const int ox = ox0 + warp * 16 + lp;
+      if (ox < G) {
+        const int t = oy * G + ox;
+        const int u = unrolled_of_spatial(oy, ox, 3, M);
+        const float* src = so + lp * OPITCH + half * 56;
+        const bf16* pr = pos + (long long)t * PATCH_CO + half * 56;
+        bf16* dst = out + ((long long)b * N + u) * PATCH_CO + half * 56;
+        float vals[56];
+#pragma unroll
+        for (int c8 = 0; c8 < 7; ++c8) {
+          const uint4 pv = __ldg(reinterpret_cast<const uint4*>(pr) + c8);
+          const float4 s0 = *reinterpret_cast<const float4*>(src + 8 * c8);
+          const float4 s1 = *reinterpret_cast<const float4*>(src + 8 * c8 + 4);
+          float v8[8] = {s0.x + bf16_lo(pv.x), s0.y + bf16_hi(pv.x), s0.z + bf16_lo(pv.y),
+                         s0.w + bf16_hi(pv.y), s1.x + bf16_lo(pv.z), s1.y + bf16_hi(pv.z),
+                         s1.z + bf16_lo(pv.w), s1.w + bf16_hi(pv.w)};
+          uint4 pk;
+          pk.x = pack_bf16x2(v8[0], v8[1]);
+          pk.y = pack_bf16x2(v8[2], v8[3]);
+          pk.z = pack_bf16x2(v8[4], v8[5]);
+          pk.w = pack_bf16x2(v8[6], v8[7]);
+          reinterpret_cast<uint4*>(dst)[c8] = pk;
+          vals[8 * c8 + 0] = bf16_lo(pk.x);
+          vals[8 * c8 + 1] = bf16_hi(pk.x);
+          vals[8 * c8 + 2] = bf16_lo(pk.y);
+          vals[8 * c8 + 3] = bf16_hi(pk.y);
+          vals[8 * c8 + 4] = bf16_lo(pk.z);
+          vals[8 * c8 + 5] = bf16_hi(pk.z);
+          vals[8 * c8 + 6] = bf16_lo(pk.w);
+          vals[8 * c8 + 7] = bf16_hi(pk.w);
+        }
+        if (stats_out != nullptr) {
+          float s = 0.f;
+#pragma unroll
+          for (int j = 0; j < 56; ++j) s += vals[j];
+          const float mean = s * (1.f / 56.f);
+          float m2 = 0.f;
+#pragma unroll
+          for (int j = 0; j < 56; ++j) m2 = fmaf(vals[j] - mean, vals[j] - mean, m2);
+          stats_out[((long long)b * N + u) * 2 + half] = make_float2(mean, m2);
+        }
+      }
+    }
+    __syncwarp();
   }
 }
 
 }  // namespace
 
-hiera_status launch_patch_embed(const void* img, const void* w, const float* b, const void* pos,
-                                void* out, float2* stats_out, int B, int img_side,
-                                int dtype_bf16, cudaStream_t stream) {
+hiera_status launch_patch_embed(const void* img, const void* packed, const void* pos, void* out,
+                                float2* stats_out, int B, int img_side, int dtype_bf16,
+                                cudaStream_t stream) {
   const int G = img_side / 4;
-  dim3 grid((G + SEG - 1) / SEG, (G + ROWS - 1) / ROWS, B);
-  if (grid.y > 65535 || grid.z > 65535) return HIERA_ERR_SHAPE;
+  const uint8_t* pk = static_cast<const uint8_t*>(packed);
+  const float* wt = reinterpret_cast<const float*>(pk);
+  const float* bias = reinterpret_cast<const float*>(pk + PATCH_OFF_BIAS);
+  const bf16* w16 = reinterpret_cast<const bf16*>(pk + PATCH_OFF_W16);
   static bool attr_done[2][64] = {{false}};
   int dev = 0;
   cudaGetDevice(&dev);
   profile_mark(K_PATCH_EMBED, stream);
   if (dtype_bf16) {
+    dim3 grid((G + SEG - 1) / SEG, (G + MMA_ROWS - 1) / MMA_ROWS, B);
+    if (grid.y > 65535 || grid.z > 65535) return HIERA_ERR_SHAPE;
     if (dev < 64 && !attr_done[1][dev]) {
-      if (cudaFuncSetAttribute(patch_embed_kernel<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               SMEM_TOTAL) != cudaSuccess)
+      if (cudaFuncSetAttribute(patch_embed_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               MMA_SMEM) != cudaSuccess)
         return HIERA_ERR_CUDA;
       attr_done[1][dev] = true;
     }
-    patch_embed_kernel<bf16><<<grid, 256, SMEM_TOTAL, stream>>>(
-        static_cast<const bf16*>(img), static_cast<const float*>(w), b,
-        static_cast<const bf16*>(pos), static_cast<bf16*>(out), stats_out, img_side);
+    patch_embed_mma_kernel<<<grid, 256, MMA_SMEM, stream>>>(
+        static_cast<const bf16*>(img), w16, bias, static_cast<const bf16*>(pos),
+        static_cast<bf16*>(out), stats_out, img_side);
   } else {
+    dim3 grid((G + SEG - 1) / SEG, (G + ROWS - 1) / ROWS, B);
+    if (grid.y > 65535 || grid.z > 65535) return HIERA_ERR_SHAPE;
     if (dev < 64 && !attr_done[0][dev]) {
-      if (cudaFuncSetAttribute(patch_embed_kernel<float>,
+      if (cudaFuncSetAttribute(patch_embed_kernel,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                SMEM_TOTAL) != cudaSuccess)
         return HIERA_ERR_CUDA;
       attr_done[0][dev] = true;
     }
-    patch_embed_kernel<float><<<grid, 256, SMEM_TOTAL, stream>>>(
-        static_cast<const float*>(img), static_cast<const float*>(w), b,
-        static_cast<const float*>(pos), static_cast<float*>(out), nullptr, img_side);
+    patch_embed_kernel<<<grid, 256, SMEM_TOTAL, stream>>>(
+        static_cast<const float*>(img), wt, bias, static_cast<const float*>(pos),
+        static_cast<float*>(out), img_side);
   }
   return cudaGetLastError() == cudaSuccess ? HIERA_OK : HIERA_ERR_CUDA;
 }
