@@ -60,9 +60,10 @@ def peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
-def launch_flops(img: int, B: int):
+def launch_flops(img: int, B: int, fused_mlp: bool = True):
     """Algorithmic FLOPs of every library launch of one backbone forward, in launch order
-    (head_dim 56, not the padded 64). Returns list of (kind-class, flops, bytes_hint)."""
+    (head_dim 56, not the padded 64). Returns list of (kind-class, flops). With fused_mlp,
+    the MLPs of dims 112 and 224 are one launch (fc1 + fc2 FLOPs)."""
     G0 = img // 4
     out = [("patch_embed", 2.0 * B * G0 * G0 * 112 * 196)]
     prev = STAGE_DIMS[0]
@@ -85,8 +86,11 @@ def launch_flops(img: int, B: int):
             out.append(("gemm", 2.0 * B * n_in * d_in * n1))
             out.append(("attention", 4.0 * B * STAGE_HEADS[s] * nW * tq * tkv * HD))
             out.append(("gemm", 2.0 * B * nq * d * d))
-            out.append(("gemm", 2.0 * B * nq * d * 4 * d))
-            out.append(("gemm", 2.0 * B * nq * 4 * d * d))
+            if fused_mlp and d in (112, 224):
+                out.append(("gemm", 4.0 * B * nq * d * 4 * d))
+            else:
+                out.append(("gemm", 2.0 * B * nq * d * 4 * d))
+                out.append(("gemm", 2.0 * B * nq * 4 * d * d))
             if i in (1, 4, 20, 23):
                 out.append(("unroll_reroll", 0.0))
             i += 1
@@ -97,7 +101,8 @@ def launch_flops(img: int, B: int):
 KIND_CLASS = {"patch_embed": "patch_embed", "unroll_reroll": "unroll_reroll",
               "gemm_qkv_lnfold": "gemm", "gemm_fc1_lnfold_gelu": "gemm",
               "gemm_bias_residual": "gemm", "attention_tiled": "attention",
-              "attention_packed": "attention", "attention_tcgen05": "attention"}
+              "attention_packed": "attention", "attention_tcgen05": "attention",
+              "mlp_fused": "gemm"}
 
 
 class ClockSampler:
@@ -211,6 +216,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
+    hb.set_option(hb.OPT_FUSED_MLP, 1 if args.mlp == "fused" else 0)
     hbm_gbs, tf_burst, tf_sust, peak_src = peaks()
     B = args.batch
 
@@ -303,22 +309,24 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             per_launch = [(n, ms) for n, ms in d] if per_launch is None else \
                 [(n, a + ms) for (n, a), (_, ms) in zip(per_launch, d)]
     per_launch = [(n, ms / reps) for n, ms in per_launch]
-    flops = launch_flops(IMG, B)
+    flops = launch_flops(IMG, B, fused_mlp=hb.get_option(hb.OPT_FUSED_MLP) == 1)
     classes = {}
+    by_kernel = {}
     if len(flops) == len(per_launch) and all(KIND_CLASS.get(n) == c for (n, _), (c, _) in
                                              zip(per_launch, flops)):
         for (n, ms), (c, fl) in zip(per_launch, flops):
-            e = classes.setdefault(c, {"launches": 0, "ms": 0.0, "gflop": 0.0})
-            e["launches"] += 1
-            e["ms"] += ms
-            e["gflop"] += fl / 1e9
+            for e in (classes.setdefault(c, {"launches": 0, "ms": 0.0, "gflop": 0.0}),
+                      by_kernel.setdefault(n, {"launches": 0, "ms": 0.0, "gflop": 0.0})):
+                e["launches"] += 1
+                e["ms"] += ms
+                e["gflop"] += fl / 1e9
     else:
         for n, ms in per_launch:
             e = classes.setdefault(KIND_CLASS.get(n, n), {"launches": 0, "ms": 0.0, "gflop": 0.0})
             e["launches"] += 1
             e["ms"] += ms
     step_ms_prof = sum(ms for _, ms in per_launch)
-    for c, e in classes.items():
+    for e in list(classes.values()) + list(by_kernel.values()):
         e["share"] = e["ms"] / step_ms_prof if step_ms_prof > 0 else None
         e["tflops"] = e["gflop"] / e["ms"] if e["ms"] > 0 else 0.0
         e["frac_of_bf16_sustained"] = e["tflops"] / tf_sust
@@ -326,7 +334,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                    key=lambda c: classes[c]["ms"])
     dom = classes[dominant]
     attn_gemm_gflop = sum(fl for c, fl in flops if c in ("gemm", "attention")) / 1e9
-    roofline = {"bound": "tensor", "kernel": {"gemm": "tcgen05 GEMM (all Linear layers)",
+    roofline = {"bound": "tensor", "kernel": {"gemm": "tcgen05 GEMM + fused MLP (all Linear layers)",
                                               "attention": "mask-unit / global attention"}
                 [dominant],
                 "achieved": dom["tflops"], "peak": tf_sust, "unit": "TFLOP/s",
@@ -384,12 +392,14 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                    "img": IMG, "batch_per_gpu": B, "global_batch": B * world,
                    "parallelism": f"replicas x{world} (no data-path collective)",
                    "l2": "flushed before every step (256 MiB write)",
-                   "timing": "CUDA-graph replay of the library launches, per-step CUDA events"},
+                   "timing": "CUDA-graph replay of the library launches, per-step CUDA events",
+                   "mlp": args.mlp},
         "tflops": gflop_per_image * images / (total_ms * 1e-3) * 1e-3,
         "attn_gemm_frac_of_bf16_peak": attn_gemm_gflop / (ms_per_step * 1e-3) / 1e3 / tf_sust,
         "gflop_per_image": gflop_per_image,
         "roofline": roofline,
         "kernels": classes,
+        "by_kernel": by_kernel,
         "cpu_baseline": cpu,
         "e2e": e2e,
         "clocks": clocks.record(),
@@ -409,6 +419,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=30)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mlp", choices=["fused", "unfused"], default="fused",
+                    help="stage-0/1 MLPs as one fused kernel (default) or two GEMMs")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

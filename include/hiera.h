@@ -271,6 +271,23 @@ HIERA_API hiera_status hiera_backbone_forward(const hiera_backbone_desc* desc, c
                                     size_t workspace_bytes, hiera_stream_t stream);
 
 /* --------------------------------------------------------------------------------
+ * Library options (process-wide, host-side; read when a forward call enqueues its
+ * launches, so change them between calls, not while another thread is enqueuing).
+ *   HIERA_OPT_FUSED_MLP  1 (default): for bf16 blocks with dim_out 112 or 224 (stages 0
+ *                        and 1), norm2 + fc1 + GELU + fc2 + residual run as one kernel
+ *                        that keeps the 4*dim hidden activation on chip (the block's
+ *                        HieraMLP, "Phase 4: Hiera Backbone MLX Port", Architecture
+ *                        Summary). 0: the two stand-alone GEMMs with the hidden
+ *                        activation in the workspace. Both give the same values (same
+ *                        tensor-core K order, same epilogue arithmetic).
+ * hiera_set_option returns HIERA_ERR_INVALID_ARG for an unknown option or value;
+ * hiera_get_option returns the current value (0 for an unknown option).
+ * -------------------------------------------------------------------------------- */
+typedef enum { HIERA_OPT_FUSED_MLP = 0, HIERA_OPT_COUNT = 1 } hiera_option;
+HIERA_API hiera_status hiera_set_option(hiera_option opt, int value);
+HIERA_API int hiera_get_option(hiera_option opt);
+
+/* --------------------------------------------------------------------------------
  * Launch profiling (host-side bookkeeping only). Between hiera_profile_begin() and
  * hiera_profile_end(), every kernel launch the library makes, on whatever stream the
  * call was given, is preceded by cudaEventRecord(events[i], stream) and its kernel id is
@@ -294,7 +311,8 @@ HIERA_API const char* hiera_kernel_name(int kind);
 HIERA_API hiera_status hiera_debug_timeout_probe(int limit_us, hiera_stream_t stream);
 
 /* Self-test of the tensor-core path's GELU: y[i] = GELU(x[i]) for n fp32 device values,
- * computed exactly as the fc1 epilogue does (erf after Abramowitz & Stegun eq. 7.1.28). */
+ * computed exactly as the fc1 epilogue does (x * sigmoid of a fitted odd polynomial for
+ * logit(Phi(x)); |error| <= 3e-5 against x Phi(x)). */
 HIERA_API hiera_status hiera_debug_gelu(const float* x, float* y, int n, hiera_stream_t stream);
 
 #ifdef __cplusplus

@@ -105,6 +105,8 @@ def lib() -> ctypes.CDLL:
                                      ctypes.POINTER(ctypes.c_int)], I),
             "hiera_profile_end": ([P], I),
             "hiera_kernel_name": ([I], ctypes.c_char_p),
+            "hiera_set_option": ([I, I], I),
+            "hiera_get_option": ([I], I),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -381,6 +383,34 @@ def status_string(code: int) -> str:
 
 def kernel_name(kind: int) -> str:
     return lib().hiera_kernel_name(kind).decode()
+
+
+# ----------------------------------------------------------------------------- options
+OPT_FUSED_MLP = 0
+
+
+def set_option(opt: int, value: int):
+    _check(lib().hiera_set_option(opt, int(value)), "hiera_set_option")
+
+
+def get_option(opt: int) -> int:
+    return lib().hiera_get_option(opt)
+
+
+class fused_mlp:
+    """Context manager: run the block MLPs fused (True, the default) or as two GEMMs."""
+
+    def __init__(self, enabled: bool):
+        self.enabled = bool(enabled)
+
+    def __enter__(self):
+        self._old = get_option(OPT_FUSED_MLP)
+        set_option(OPT_FUSED_MLP, int(self.enabled))
+        return self
+
+    def __exit__(self, *exc):
+        set_option(OPT_FUSED_MLP, self._old)
+        return False
 
 
 class LaunchProfile:

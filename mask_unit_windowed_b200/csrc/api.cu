@@ -286,6 +286,24 @@ hiera_status forward_bf16(const Geom& g, const uint8_t* packed, const void* x, v
   pj.stats_out = ws + W.st2;
   pj.stats_out_parts = parts_out;
   HIERA_TRY(launch_tc_gemm(EPI_STORE, pj, st));
+  if (g_option(HIERA_OPT_FUSED_MLP) && mlp_fused_supported(g.d_out) && parts_out == 2) {
+    // (a10-a12) norm2 + fc1 + GELU + fc2 + residual in one kernel, hidden kept on chip
+    MlpArgs ml{};
+    ml.M = (int)qrows;
+    ml.D = g.d_out;
+    ml.x = ws + W.x1;
+    ml.w1 = packed + P.W2;
+    ml.colsum1 = (const float*)(packed + P.s2);
+    ml.colconst1 = (const float*)(packed + P.c2);
+    ml.w2 = packed + P.W3;
+    ml.bias2 = (const float*)(packed + P.b3);
+    ml.stats_in = ws + W.st2;
+    ml.stats_parts = parts_out;
+    ml.ln_eps = g.eps;
+    ml.out = y;
+    ml.stats_out = stats_y;
+    return launch_mlp_fused(ml, st);
+  }
   // (a10, a11) norm2 + fc1 + GELU
   TcGemmArgs f1{};
   f1.M = (int)qrows;
@@ -576,6 +594,12 @@ void profile_mark(int kind, cudaStream_t stream) {
   }
   ++g_prof.count;
 }
+
+namespace {
+int g_options[HIERA_OPT_COUNT] = {1};  // HIERA_OPT_FUSED_MLP on
+}  // namespace
+
+int g_option(int opt) { return (opt >= 0 && opt < HIERA_OPT_COUNT) ? g_options[opt] : 0; }
 
 uint64_t g_wait_limit_ns() {
   static uint64_t limit = [] {
@@ -892,12 +916,21 @@ int hiera_profile_end(hiera_stream_t stream) {
   return g_prof.count;
 }
 
+hiera_status hiera_set_option(hiera_option opt, int value) {
+  if (opt < 0 || opt >= HIERA_OPT_COUNT) return HIERA_ERR_INVALID_ARG;
+  if (opt == HIERA_OPT_FUSED_MLP && value != 0 && value != 1) return HIERA_ERR_INVALID_ARG;
+  g_options[opt] = value;
+  return HIERA_OK;
+}
+
+int hiera_get_option(hiera_option opt) { return g_option(opt); }
+
 const char* hiera_kernel_name(int kind) {
   static const char* names[K_COUNT] = {
       "patch_embed", "unroll_reroll", "gemm_qkv_lnfold", "gemm_fc1_lnfold_gelu",
       "gemm_bias_residual", "attention_tiled", "attention_packed", "f32_gemm",
       "f32_attention", "f32_row_stats", "pack", "timeout_probe", "row_stats",
-      "attention_tcgen05"};
+      "attention_tcgen05", "mlp_fused"};
   return (kind >= 0 && kind < K_COUNT) ? names[kind] : "unknown";
 }
 

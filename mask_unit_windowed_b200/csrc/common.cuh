@@ -282,32 +282,91 @@ __device__ __forceinline__ float gelu_erf(float x) {
   return 0.5f * x * (1.0f + erff(x * 0.70710678118654752440f));
 }
 
-// erf by Abramowitz & Stegun, Handbook of Mathematical Functions, eq. 7.1.28 (after
-// Hastings): for x >= 0, erf(x) = 1 - (1 + a1 x + ... + a6 x^6)^-16 with |error| <= 3e-7.
-// One approximate reciprocal (MUFU) and FMAs; the 16th power by four squarings, so large
-// x underflows cleanly to erf = 1. Odd extension for x < 0.
-__device__ __forceinline__ float erf_as7128(float x) {
-  const float ax = fabsf(x);
-  float p = fmaf(0.0000430638f, ax, 0.0002765672f);
-  p = fmaf(p, ax, 0.0001520143f);
-  p = fmaf(p, ax, 0.0092705272f);
-  p = fmaf(p, ax, 0.0422820123f);
-  p = fmaf(p, ax, 0.0705230784f);
-  p = fmaf(p, ax, 1.0f);
+// GELU(x) = x Phi(x) = x sigmoid(g(x)) with g = logit(Phi). g is odd; it is approximated by
+// x (c0 + c1 x^2 + c2 x^4), a minimax fit (made for this library, weighted by dGELU/dg) of
+// c0 = 1.5950153, c1 = 0.074011831, c2 = -7.0316069e-4, with x^2 clamped at 36: past
+// |x| = 6 the sigmoid is 0 or 1 to fp32 precision and the clamp keeps the polynomial
+// positive. Max |GELU error| 2.6e-5 over the real line, far below bf16 resolution of the
+// stored result. Two MUFU operations (ex2.approx, rcp.approx) and five FP32 operations per
+// element; exp(-g) overflowing to +inf gives x * 0. The constants below are -c_k log2(e).
+// Used by the bf16 tensor-core path.
+__device__ __forceinline__ float gelu_fast(float x) {
+  const float x2 = fminf(x * x, 36.0f);
+  float p = fmaf(1.014446490e-03f, x2, -1.067765057e-01f);
+  p = fmaf(p, x2, -2.301120758e+00f);
+  const float e = ex2_approx(x * p);  // exp(-g(x))
   float r;
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(p));
-  r = r * r;
-  r = r * r;
-  r = r * r;
-  r = r * r;
-  return copysignf(1.0f - r, x);
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.0f + e));
+  return x * r;
 }
 
-// GELU(x) = x * Phi(x) = 0.5 x (1 + erf(x / sqrt 2)) with the erf above (|error| of the
-// result <= ~1e-6 |x|, far below bf16 resolution). Used by the bf16 tensor-core path.
-__device__ __forceinline__ float gelu_fast(float x) {
-  const float e = erf_as7128(x * 0.70710678118654752440f);
-  return fmaf(0.5f * x, e, 0.5f * x);
+// ------------------------------------------------------------------ tcgen05 epilogue helpers
+// Every lane observes the barrier phase itself (so each has acquired the producer's
+// writes), then the warp agrees on the outcome so that it stays converged for the
+// .sync.aligned tcgen05 instructions that follow.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint64_t limit,
+                                          unsigned int* status, volatile int* abort_flag) {
+  int ok = mbar_wait(bar, parity, limit, status, abort_flag) ? 1 : 0;
+  ok = __all_sync(0xffffffffu, ok);
+  if (!ok) *abort_flag = 1;
+  return ok != 0;
+}
+
+// CH consecutive accumulator columns of this thread's TMEM lane, one wait.
+template <int CH>
+__device__ __forceinline__ void tmem_load(uint32_t taddr, uint32_t (&r)[CH]) {
+  if constexpr (CH == 56) {
+    tc_ld_32x32b_x32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+    tc_ld_32x32b_x16(taddr + 32, *reinterpret_cast<uint32_t(*)[16]>(&r[32]));
+    tc_ld_32x32b_x8(taddr + 48, *reinterpret_cast<uint32_t(*)[8]>(&r[48]));
+  } else if constexpr (CH == 32) {
+    tc_ld_32x32b_x32(taddr, r);
+  } else if constexpr (CH == 16) {
+    tc_ld_32x32b_x16(taddr, r);
+  } else {
+    static_assert(CH == 8, "chunk");
+    tc_ld_32x32b_x8(taddr, r);
+  }
+  tc_wait_ld();
+  // tcgen05.ld fills its registers asynchronously; only after tcgen05.wait::ld are they
+  // valid. Re-define each one after the wait so no use can be scheduled above it.
+#pragma unroll
+  for (int i = 0; i < CH; ++i) asm volatile("" : "+r"(r[i]));
+}
+
+__device__ __forceinline__ uint4 pack8(const float* v) {
+  uint4 pk;
+  pk.x = pack_bf16x2(v[0], v[1]);
+  pk.y = pack_bf16x2(v[2], v[3]);
+  pk.z = pack_bf16x2(v[4], v[5]);
+  pk.w = pack_bf16x2(v[6], v[7]);
+  return pk;
+}
+
+// LayerNorm of a row of K values from P partial (mean, M2) pairs over K / P values each
+// (Chan et al. merge with equal counts): LN(x) W^T + b = fa (x W'^T) + fb s + c with
+// fa = rstd, fb = -mean rstd (s, c the packed column constants of the folded weight).
+__device__ __forceinline__ void ln_fold_coeffs(const float2* __restrict__ sp, int P, int K,
+                                               float eps, float& fa, float& fb) {
+  float2 part[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) part[j] = j < P ? __ldg(sp + j) : make_float2(0.f, 0.f);
+  float mean = 0.f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) mean += part[j].x;
+  mean /= (float)P;
+  float m2 = 0.f, dev2 = 0.f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    if (j < P) {
+      const float dlt = part[j].x - mean;
+      m2 += part[j].y;
+      dev2 = fmaf(dlt, dlt, dev2);
+    }
+  }
+  m2 = fmaf((float)(K / P), dev2, m2);
+  fa = rsqrtf(m2 / (float)K + eps);
+  fb = -mean * fa;
 }
 
 // ------------------------------------------------------------------ Unroll map

@@ -86,48 +86,6 @@ struct Cfg {
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
-// Every lane observes the barrier phase itself (so each has acquired the producer's
-// writes), then the warp agrees on the outcome so that it stays converged for the
-// .sync.aligned tcgen05 instructions that follow.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint64_t limit,
-                                          unsigned int* status, volatile int* abort_flag) {
-  int ok = mbar_wait(bar, parity, limit, status, abort_flag) ? 1 : 0;
-  ok = __all_sync(0xffffffffu, ok);
-  if (!ok) *abort_flag = 1;
-  return ok != 0;
-}
-
-// CH consecutive accumulator columns of this thread's TMEM lane, one wait.
-template <int CH>
-__device__ __forceinline__ void tmem_load(uint32_t taddr, uint32_t (&r)[CH]) {
-  if constexpr (CH == 56) {
-    tc_ld_32x32b_x32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-    tc_ld_32x32b_x16(taddr + 32, *reinterpret_cast<uint32_t(*)[16]>(&r[32]));
-    tc_ld_32x32b_x8(taddr + 48, *reinterpret_cast<uint32_t(*)[8]>(&r[48]));
-  } else if constexpr (CH == 32) {
-    tc_ld_32x32b_x32(taddr, r);
-  } else if constexpr (CH == 16) {
-    tc_ld_32x32b_x16(taddr, r);
-  } else {
-    static_assert(CH == 8, "chunk");
-    tc_ld_32x32b_x8(taddr, r);
-  }
-  tc_wait_ld();
-  // tcgen05.ld fills its registers asynchronously; only after tcgen05.wait::ld are they
-  // valid. Re-define each one after the wait so no use can be scheduled above it.
-#pragma unroll
-  for (int i = 0; i < CH; ++i) asm volatile("" : "+r"(r[i]));
-}
-
-__device__ __forceinline__ uint4 pack8(const float* v) {
-  uint4 pk;
-  pk.x = pack_bf16x2(v[0], v[1]);
-  pk.y = pack_bf16x2(v[2], v[3]);
-  pk.z = pack_bf16x2(v[4], v[5]);
-  pk.w = pack_bf16x2(v[6], v[7]);
-  return pk;
-}
-
 template <int BN, int EPI, bool FOLD, bool POOLED>
 __global__ void __launch_bounds__(320, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -316,29 +274,7 @@ __global__ void __launch_bounds__(320, 1)
       }
       // LayerNorm statistics of this row, merged from the producer's partials
       float fa = 1.f, fb = 0.f;  // v = fa * acc + fb * colsum + colconst
-      if (FOLD && row_ok) {
-        const int P = p.stats_parts;
-        const float2* sp = p.stats_in + m * P;
-        float2 part[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) part[j] = j < P ? __ldg(sp + j) : make_float2(0.f, 0.f);
-        float mean = 0.f;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) mean += part[j].x;
-        mean /= (float)P;
-        float m2 = 0.f, dev2 = 0.f;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (j < P) {
-            const float dlt = part[j].x - mean;
-            m2 += part[j].y;
-            dev2 = fmaf(dlt, dlt, dev2);
-          }
-        }
-        m2 = fmaf((float)(p.K / P), dev2, m2);   // Chan et al., equal counts K / P
-        fa = rsqrtf(m2 / (float)p.K + p.ln_eps);
-        fb = -mean * fa;
-      }
+      if (FOLD && row_ok) ln_fold_coeffs(p.stats_in + m * p.stats_parts, p.stats_parts, p.K, p.ln_eps, fa, fb);
       // per-column constants of this tile into shared memory
       named_bar_sync(1, EPI_THREADS);  // every epilogue thread is done with the last tile's
       for (int i = etid; i < BN; i += EPI_THREADS) {

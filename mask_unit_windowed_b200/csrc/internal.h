@@ -17,7 +17,7 @@ unsigned int* g_status_ptr();            // device address of the status word (c
 enum KernelId {
   K_PATCH_EMBED = 0, K_PERMUTE = 1, K_GEMM_QKV = 2, K_GEMM_GELU = 3, K_GEMM_STORE = 4,
   K_ATTN_TILED = 5, K_ATTN_PACKED = 6, K_F32_GEMM = 7, K_F32_ATTN = 8, K_F32_STATS = 9,
-  K_PACK = 10, K_PROBE = 11, K_ROW_STATS = 12, K_ATTN_TC = 13, K_COUNT = 14
+  K_PACK = 10, K_PROBE = 11, K_ROW_STATS = 12, K_ATTN_TC = 13, K_MLP_FUSED = 14, K_COUNT = 15
 };
 void profile_mark(int kind, cudaStream_t stream);  // no-op unless a session is open
 
@@ -58,6 +58,26 @@ struct TcGemmArgs {
 };
 
 hiera_status launch_tc_gemm(int epi, const TcGemmArgs& a, cudaStream_t stream);
+
+// ---------------------------------------------------------------- fused MLP (bf16, tcgen05)
+// out = x + GELU(LN(x) W1'^T folded) W2^T + b2 with the hidden kept on chip (D = 112, 224)
+struct MlpArgs {
+  int M, D;
+  const void* x;            // bf16 [M, D] input and residual
+  const void* w1;           // bf16 [4D, D] LayerNorm-folded fc1 weight
+  const float* colsum1;     // [4D]
+  const float* colconst1;   // [4D]
+  const void* w2;           // bf16 [D, 4D]
+  const float* bias2;       // [D]
+  const void* stats_in;     // float2 [M][stats_parts] partials of x's rows
+  int stats_parts;
+  float ln_eps;
+  void* out;                // bf16 [M, D]
+  void* stats_out;          // float2 [M][2] partials of out (row halves), or nullptr
+};
+bool mlp_fused_supported(int d);
+hiera_status launch_mlp_fused(const MlpArgs& a, cudaStream_t stream);
+int g_option(int opt);      // library options (hiera_set_option)
 
 // N-tile width the plain-store GEMM uses for N output columns (N a multiple of 16).
 inline int store_bn(int N) {

@@ -31,12 +31,18 @@ def test_workspace_too_small_rejected():
 
 
 def test_tensor_core_path_gelu_within_error_bound():
-    """The fc1 epilogue's GELU (erf by Abramowitz & Stegun 7.1.28, |erf error| <= 3e-7)
-    against the fp64 definition x * Phi(x)."""
+    """The fc1 epilogue's GELU (x * sigmoid of a fitted odd polynomial for logit(Phi);
+    fit error 2.55e-5 at most, evaluated in fp32 with ex2.approx / rcp.approx) against the
+    fp64 definition x * Phi(x): |error| <= 3e-5 everywhere, 0 at x = 0, x to 2^-22 for
+    x >= 6 and within 2e-8 of 0 for x <= -6."""
     import numpy as np
     from oracle import unrolled as U
     x = np.linspace(-12, 12, 200001).astype(np.float32)
     y = hb.debug_gelu(torch.from_numpy(x).cuda()).cpu().numpy().astype(np.float64)
     ref = U.gelu(x.astype(np.float64))
     err = np.abs(y - ref)
-    assert np.all(err <= 1e-6 + 1e-6 * np.abs(x)), float(err.max())
+    assert np.all(err <= 3e-5), float(err.max())
+    assert y[np.argmin(np.abs(x))] == 0.0
+    hi = x >= 6
+    assert np.all(np.abs(y[hi] - x[hi]) <= 2.0 ** -22 * x[hi])
+    assert np.all(np.abs(y[x <= -6]) <= 2e-8)
