@@ -212,6 +212,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     import torch.distributed as dist
 
     from mask_unit_windowed_b200 import binding as hb
+    from mask_unit_windowed_b200 import replicas
     from mask_unit_windowed_b200 import synthetic as syn
 
     torch.cuda.set_device(local_rank)
@@ -289,12 +290,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     st = hb.device_status(stream)
     if st != 0:
         raise RuntimeError(f"device status after timing: {hb.status_string(st)}")
-    if world > 1:
-        tt = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = replicas.max_over_ranks(total_ms, dev)
     images = B * args.steps * world
-    value = images / (total_ms / 1000.0)
+    value = replicas.job_throughput(B * args.steps, world, total_ms)
     ms_per_step = total_ms / args.steps
 
     # ---- per-kernel breakdown from the instrumented graph (same workload, L2 flushed)
@@ -363,11 +361,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                     ee[k - 2].record(stream)
         torch.cuda.synchronize()
         e2e_ms = sum(s.elapsed_time(e) for s, e in zip(es, ee))
-        if world > 1:
-            tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e2e_ms = float(tt.item())
-        e2e = {"value": B * args.e2e_steps * world / (e2e_ms / 1000.0), "unit": UNIT,
+        e2e_ms = replicas.max_over_ranks(e2e_ms, dev)
+        e2e = {"value": replicas.job_throughput(B * args.e2e_steps, world, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": img.numel() * img.element_size(),
                "d2h_bytes_per_step": sum(f.numel() * f.element_size() for f in feats),
                "steps": args.e2e_steps,

@@ -20,10 +20,16 @@
 // stand-alone fc1 (K = D in steps of 16) and fc2 (K = 4 D in steps of 16) GEMMs, and the
 // fold / GELU / rounding code is shared, so the result is the same as the unfused pair's.
 //
-// Roles (320 threads, one CTA per SM, row tiles strided over the grid):
+// Roles (576 threads, one CTA per SM, row tiles strided over the grid):
 //   warp 0      TMA producer: x tile, W1 chunk and W2 chunk rings (128-byte swizzle)
 //   warp 1      TMEM owner (all 512 columns) and single-thread tcgen05.mma issuer
-//   warps 2-9   epilogue, two warps per TMEM lane quarter, each half of the columns
+//   warps 2-17  epilogue, four warps per TMEM lane quarter (a warp reaches only the lanes
+//               32 (warp % 4) .. + 31): 16 columns of every hidden chunk each, and one
+//               56-column piece of the output each (D = 224; for D = 112 the first two
+//               warps of each quarter). Four warps per scheduler hide the latency of the
+//               GELU chains; the per-row LayerNorm partial of each 112-column half of a
+//               D = 224 row is merged from its two pieces in shared memory, in the order
+//               the stand-alone GEMM's epilogue merges them.
 // TMEM: output accumulator at column 0 (D columns), fc1 chunk accumulators from ACC1_COL.
 #include "common.cuh"
 #include "internal.h"
@@ -33,8 +39,9 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int HC = 64;  // hidden chunk width
-constexpr int EPI_WARPS = 8;
+constexpr int EPI_WARPS = 16;
 constexpr int EPI_THREADS = EPI_WARPS * 32;
+constexpr int THREADS = 64 + EPI_THREADS;
 
 template <int D>
 struct MlpCfg {
@@ -56,17 +63,20 @@ struct MlpCfg {
   static constexpr int H_OFF = X_OFF + NX * X_BYTES;
   static constexpr int W1_OFF = H_OFF + NH * H_BYTES;
   static constexpr int W2_OFF = W1_OFF + S1 * W1_BYTES;
-  static constexpr int CONST_OFF = W2_OFF + S2 * W2_BYTES;   // colsum1, colconst1 [HID], b2 [D]
-  static constexpr int BAR_OFF = CONST_OFF + (2 * HID + D) * 4;
-  static constexpr int SMEM_BYTES = BAR_OFF + 512 + 1024;    // + alignment slack
+  static constexpr int CONST_OFF = W2_OFF + S2 * W2_BYTES;   // colsum1, colconst1 [HID]
+  static constexpr int BAR_OFF = CONST_OFF + 2 * HID * 4;
+  static constexpr int SMEM_BYTES = BAR_OFF + 512 + 2 * BM * 8 + 1024;  // + alignment slack
   static constexpr int ACC1_COL = D <= 128 ? 128 : 256;
   static constexpr int TMEM_COLS = 512;
-  static constexpr int HALF = D / 2;                         // output columns per thread
+  static constexpr int PIECES = D / 56;                      // 56-column output pieces per row
+  static constexpr int FIN_THREADS = PIECES * 4 * 32;        // threads that read the output
+  static constexpr int XCH_OFF = BAR_OFF + 512;              // float2 [2][128] partial exchange
   static_assert(D % 56 == 0 && D % 16 == 0, "D is a multiple of 112");
   static_assert(ACC1_COL >= D && ACC1_COL + NB * HC <= TMEM_COLS, "TMEM plan");
   static_assert(LAG < S2 && LAG < NB, "issue lag within the rings");
   static_assert(W2_BYTES % 1024 == 0 && X_BYTES % 1024 == 0, "operand alignment");
-  static_assert(NH * H_BYTES >= EPI_WARPS * 4096, "output staging aliases the hidden buffers");
+  static_assert(NH * H_BYTES >= EPI_WARPS * 2048, "output staging aliases the hidden buffers");
+  static_assert(PIECES == 2 || PIECES == 4, "output pieces");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
   static_assert(NC > LAG, "chunks");
 };
@@ -86,8 +96,31 @@ struct MlpParams {
   unsigned int* status;
 };
 
+// Output groups G0 .. G0 + NG - 1 (8 columns each) of a 56-column piece: accumulator + b2 +
+// residual (res[g], bf16), rounded; the packed result replaces res[g].
+template <int G0, int NG, int NR>
+__device__ __forceinline__ void out_groups(const uint32_t (&r)[NR], uint4 (&res)[7],
+                                           const float4* b4) {
+#pragma unroll
+  for (int gg = 0; gg < NG; ++gg) {
+    const int g = G0 + gg;
+    const uint4 rr = res[g];
+    const float4 q0 = __ldg(b4 + 2 * g), q1 = __ldg(b4 + 2 * g + 1);
+    float v[8];
+    v[0] = __uint_as_float(r[8 * gg + 0]) + q0.x + bf16_lo(rr.x);
+    v[1] = __uint_as_float(r[8 * gg + 1]) + q0.y + bf16_hi(rr.x);
+    v[2] = __uint_as_float(r[8 * gg + 2]) + q0.z + bf16_lo(rr.y);
+    v[3] = __uint_as_float(r[8 * gg + 3]) + q0.w + bf16_hi(rr.y);
+    v[4] = __uint_as_float(r[8 * gg + 4]) + q1.x + bf16_lo(rr.z);
+    v[5] = __uint_as_float(r[8 * gg + 5]) + q1.y + bf16_hi(rr.z);
+    v[6] = __uint_as_float(r[8 * gg + 6]) + q1.z + bf16_lo(rr.w);
+    v[7] = __uint_as_float(r[8 * gg + 7]) + q1.w + bf16_hi(rr.w);
+    res[g] = pack8(v);
+  }
+}
+
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(THREADS, 1)
     mlp_fused_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW1,
                      const __grid_constant__ CUtensorMap tmW2, const MlpParams p) {
   using C = MlpCfg<D>;
@@ -100,7 +133,6 @@ __global__ void __launch_bounds__(320, 1)
   uint8_t* sW2 = smem + C::W2_OFF;
   float* c_sum = reinterpret_cast<float*>(smem + C::CONST_OFF);
   float* c_const = c_sum + C::HID;
-  float* c_bias2 = c_const + C::HID;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint64_t* x_full = bars;                  // [NX]
   uint64_t* x_empty = x_full + C::NX;       // [NX]
@@ -143,7 +175,7 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&h_empty[i], 1);
     }
     mbar_init(a2_full, 1);
-    mbar_init(a2_empty, EPI_THREADS);
+    mbar_init(a2_empty, C::FIN_THREADS);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -159,7 +191,6 @@ __global__ void __launch_bounds__(320, 1)
     c_sum[i] = __ldg(p.colsum1 + i);
     c_const[i] = __ldg(p.colconst1 + i);
   }
-  for (int i = threadIdx.x; i < D; i += blockDim.x) c_bias2[i] = __ldg(p.bias2 + i);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -170,7 +201,7 @@ __global__ void __launch_bounds__(320, 1)
     if (lane == 0) {
       int xs = 0, s1 = 0, s2 = 0;
       uint32_t xph = 0, ph1 = 0, ph2 = 0;
-      long long nx = 0, n1 = 0, n2 = 0;  // loads issued per ring
+      uint32_t nx = 0, n1 = 0, n2 = 0;  // loads issued per ring
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         if (!mbar_wait(&x_empty[xs], xph ^ 1u, p.limit_ns, p.status, abort_flag)) {
@@ -221,11 +252,11 @@ __global__ void __launch_bounds__(320, 1)
       if (!ok) {
         *abort_flag = 1;
         // let copies already in flight land before the CTA's shared memory goes away
-        for (long long i = nx > C::NX ? nx - C::NX : 0; i < nx; ++i)
+        for (uint32_t i = nx > (uint32_t)C::NX ? nx - C::NX : 0; i < nx; ++i)
           mbar_wait(&x_full[i % C::NX], (uint32_t)((i / C::NX) & 1), p.limit_ns, p.status);
-        for (long long i = n1 > C::S1 ? n1 - C::S1 : 0; i < n1; ++i)
+        for (uint32_t i = n1 > (uint32_t)C::S1 ? n1 - C::S1 : 0; i < n1; ++i)
           mbar_wait(&w1_full[i % C::S1], (uint32_t)((i / C::S1) & 1), p.limit_ns, p.status);
-        for (long long i = n2 > C::S2 ? n2 - C::S2 : 0; i < n2; ++i)
+        for (uint32_t i = n2 > (uint32_t)C::S2 ? n2 - C::S2 : 0; i < n2; ++i)
           mbar_wait(&w2_full[i % C::S2], (uint32_t)((i / C::S2) & 1), p.limit_ns, p.status);
       }
     }
@@ -236,7 +267,7 @@ __global__ void __launch_bounds__(320, 1)
       constexpr uint32_t IDESC2 = idesc_bf16_f32(BM, D);
       int xs = 0, s1 = 0, s2 = 0;
       uint32_t xph = 0, ph1 = 0, ph2 = 0;
-      long long a1 = 0, hc = 0, t = 0;
+      uint32_t a1 = 0, hc = 0, t = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++t) {
         if (!mbar_wait(&x_full[xs], xph, p.limit_ns, p.status, abort_flag)) {
@@ -318,10 +349,11 @@ __global__ void __launch_bounds__(320, 1)
     // ------------------------------------------------------------ epilogue
     const int ew = warp - 2;
     const int quarter = warp & 3;  // TMEM lanes 32 quarter .. + 31
-    const int half = ew >> 2;      // which half of the columns
+    const int cg = ew >> 2;        // column group: 16 hidden columns / one 56-column piece
     const int rt = quarter * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    long long a1 = 0, hc = 0, t = 0;
+    float2* xch = reinterpret_cast<float2*>(smem + C::XCH_OFF);
+    uint32_t a1 = 0, hc = 0, t = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++t) {
       const long long m = (long long)tile * BM + rt;
@@ -338,22 +370,24 @@ __global__ void __launch_bounds__(320, 1)
           break;
         }
         tc_fence_after();
-        uint32_t r[32];
-        tmem_load<32>(tmem + lane_base + (uint32_t)(C::ACC1_COL + b * HC + half * 32), r);
+        uint32_t r[16];
+        tmem_load<16>(tmem + lane_base + (uint32_t)(C::ACC1_COL + b * HC + cg * 16), r);
         tc_fence_before();
         mbar_arrive(&a1_empty[b]);
         ++a1;
-        const float* cs = c_sum + j * HC + half * 32;
-        const float* cc = c_const + j * HC + half * 32;
-        uint4 pk[4];
+        const float4* cs4 = reinterpret_cast<const float4*>(c_sum + j * HC + cg * 16);
+        const float4* cc4 = reinterpret_cast<const float4*>(c_const + j * HC + cg * 16);
+        uint4 pk[2];
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
+        for (int g = 0; g < 2; ++g) {
+          const float4 s0 = cs4[2 * g], s1 = cs4[2 * g + 1];
+          const float4 k0 = cc4[2 * g], k1 = cc4[2 * g + 1];
+          const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+          const float kv[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
           float v[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int i = 8 * g + e;
-            v[e] = gelu_fast(fmaf(fa, __uint_as_float(r[i]), fmaf(fb, cs[i], cc[i])));
-          }
+          for (int e = 0; e < 8; ++e)
+            v[e] = gelu_fast(fmaf(fa, __uint_as_float(r[8 * g + e]), fmaf(fb, sv[e], kv[e])));
           pk[g] = pack8(v);
         }
         const int hb = (int)(hc % C::NH);
@@ -364,97 +398,119 @@ __global__ void __launch_bounds__(320, 1)
         }
         uint8_t* hrow = sH + hb * C::H_BYTES + rt * 128;
 #pragma unroll
-        for (int g = 0; g < 4; ++g)
-          *reinterpret_cast<uint4*>(hrow + (((half * 4 + g) ^ (rt & 7)) << 4)) = pk[g];
+        for (int g = 0; g < 2; ++g)
+          *reinterpret_cast<uint4*>(hrow + (((cg * 2 + g) ^ (rt & 7)) << 4)) = pk[g];
         fence_proxy_async_smem();
         mbar_arrive(&h_full[hb]);
         ++hc;
       }
-      // ---- output: + b2 + residual, bf16, LayerNorm partials, coalesced store
-      if (ok) {
-        constexpr int NV = C::HALF / 8;
-        uint4 res[NV];
-        const bf16* xrow = p.x + m * D + half * C::HALF;
+      // ---- output piece [56 cg, 56 cg + 56): + b2 + residual, bf16, LayerNorm partial,
+      //      coalesced store
+      const bool fin = cg < C::PIECES;
+      float st_mean = 0.f, st_m2 = 0.f;
+      if (fin && ok) {
+        const int c0 = cg * 56;
+        uint4 res[7];
+        const bf16* xrow = p.x + m * D + c0;
 #pragma unroll
-        for (int i = 0; i < NV; ++i)
+        for (int i = 0; i < 7; ++i)
           res[i] = row_ok ? __ldg(reinterpret_cast<const uint4*>(xrow) + i) : make_uint4(0u, 0u, 0u, 0u);
         if (!warp_wait(a2_full, (uint32_t)(t & 1), p.limit_ns, p.status, abort_flag)) ok = false;
         if (ok) {
           tc_fence_after();
-          uint8_t* stg = sH + (ew << 12);  // the hidden buffers are idle until the next tile
-          float st_mean = 0.f, st_m2 = 0.f;
+          const float4* b4 = reinterpret_cast<const float4*>(p.bias2 + c0);
+          // columns 0..31 then 32..55 of the piece (fewer live registers); the packed
+          // bf16 results replace the residual words in res[]
+          {
+            uint32_t r[32];
+            tmem_load<32>(tmem + lane_base + (uint32_t)c0, r);
+            out_groups<0, 4>(r, res, b4);
+          }
+          {
+            uint32_t r[24];
+            tc_ld_32x32b_x16(tmem + lane_base + (uint32_t)(c0 + 32),
+                             *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+            tc_ld_32x32b_x8(tmem + lane_base + (uint32_t)(c0 + 48),
+                            *reinterpret_cast<uint32_t(*)[8]>(&r[16]));
+            tc_wait_ld();
 #pragma unroll
-          for (int c = 0; c < C::HALF; c += 56) {
-            uint32_t r[56];
-            tmem_load<56>(tmem + lane_base + (uint32_t)(half * C::HALF + c), r);
-            if (c + 56 == C::HALF) {
-              tc_fence_before();
-              mbar_arrive(a2_empty);
-            }
-            float v[56];
+            for (int i = 0; i < 24; ++i) asm volatile("" : "+r"(r[i]));
+            tc_fence_before();
+            mbar_arrive(a2_empty);
+            out_groups<4, 3>(r, res, b4);
+          }
+          if (p.stats_out != nullptr) {
+            // statistics of the values as stored, in column order
+            float s = 0.f;
+#pragma unroll
+            for (int g = 0; g < 7; ++g)
+              s = (((((((s + bf16_lo(res[g].x)) + bf16_hi(res[g].x)) + bf16_lo(res[g].y)) +
+                      bf16_hi(res[g].y)) + bf16_lo(res[g].z)) + bf16_hi(res[g].z)) +
+                   bf16_lo(res[g].w)) + bf16_hi(res[g].w);
+            st_mean = s * (1.f / 56.f);
 #pragma unroll
             for (int g = 0; g < 7; ++g) {
-              const uint4 rr = res[c / 8 + g];
-              const float* bb = c_bias2 + half * C::HALF + c + 8 * g;
-              v[8 * g + 0] = __uint_as_float(r[8 * g + 0]) + bb[0] + bf16_lo(rr.x);
-              v[8 * g + 1] = __uint_as_float(r[8 * g + 1]) + bb[1] + bf16_hi(rr.x);
-              v[8 * g + 2] = __uint_as_float(r[8 * g + 2]) + bb[2] + bf16_lo(rr.y);
-              v[8 * g + 3] = __uint_as_float(r[8 * g + 3]) + bb[3] + bf16_hi(rr.y);
-              v[8 * g + 4] = __uint_as_float(r[8 * g + 4]) + bb[4] + bf16_lo(rr.z);
-              v[8 * g + 5] = __uint_as_float(r[8 * g + 5]) + bb[5] + bf16_hi(rr.z);
-              v[8 * g + 6] = __uint_as_float(r[8 * g + 6]) + bb[6] + bf16_lo(rr.w);
-              v[8 * g + 7] = __uint_as_float(r[8 * g + 7]) + bb[7] + bf16_hi(rr.w);
+              const uint32_t w4[4] = {res[g].x, res[g].y, res[g].z, res[g].w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float lo = bf16_lo(w4[e]) - st_mean, hi = bf16_hi(w4[e]) - st_mean;
+                st_m2 = fmaf(lo, lo, st_m2);
+                st_m2 = fmaf(hi, hi, st_m2);
+              }
             }
+          }
+          // staging (2 KB per warp, aliasing the idle hidden buffers): 16 rows at a time,
+          // then 8 lanes per row, 4 rows per store instruction
+          uint8_t* stg = sH + (ew << 11);
+          const unsigned long long my_dst =
+              reinterpret_cast<unsigned long long>(p.out + m * D + c0);
 #pragma unroll
-            for (int g = 0; g < 7; ++g) {
-              const uint4 pkv = pack8(&v[8 * g]);
-              *reinterpret_cast<uint4*>(stg + (lane << 7) + ((g ^ (lane & 7)) << 4)) = pkv;
-              v[8 * g + 0] = bf16_lo(pkv.x);
-              v[8 * g + 1] = bf16_hi(pkv.x);
-              v[8 * g + 2] = bf16_lo(pkv.y);
-              v[8 * g + 3] = bf16_hi(pkv.y);
-              v[8 * g + 4] = bf16_lo(pkv.z);
-              v[8 * g + 5] = bf16_hi(pkv.z);
-              v[8 * g + 6] = bf16_lo(pkv.w);
-              v[8 * g + 7] = bf16_hi(pkv.w);
-            }
-            if (p.stats_out != nullptr) {
-              float s = 0.f;
+          for (int hh = 0; hh < 2; ++hh) {
+            if ((lane >> 4) == hh) {
+              const int sr = lane & 15;
 #pragma unroll
-              for (int i = 0; i < 56; ++i) s += v[i];
-              const float cmean = s * (1.f / 56.f);
-              float cm2 = 0.f;
-#pragma unroll
-              for (int i = 0; i < 56; ++i) cm2 = fmaf(v[i] - cmean, v[i] - cmean, cm2);
-              const float na = (float)c, nb = 56.f, ntot = na + nb;
-              const float dlt = cmean - st_mean;
-              st_mean = fmaf(dlt, nb / ntot, st_mean);
-              st_m2 = st_m2 + cm2 + dlt * dlt * (na * nb / ntot);
+              for (int g = 0; g < 7; ++g)
+                *reinterpret_cast<uint4*>(stg + (sr << 7) + ((g ^ (sr & 7)) << 4)) = res[g];
             }
             __syncwarp();
-            // copy out: 8 lanes per row, 4 rows per instruction
-            const unsigned long long my_dst =
-                reinterpret_cast<unsigned long long>(p.out + m * D + half * C::HALF + c);
 #pragma unroll
-            for (int it = 0; it < 8; ++it) {
-              const int row = it * 4 + (lane >> 3), ch = lane & 7;
+            for (int it = 0; it < 4; ++it) {
+              const int sr = it * 4 + (lane >> 3), ch = lane & 7;
+              const int row = hh * 16 + sr;
               const unsigned long long dst = __shfl_sync(0xffffffffu, my_dst, row);
               const int wr = __shfl_sync(0xffffffffu, row_ok ? 1 : 0, row);
               if (wr && ch < 7) {
                 const uint4 val =
-                    *reinterpret_cast<const uint4*>(stg + (row << 7) + ((ch ^ (row & 7)) << 4));
+                    *reinterpret_cast<const uint4*>(stg + (sr << 7) + ((ch ^ (sr & 7)) << 4));
                 *reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(dst) + ch * 8) = val;
               }
             }
             __syncwarp();
           }
-          if (p.stats_out != nullptr && row_ok)
-            p.stats_out[m * 2 + half] = make_float2(st_mean, st_m2);
+          // LayerNorm partial per 112-column half: D = 112 pieces are halves already; for
+          // D = 224 the odd piece hands its (mean, M2) to the even one
+          if (p.stats_out != nullptr && C::PIECES == 4 && (cg & 1)) xch[(cg >> 1) * BM + rt] =
+              make_float2(st_mean, st_m2);
+        }
+      }
+      if (C::PIECES == 4) named_bar_sync(2, EPI_THREADS);
+      if (fin && ok && p.stats_out != nullptr && row_ok) {
+        if (C::PIECES == 2) {
+          p.stats_out[m * 2 + cg] = make_float2(st_mean, st_m2);
+        } else if ((cg & 1) == 0) {
+          // Chan et al. merge of the second 56 columns into the first, as the GEMM's
+          // epilogue merges its consecutive chunks
+          const float2 o = xch[(cg >> 1) * BM + rt];
+          const float na = 56.f, nb = 56.f, ntot = na + nb;
+          const float dlt = o.x - st_mean;
+          const float mean = fmaf(dlt, nb / ntot, st_mean);
+          const float m2 = st_m2 + o.y + dlt * dlt * (na * nb / ntot);
+          p.stats_out[m * 2 + (cg >> 1)] = make_float2(mean, m2);
         }
       }
       // every epilogue warp is done with the staging area (it aliases the hidden buffers)
-      // before any warp writes the next tile's hidden chunk; taken on every path, so the
-      // warps stay matched even after a timeout
+      // and the exchange slots before any warp writes the next tile's hidden chunk; taken
+      // on every path, so the warps stay matched even after a timeout
       named_bar_sync(1, EPI_THREADS);
     }
   }
@@ -517,7 +573,7 @@ hiera_status run_mlp(const MlpArgs& a, cudaStream_t stream) {
   int grid = g_num_sms();
   if (grid > tiles) grid = tiles;
   profile_mark(K_MLP_FUSED, stream);
-  kern<<<grid, 320, C::SMEM_BYTES, stream>>>(tmX, tmW1, tmW2, p);
+  kern<<<grid, THREADS, C::SMEM_BYTES, stream>>>(tmX, tmW1, tmW2, p);
   return cudaGetLastError() == cudaSuccess ? HIERA_OK : HIERA_ERR_CUDA;
 }
 
