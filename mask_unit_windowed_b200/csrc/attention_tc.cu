@@ -117,27 +117,32 @@ __global__ void __launch_bounds__(320, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      mbar_arrive_expect_tx(q_full, 2 * Q_BYTES);
-      tma_load_3d(smem + OFF_Q, &tmQ, q_full, 0, q0, unit);
-      tma_load_3d(smem + OFF_Q + Q_BYTES, &tmQ, q_full, 0, q0 + QT, unit);
-      long long issued = 0;
-      bool ok = true;
-      for (int j = 0; j < n_tiles; ++j) {
-        const int s = j % KV_STAGES;
-        if (!mbar_wait(&kv_empty[s], (uint32_t)(((j / KV_STAGES) & 1) ^ 1), p.limit_ns, p.status,
-                       abort_flag)) {
-          *abort_flag = 1;
-          ok = false;
-          break;
-        }
-        uint8_t* st = smem + OFF_KV + s * KV_BYTES;
-        mbar_arrive_expect_tx(&kv_full[s], KV_BYTES);
-        tma_load_3d(st, &tmK, &kv_full[s], 0, j * KT, unit);
-        tma_load_3d(st + K_BYTES, &tmV, &kv_full[s], j * KT, 0, unit);
-        tma_load_3d(st + K_BYTES + 64 * 128, &tmV, &kv_full[s], j * KT + 64, 0, unit);
-        ++issued;
+    // One thread's TMA loads complete one after another, so the boxes are issued by lanes
+    // rotating over 8; every lane walks the same sequence and waits on the same barriers.
+    if (lane == 0) mbar_arrive_expect_tx(q_full, 2 * Q_BYTES);
+    __syncwarp();
+    if (lane == 0) tma_load_3d(smem + OFF_Q, &tmQ, q_full, 0, q0, unit);
+    if (lane == 1) tma_load_3d(smem + OFF_Q + Q_BYTES, &tmQ, q_full, 0, q0 + QT, unit);
+    long long issued = 0;
+    bool ok = true;
+    int rr = 2;
+    for (int j = 0; j < n_tiles; ++j) {
+      const int s = j % KV_STAGES;
+      if (!warp_wait(&kv_empty[s], (uint32_t)(((j / KV_STAGES) & 1) ^ 1), p, abort_flag)) {
+        ok = false;
+        break;
       }
+      uint8_t* st = smem + OFF_KV + s * KV_BYTES;
+      if (lane == 0) mbar_arrive_expect_tx(&kv_full[s], KV_BYTES);
+      __syncwarp();
+      if (lane == rr) tma_load_3d(st, &tmK, &kv_full[s], 0, j * KT, unit);
+      if (lane == ((rr + 1) & 7)) tma_load_3d(st + K_BYTES, &tmV, &kv_full[s], j * KT, 0, unit);
+      if (lane == ((rr + 2) & 7))
+        tma_load_3d(st + K_BYTES + 64 * 128, &tmV, &kv_full[s], j * KT + 64, 0, unit);
+      rr = (rr + 3) & 7;
+      ++issued;
+    }
+    if (lane == 0) {
       mbar_wait(q_full, 0, p.limit_ns, p.status);
       if (!ok) {
         for (long long i = issued > KV_STAGES ? issued - KV_STAGES : 0; i < issued; ++i)
@@ -150,6 +155,7 @@ __global__ void __launch_bounds__(320, 1)
     if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, KT);
       constexpr uint32_t IDESC_O = idesc_bf16_f32(128, 64);
+      const uint64_t desc0 = smem_desc_sw128(smem_u32(smem));
       bool ok = mbar_wait(q_full, 0, p.limit_ns, p.status, abort_flag);
       tc_fence_after();
       for (int j = 0; ok && j <= n_tiles; ++j) {
@@ -160,7 +166,7 @@ __global__ void __launch_bounds__(320, 1)
             ok = false;
             break;
           }
-          const uint64_t kdesc = smem_desc_sw128(smem_u32(smem + OFF_KV + s * KV_BYTES));
+          const uint64_t kdesc = desc_advance(desc0, (uint32_t)(OFF_KV + s * KV_BYTES));
           for (int t = 0; t < 2 && ok; ++t) {
             // the softmax of tile t has read S_t(j-1) out of TMEM
             if (j >= 1 && !mbar_wait(&s_free[t], (uint32_t)((j - 1) & 1), p.limit_ns, p.status,
@@ -169,32 +175,36 @@ __global__ void __launch_bounds__(320, 1)
               break;
             }
             tc_fence_after();
-            const uint64_t qdesc = smem_desc_sw128(smem_u32(smem + OFF_Q + t * Q_BYTES));
+            const uint64_t qdesc = desc_advance(desc0, (uint32_t)(OFF_Q + t * Q_BYTES));
+            tc_mma_bf16_k<false>(tmem + (uint32_t)(t * KT), qdesc, kdesc, IDESC_S);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              tc_mma_bf16(tmem + (uint32_t)(t * KT), qdesc + (uint64_t)(2 * kk),
-                          kdesc + (uint64_t)(2 * kk), IDESC_S, kk > 0 ? 1u : 0u);
+            for (int kk = 1; kk < 4; ++kk)
+              tc_mma_bf16_k<true>(tmem + (uint32_t)(t * KT), desc_advance(qdesc, 32u * kk),
+                                  desc_advance(kdesc, 32u * kk), IDESC_S);
             tc_commit(&s_full[t]);
           }
           if (!ok) break;
         }
         if (j >= 1) {
           const int jj = j - 1, s2 = jj % KV_STAGES;
-          const uint32_t vbase = smem_u32(smem + OFF_KV + s2 * KV_BYTES + K_BYTES);
+          const uint64_t vdesc = desc_advance(desc0, (uint32_t)(OFF_KV + s2 * KV_BYTES + K_BYTES));
           for (int t = 0; t < 2 && ok; ++t) {
             if (!mbar_wait(&p_full[t], (uint32_t)(jj & 1), p.limit_ns, p.status, abort_flag)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            const uint32_t pbase = smem_u32(smem + OFF_P + t * P_BYTES);
+            const uint64_t pdesc = desc_advance(desc0, (uint32_t)(OFF_P + t * P_BYTES));
+            const uint32_t od = tmem + O_COL + (uint32_t)(t * 64);
+            if (jj == 0)
+              tc_mma_bf16_k<false>(od, pdesc, vdesc, IDESC_O);
+            else
+              tc_mma_bf16_k<true>(od, pdesc, vdesc, IDESC_O);
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const int blk = kk >> 2, k4 = kk & 3;
-              const uint64_t pd = smem_desc_sw128(pbase + blk * (QT * 128)) + (uint64_t)(2 * k4);
-              const uint64_t vd = smem_desc_sw128(vbase + blk * (64 * 128)) + (uint64_t)(2 * k4);
-              tc_mma_bf16(tmem + O_COL + (uint32_t)(t * 64), pd, vd, IDESC_O,
-                          (jj > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 1; kk < 8; ++kk) {
+              const uint32_t blk = kk >> 2, k4 = kk & 3;
+              tc_mma_bf16_k<true>(od, desc_advance(pdesc, blk * (QT * 128) + 32u * k4),
+                                  desc_advance(vdesc, blk * (64 * 128) + 32u * k4), IDESC_O);
             }
             tc_commit(&o_done[t]);
             tc_commit(&p_free[t]);

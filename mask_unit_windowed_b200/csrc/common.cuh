@@ -261,6 +261,32 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
   return d;
 }
 
+// A descriptor with its start address advanced by `bytes` (a multiple of 16, staying inside
+// shared memory, so the 14-bit address field cannot carry into the next field): only the
+// low word changes, one 32-bit add instead of rebuilding the descriptor.
+__device__ __forceinline__ uint64_t desc_advance(uint64_t desc, uint32_t bytes) {
+  return desc + (uint64_t)(bytes >> 4);
+}
+
+// tcgen05.mma with the accumulate flag fixed at compile time (no predicate computation).
+template <bool ACC>
+__device__ __forceinline__ void tc_mma_bf16_k(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                              uint32_t idesc) {
+  if constexpr (ACC) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.eq.u32 p, 1, 1;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.eq.u32 p, 1, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc)
+        : "memory");
+  }
+}
+
 // Instruction descriptor for kind::f16 with bf16 A/B, fp32 accumulator, both operands
 // K-major: D format bits 4-5 = 1 (f32), A format bits 7-9 = 1 (bf16), B format bits
 // 10-12 = 1 (bf16), N >> 3 in bits 17-22, M >> 4 in bits 24-28.
@@ -346,11 +372,8 @@ __device__ __forceinline__ uint4 pack8(const float* v) {
 // LayerNorm of a row of K values from P partial (mean, M2) pairs over K / P values each
 // (Chan et al. merge with equal counts): LN(x) W^T + b = fa (x W'^T) + fb s + c with
 // fa = rstd, fb = -mean rstd (s, c the packed column constants of the folded weight).
-__device__ __forceinline__ void ln_fold_coeffs(const float2* __restrict__ sp, int P, int K,
-                                               float eps, float& fa, float& fb) {
-  float2 part[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) part[j] = j < P ? __ldg(sp + j) : make_float2(0.f, 0.f);
+__device__ __forceinline__ void ln_merge_parts(const float2 (&part)[8], int P, int K, float eps,
+                                               float& fa, float& fb) {
   float mean = 0.f;
 #pragma unroll
   for (int j = 0; j < 8; ++j) mean += part[j].x;
@@ -367,6 +390,14 @@ __device__ __forceinline__ void ln_fold_coeffs(const float2* __restrict__ sp, in
   m2 = fmaf((float)(K / P), dev2, m2);
   fa = rsqrtf(m2 / (float)K + eps);
   fb = -mean * fa;
+}
+
+__device__ __forceinline__ void ln_fold_coeffs(const float2* __restrict__ sp, int P, int K,
+                                               float eps, float& fa, float& fb) {
+  float2 part[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) part[j] = j < P ? __ldg(sp + j) : make_float2(0.f, 0.f);
+  ln_merge_parts(part, P, K, eps, fa, fb);
 }
 
 // ------------------------------------------------------------------ Unroll map

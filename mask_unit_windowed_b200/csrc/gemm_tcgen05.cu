@@ -139,21 +139,25 @@ __global__ void __launch_bounds__(320, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      int s = 0;
-      uint32_t ph = 0;
-      long long issued = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int mt = tile / n_tiles, nt = tile - (tile / n_tiles) * n_tiles;
-        for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(&empty[s], ph ^ 1u, p.limit_ns, p.status, abort_flag)) {
-            *abort_flag = 1;
-            ok = false;
-            break;
-          }
-          uint8_t* sa = smem + s * C::STAGE_BYTES;
-          mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
+    // One thread's TMA loads complete one after another, so the loads of consecutive
+    // stages are issued by different lanes (A and B of a stage by two lanes, rotating over
+    // 8 lanes); every lane walks the same stage sequence and waits on the same barriers.
+    int s = 0;
+    uint32_t ph = 0;
+    long long issued = 0;
+    bool ok = true;
+    int rr = 0;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      const int mt = tile / n_tiles, nt = tile - (tile / n_tiles) * n_tiles;
+      for (int kb = 0; kb < kblocks; ++kb) {
+        if (!warp_wait(&empty[s], ph ^ 1u, p.limit_ns, p.status, abort_flag)) {
+          ok = false;
+          break;
+        }
+        uint8_t* sa = smem + s * C::STAGE_BYTES;
+        if (lane == 0) mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
+        __syncwarp();
+        if (lane == rr) {
           if (POOLED) {
             const int per = p.tokens >> 2;
             if (per >= 32) {
@@ -168,24 +172,26 @@ __global__ void __launch_bounds__(320, 1)
           } else {
             tma_load_2d(sa, &tmA, &full[s], kb * BK, mt * BM);
           }
-          tma_load_2d(sa + C::A_BYTES, &tmB, &full[s], kb * BK, nt * BN);
-          ++issued;
-          if (++s == STAGES) {
-            s = 0;
-            ph ^= 1u;
-          }
+        }
+        if (lane == rr + 1) tma_load_2d(sa + C::A_BYTES, &tmB, &full[s], kb * BK, nt * BN);
+        rr = (rr + 2) & 7;
+        ++issued;
+        if (++s == STAGES) {
+          s = 0;
+          ph ^= 1u;
         }
       }
-      if (!ok) {
-        // let copies already in flight land before the CTA's shared memory goes away
-        for (long long i = issued > STAGES ? issued - STAGES : 0; i < issued; ++i)
-          mbar_wait(&full[i % STAGES], (uint32_t)((i / STAGES) & 1), p.limit_ns, p.status);
-      }
+    }
+    if (!ok && lane == 0) {
+      // let copies already in flight land before the CTA's shared memory goes away
+      for (long long i = issued > STAGES ? issued - STAGES : 0; i < issued; ++i)
+        mbar_wait(&full[i % STAGES], (uint32_t)((i / STAGES) & 1), p.limit_ns, p.status);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
+      const uint64_t desc0 = smem_desc_sw128(smem_u32(smem));  // stage 0, A tile
       int s = 0, acc = 0;
       uint32_t ph = 0, aph = 0;
       bool ok = true;
@@ -203,15 +209,17 @@ __global__ void __launch_bounds__(320, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
-          const uint64_t adesc = smem_desc_sw128(sa);
-          const uint64_t bdesc = smem_desc_sw128(sa + C::A_BYTES);
+          const uint64_t adesc = desc_advance(desc0, (uint32_t)(s * C::STAGE_BYTES));
+          const uint64_t bdesc = desc_advance(adesc, (uint32_t)C::A_BYTES);
+          if (kb == 0)
+            tc_mma_bf16_k<false>(d, adesc, bdesc, IDESC);
+          else
+            tc_mma_bf16_k<true>(d, adesc, bdesc, IDESC);
 #pragma unroll
-          for (int j = 0; j < BK / 16; ++j) {
+          for (int j = 1; j < BK / 16; ++j)
             if (kb * BK + j * 16 < p.K)
-              tc_mma_bf16(d, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(2 * j), IDESC,
-                          (kb | j) != 0 ? 1u : 0u);
-          }
+              tc_mma_bf16_k<true>(d, desc_advance(adesc, 32u * j), desc_advance(bdesc, 32u * j),
+                                  IDESC);
           tc_commit(&empty[s]);
           if (++s == STAGES) {
             s = 0;
@@ -236,14 +244,50 @@ __global__ void __launch_bounds__(320, 1)
     const int quarter = warp & 3;          // TMEM lanes 32*quarter .. +31
     const int c_begin = (ew >> 2) * HALF;  // this warp's half of the tile's columns
     const int rt = quarter * 32 + lane;    // tile row == TMEM lane
-    const int etid = ew * 32 + lane;
     int acc = 0;
     uint32_t aph = 0;
+    // global row of this thread's TMEM lane in a tile (pooled tiles interleave 4 rows per
+    // pooled token)
+    auto row_of = [&](int tile) -> long long {
+      const int mt = tile / n_tiles;
+      if (POOLED) {
+        const int per = p.tokens >> 2;
+        const int pm = mt * 32 + (rt >> 2);
+        const int bb = pm / per, npp = pm - (pm / per) * per;
+        return (long long)bb * p.tokens + (rt & 3) * per + npp;
+      }
+      return (long long)mt * BM + rt;
+    };
+    // the LayerNorm partials of the next tile's row are loaded while this tile is processed
+    float2 part[8];
+    auto load_parts = [&](int tile) {
+      const long long mm = row_of(tile);
+      const int P = p.stats_parts;
+      const float2* sp = p.stats_in + (mm < p.M ? mm : 0) * P;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) part[j] = j < P ? __ldg(sp + j) : make_float2(0.f, 0.f);
+    };
+    // this thread's share of a tile's column constants (BN <= 256 columns, one per thread),
+    // also loaded one tile ahead and staged in shared memory at the tile's start
+    const int etid = ew * 32 + lane;
+    float nsum = 0.f, nconst = 0.f;
+    auto load_consts = [&](int tile) {
+      const int c = (tile - (tile / n_tiles) * n_tiles) * BN + etid;
+      if (etid < BN) {
+        nsum = FOLD ? __ldg(p.colsum + c) : 0.f;
+        nconst = p.colconst != nullptr ? __ldg(p.colconst + c)
+                 : (p.bias16 != nullptr ? __bfloat162float(p.bias16[c]) : 0.f);
+      }
+    };
+    if ((int)blockIdx.x < num_tiles) {
+      if (FOLD) load_parts(blockIdx.x);
+      load_consts(blockIdx.x);
+    }
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       const int mt = tile / n_tiles, nt = tile - (tile / n_tiles) * n_tiles;
       const int n0 = nt * BN;
       // row bookkeeping
-      long long m;
+      const long long m = row_of(tile);
       int b = 0, tok = 0, np = 0;
       if (POOLED) {
         const int per = p.tokens >> 2;
@@ -251,13 +295,9 @@ __global__ void __launch_bounds__(320, 1)
         b = pm / per;
         np = pm - b * per;
         tok = (rt & 3) * per + np;
-        m = (long long)b * p.tokens + tok;
-      } else {
-        m = (long long)mt * BM + rt;
-        if (EPI == EPI_QKV) {
-          b = (int)(m / p.tokens);
-          tok = (int)(m - (long long)b * p.tokens);
-        }
+      } else if (EPI == EPI_QKV) {
+        b = (int)(m / p.tokens);
+        tok = (int)(m - (long long)b * p.tokens);
       }
       const bool row_ok = m < p.M;
       // residual of this row / half, in flight while the mainloop runs
@@ -274,15 +314,18 @@ __global__ void __launch_bounds__(320, 1)
       }
       // LayerNorm statistics of this row, merged from the producer's partials
       float fa = 1.f, fb = 0.f;  // v = fa * acc + fb * colsum + colconst
-      if (FOLD && row_ok) ln_fold_coeffs(p.stats_in + m * p.stats_parts, p.stats_parts, p.K, p.ln_eps, fa, fb);
-      // per-column constants of this tile into shared memory
+      if (FOLD && row_ok) ln_merge_parts(part, p.stats_parts, p.K, p.ln_eps, fa, fb);
+      // per-column constants of this tile into shared memory (loaded a tile ahead)
       named_bar_sync(1, EPI_THREADS);  // every epilogue thread is done with the last tile's
-      for (int i = etid; i < BN; i += EPI_THREADS) {
-        col_sum[i] = FOLD ? __ldg(p.colsum + n0 + i) : 0.f;
-        col_const[i] = p.colconst != nullptr ? __ldg(p.colconst + n0 + i)
-                       : (p.bias16 != nullptr ? __bfloat162float(p.bias16[n0 + i]) : 0.f);
+      if (etid < BN) {
+        col_sum[etid] = nsum;
+        col_const[etid] = nconst;
       }
       named_bar_sync(1, EPI_THREADS);
+      if (tile + (int)gridDim.x < num_tiles) {
+        if (FOLD) load_parts(tile + gridDim.x);
+        load_consts(tile + gridDim.x);
+      }
       if (!warp_wait(&acc_full[acc], aph, p.limit_ns, p.status, abort_flag)) break;
       tc_fence_after();
       const uint32_t tbase = tmem + (uint32_t)(acc * C::ACC_STRIDE) +

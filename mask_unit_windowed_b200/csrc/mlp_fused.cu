@@ -11,19 +11,22 @@
 //                 written to a shared-memory chunk buffer in the tensor-core operand layout
 //   fc2 chunk j   hidden chunk (128 x 64) x W2 columns [64 j, 64 j + 64)
 //                 -> the D-column fp32 output accumulator in TMEM, accumulated over j
-// fc2 of chunk j is issued after fc1 of chunk j + LAG, so the tensor pipe computes the next
-// fc1 chunks while the epilogue warps turn chunk j into bf16. After the last chunk the
-// epilogue adds b2 and the residual, rounds to bf16, stores the tile and emits the
-// LayerNorm partials (mean, M2 per row half) of what it stored for the next block's norm1.
+// fc1 runs up to NB chunks ahead of the epilogue, so the tensor pipe computes the next fc1
+// chunks while the epilogue warps turn chunk j into bf16; the producer loads the W2 chunk
+// LAG chunks behind the W1 chunk, in the order the two issuers consume them. After the
+// last chunk the epilogue adds b2 and the residual, rounds to bf16, stores the tile and
+// emits the LayerNorm partials (mean, M2 per row half) of what it stored for the next
+// block's norm1.
 //
 // The order of the tensor-core K steps for every output element is the same as in the
 // stand-alone fc1 (K = D in steps of 16) and fc2 (K = 4 D in steps of 16) GEMMs, and the
 // fold / GELU / rounding code is shared, so the result is the same as the unfused pair's.
 //
-// Roles (576 threads, one CTA per SM, row tiles strided over the grid):
+// Roles (608 threads, one CTA per SM, row tiles strided over the grid):
 //   warp 0      TMA producer: x tile, W1 chunk and W2 chunk rings (128-byte swizzle)
-//   warp 1      TMEM owner (all 512 columns) and single-thread tcgen05.mma issuer
-//   warps 2-17  epilogue, four warps per TMEM lane quarter (a warp reaches only the lanes
+//   warp 1      TMEM owner (all 512 columns), fc1 tcgen05.mma issuer (one thread)
+//   warp 2      fc2 tcgen05.mma issuer (one thread)
+//   warps 3-18  epilogue, four warps per TMEM lane quarter (a warp reaches only the lanes
 //               32 (warp % 4) .. + 31): 16 columns of every hidden chunk each, and one
 //               56-column piece of the output each (D = 224; for D = 112 the first two
 //               warps of each quarter). Four warps per scheduler hide the latency of the
@@ -41,7 +44,7 @@ constexpr int BM = 128;
 constexpr int HC = 64;  // hidden chunk width
 constexpr int EPI_WARPS = 16;
 constexpr int EPI_THREADS = EPI_WARPS * 32;
-constexpr int THREADS = 64 + EPI_THREADS;
+constexpr int THREADS = 96 + EPI_THREADS;
 
 template <int D>
 struct MlpCfg {
@@ -54,7 +57,7 @@ struct MlpCfg {
   static constexpr int NH = 2;                  // hidden chunk buffers in shared memory
   static constexpr int S1 = D <= 128 ? 4 : 2;   // W1 chunk ring
   static constexpr int S2 = D <= 128 ? 4 : 2;   // W2 chunk ring
-  static constexpr int LAG = D <= 128 ? 2 : 1;  // fc2(j) is issued after fc1(j + LAG)
+  static constexpr int LAG = D <= 128 ? 2 : 1;  // W2 chunk j is loaded after W1 chunk j + LAG
   static constexpr int X_BYTES = KB1 * BM * 128;
   static constexpr int H_BYTES = BM * 128;
   static constexpr int W1_BYTES = KB1 * HC * 128;
@@ -147,7 +150,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* a2_full = h_empty + C::NH;
   uint64_t* a2_empty = a2_full + 1;
   uint64_t* drain = a2_empty + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* drain2 = drain + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain2 + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -177,6 +181,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(a2_full, 1);
     mbar_init(a2_empty, C::FIN_THREADS);
     mbar_init(drain, 1);
+    mbar_init(drain2, 1);
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmX);
@@ -198,156 +203,181 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      int xs = 0, s1 = 0, s2 = 0;
-      uint32_t xph = 0, ph1 = 0, ph2 = 0;
-      uint32_t nx = 0, n1 = 0, n2 = 0;  // loads issued per ring
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        if (!mbar_wait(&x_empty[xs], xph ^ 1u, p.limit_ns, p.status, abort_flag)) {
-          ok = false;
-          break;
-        }
-        mbar_arrive_expect_tx(&x_full[xs], C::X_BYTES);
+    // One thread's TMA loads complete one after another, so the boxes are issued by lanes
+    // rotating over 8; every lane walks the same sequence and waits on the same barriers.
+    int xs = 0, s1 = 0, s2 = 0, rr = 0;
+    uint32_t xph = 0, ph1 = 0, ph2 = 0;
+    uint32_t nx = 0, n1 = 0, n2 = 0;  // loads issued per ring
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      if (!warp_wait(&x_empty[xs], xph ^ 1u, p.limit_ns, p.status, abort_flag)) {
+        ok = false;
+        break;
+      }
+      if (lane == 0) mbar_arrive_expect_tx(&x_full[xs], C::X_BYTES);
+      __syncwarp();
 #pragma unroll
-        for (int kb = 0; kb < C::KB1; ++kb)
+      for (int kb = 0; kb < C::KB1; ++kb)
+        if (lane == ((rr + kb) & 7))
           tma_load_2d(sX + xs * C::X_BYTES + kb * BM * 128, &tmX, &x_full[xs], kb * 64, tile * BM);
-        ++nx;
-        if (++xs == C::NX) {
-          xs = 0;
-          xph ^= 1u;
-        }
-        for (int j = 0; j < C::NC + C::LAG && ok; ++j) {
-          if (j < C::NC) {
-            if (!mbar_wait(&w1_empty[s1], ph1 ^ 1u, p.limit_ns, p.status, abort_flag)) {
-              ok = false;
-              break;
-            }
-            mbar_arrive_expect_tx(&w1_full[s1], C::W1_BYTES);
+      rr = (rr + C::KB1) & 7;
+      ++nx;
+      if (++xs == C::NX) {
+        xs = 0;
+        xph ^= 1u;
+      }
+      for (int j = 0; j < C::NC + C::LAG && ok; ++j) {
+        if (j < C::NC) {
+          if (!warp_wait(&w1_empty[s1], ph1 ^ 1u, p.limit_ns, p.status, abort_flag)) {
+            ok = false;
+            break;
+          }
+          if (lane == 0) mbar_arrive_expect_tx(&w1_full[s1], C::W1_BYTES);
+          __syncwarp();
 #pragma unroll
-            for (int kb = 0; kb < C::KB1; ++kb)
+          for (int kb = 0; kb < C::KB1; ++kb)
+            if (lane == ((rr + kb) & 7))
               tma_load_2d(sW1 + s1 * C::W1_BYTES + kb * HC * 128, &tmW1, &w1_full[s1], kb * 64,
                           j * HC);
-            ++n1;
-            if (++s1 == C::S1) {
-              s1 = 0;
-              ph1 ^= 1u;
-            }
+          rr = (rr + C::KB1) & 7;
+          ++n1;
+          if (++s1 == C::S1) {
+            s1 = 0;
+            ph1 ^= 1u;
           }
-          if (j >= C::LAG) {
-            if (!mbar_wait(&w2_empty[s2], ph2 ^ 1u, p.limit_ns, p.status, abort_flag)) {
-              ok = false;
-              break;
-            }
-            mbar_arrive_expect_tx(&w2_full[s2], C::W2_BYTES);
+        }
+        if (j >= C::LAG) {
+          if (!warp_wait(&w2_empty[s2], ph2 ^ 1u, p.limit_ns, p.status, abort_flag)) {
+            ok = false;
+            break;
+          }
+          if (lane == 0) mbar_arrive_expect_tx(&w2_full[s2], C::W2_BYTES);
+          __syncwarp();
+          if (lane == rr)
             tma_load_2d(sW2 + s2 * C::W2_BYTES, &tmW2, &w2_full[s2], (j - C::LAG) * HC, 0);
-            ++n2;
-            if (++s2 == C::S2) {
-              s2 = 0;
-              ph2 ^= 1u;
-            }
+          rr = (rr + 1) & 7;
+          ++n2;
+          if (++s2 == C::S2) {
+            s2 = 0;
+            ph2 ^= 1u;
           }
         }
       }
-      if (!ok) {
-        *abort_flag = 1;
-        // let copies already in flight land before the CTA's shared memory goes away
-        for (uint32_t i = nx > (uint32_t)C::NX ? nx - C::NX : 0; i < nx; ++i)
-          mbar_wait(&x_full[i % C::NX], (uint32_t)((i / C::NX) & 1), p.limit_ns, p.status);
-        for (uint32_t i = n1 > (uint32_t)C::S1 ? n1 - C::S1 : 0; i < n1; ++i)
-          mbar_wait(&w1_full[i % C::S1], (uint32_t)((i / C::S1) & 1), p.limit_ns, p.status);
-        for (uint32_t i = n2 > (uint32_t)C::S2 ? n2 - C::S2 : 0; i < n2; ++i)
-          mbar_wait(&w2_full[i % C::S2], (uint32_t)((i / C::S2) & 1), p.limit_ns, p.status);
-      }
+    }
+    if (!ok && lane == 0) {
+      *abort_flag = 1;
+      // let copies already in flight land before the CTA's shared memory goes away
+      for (uint32_t i = nx > (uint32_t)C::NX ? nx - C::NX : 0; i < nx; ++i)
+        mbar_wait(&x_full[i % C::NX], (uint32_t)((i / C::NX) & 1), p.limit_ns, p.status);
+      for (uint32_t i = n1 > (uint32_t)C::S1 ? n1 - C::S1 : 0; i < n1; ++i)
+        mbar_wait(&w1_full[i % C::S1], (uint32_t)((i / C::S1) & 1), p.limit_ns, p.status);
+      for (uint32_t i = n2 > (uint32_t)C::S2 ? n2 - C::S2 : 0; i < n2; ++i)
+        mbar_wait(&w2_full[i % C::S2], (uint32_t)((i / C::S2) & 1), p.limit_ns, p.status);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ fc1 issuer
+    // Two issuing threads: the issue cost of tcgen05.mma / commit / barrier waits is paid
+    // by one thread each for fc1 and fc2. Their MMAs touch disjoint TMEM columns and
+    // shared memory, so they need no ordering between them; each commits its own.
     if (lane == 0) {
       constexpr uint32_t IDESC1 = idesc_bf16_f32(BM, HC);
-      constexpr uint32_t IDESC2 = idesc_bf16_f32(BM, D);
-      int xs = 0, s1 = 0, s2 = 0;
-      uint32_t xph = 0, ph1 = 0, ph2 = 0;
-      uint32_t a1 = 0, hc = 0, t = 0;
+      const uint64_t xdesc0 = smem_desc_sw128(smem_u32(sX));
+      const uint64_t w1desc0 = smem_desc_sw128(smem_u32(sW1));
+      int xs = 0, s1 = 0;
+      uint32_t xph = 0, ph1 = 0, a1 = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++t) {
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         if (!mbar_wait(&x_full[xs], xph, p.limit_ns, p.status, abort_flag)) {
           ok = false;
           break;
         }
-        const uint32_t xa = smem_u32(sX + xs * C::X_BYTES);
-        for (int j = 0; j < C::NC + C::LAG && ok; ++j) {
-          if (j < C::NC) {
-            const int b = (int)(a1 % C::NB);
-            const uint32_t bph = (uint32_t)((a1 / C::NB) & 1);
-            if (!mbar_wait(&a1_empty[b], bph ^ 1u, p.limit_ns, p.status, abort_flag) ||
-                !mbar_wait(&w1_full[s1], ph1, p.limit_ns, p.status, abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t wa = smem_u32(sW1 + s1 * C::W1_BYTES);
-            const uint32_t d1 = tmem + (uint32_t)(C::ACC1_COL + b * HC);
-#pragma unroll
-            for (int ks = 0; ks < C::K1_STEPS; ++ks) {
-              const int kb = ks >> 2, kk = ks & 3;
-              tc_mma_bf16(d1, smem_desc_sw128(xa + kb * BM * 128) + (uint64_t)(2 * kk),
-                          smem_desc_sw128(wa + kb * HC * 128) + (uint64_t)(2 * kk), IDESC1,
-                          ks != 0 ? 1u : 0u);
-            }
-            tc_commit(&w1_empty[s1]);
-            tc_commit(&a1_full[b]);
-            ++a1;
-            if (++s1 == C::S1) {
-              s1 = 0;
-              ph1 ^= 1u;
-            }
-            if (j == C::NC - 1) {
-              tc_commit(&x_empty[xs]);
-              if (++xs == C::NX) {
-                xs = 0;
-                xph ^= 1u;
-              }
-            }
+        const uint64_t xdesc = desc_advance(xdesc0, (uint32_t)(xs * C::X_BYTES));
+        for (int j = 0; j < C::NC; ++j) {
+          const int b = (int)(a1 % C::NB);
+          if (!mbar_wait(&a1_empty[b], (uint32_t)((a1 / C::NB) & 1) ^ 1u, p.limit_ns, p.status,
+                         abort_flag) ||
+              !mbar_wait(&w1_full[s1], ph1, p.limit_ns, p.status, abort_flag)) {
+            ok = false;
+            break;
           }
-          if (j >= C::LAG) {
-            const int i = j - C::LAG;
-            const int hb = (int)(hc % C::NH);
-            const uint32_t hph = (uint32_t)((hc / C::NH) & 1);
-            // the output accumulator is free once the previous tile's epilogue read it
-            if ((i == 0 && !mbar_wait(a2_empty, (uint32_t)(t & 1) ^ 1u, p.limit_ns, p.status,
-                                      abort_flag)) ||
-                !mbar_wait(&h_full[hb], hph, p.limit_ns, p.status, abort_flag) ||
-                !mbar_wait(&w2_full[s2], ph2, p.limit_ns, p.status, abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t ha = smem_u32(sH + hb * C::H_BYTES);
-            const uint32_t w2a = smem_u32(sW2 + s2 * C::W2_BYTES);
+          tc_fence_after();
+          const uint64_t wdesc = desc_advance(w1desc0, (uint32_t)(s1 * C::W1_BYTES));
+          const uint32_t d1 = tmem + (uint32_t)(C::ACC1_COL + b * HC);
+          tc_mma_bf16_k<false>(d1, xdesc, wdesc, IDESC1);
 #pragma unroll
-            for (int kk = 0; kk < HC / 16; ++kk)
-              tc_mma_bf16(tmem, smem_desc_sw128(ha) + (uint64_t)(2 * kk),
-                          smem_desc_sw128(w2a) + (uint64_t)(2 * kk), IDESC2,
-                          (i | kk) != 0 ? 1u : 0u);
-            tc_commit(&w2_empty[s2]);
-            tc_commit(&h_empty[hb]);
-            ++hc;
-            if (++s2 == C::S2) {
-              s2 = 0;
-              ph2 ^= 1u;
-            }
+          for (int ks = 1; ks < C::K1_STEPS; ++ks) {
+            const int kb = ks >> 2, kk = ks & 3;
+            tc_mma_bf16_k<true>(d1, desc_advance(xdesc, (uint32_t)(kb * BM * 128 + 32 * kk)),
+                                desc_advance(wdesc, (uint32_t)(kb * HC * 128 + 32 * kk)), IDESC1);
+          }
+          tc_commit(&w1_empty[s1]);
+          tc_commit(&a1_full[b]);
+          ++a1;
+          if (++s1 == C::S1) {
+            s1 = 0;
+            ph1 ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&x_empty[xs]);
+        if (++xs == C::NX) {
+          xs = 0;
+          xph ^= 1u;
+        }
+      }
+      if (!ok) *abort_flag = 1;
+      // no MMA of this thread may still be writing TMEM when it is released
+      tc_commit(drain);
+      mbar_wait(drain, 0, p.limit_ns, p.status);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ fc2 issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC2 = idesc_bf16_f32(BM, D);
+      const uint64_t hdesc0 = smem_desc_sw128(smem_u32(sH));
+      const uint64_t w2desc0 = smem_desc_sw128(smem_u32(sW2));
+      int s2 = 0;
+      uint32_t ph2 = 0, hc = 0, t = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++t) {
+        for (int i = 0; i < C::NC; ++i) {
+          const int hb = (int)(hc % C::NH);
+          // the output accumulator is free once the previous tile's epilogue read it
+          if ((i == 0 && !mbar_wait(a2_empty, (t & 1u) ^ 1u, p.limit_ns, p.status, abort_flag)) ||
+              !mbar_wait(&h_full[hb], (uint32_t)((hc / C::NH) & 1), p.limit_ns, p.status,
+                         abort_flag) ||
+              !mbar_wait(&w2_full[s2], ph2, p.limit_ns, p.status, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t hdesc = desc_advance(hdesc0, (uint32_t)(hb * C::H_BYTES));
+          const uint64_t w2desc = desc_advance(w2desc0, (uint32_t)(s2 * C::W2_BYTES));
+          if (i == 0)
+            tc_mma_bf16_k<false>(tmem, hdesc, w2desc, IDESC2);
+          else
+            tc_mma_bf16_k<true>(tmem, hdesc, w2desc, IDESC2);
+#pragma unroll
+          for (int kk = 1; kk < HC / 16; ++kk)
+            tc_mma_bf16_k<true>(tmem, desc_advance(hdesc, 32u * kk), desc_advance(w2desc, 32u * kk),
+                                IDESC2);
+          tc_commit(&w2_empty[s2]);
+          tc_commit(&h_empty[hb]);
+          ++hc;
+          if (++s2 == C::S2) {
+            s2 = 0;
+            ph2 ^= 1u;
           }
         }
         if (ok) tc_commit(a2_full);
       }
       if (!ok) *abort_flag = 1;
-      // no MMA may still be writing TMEM when it is released
-      tc_commit(drain);
-      mbar_wait(drain, 0, p.limit_ns, p.status);
+      tc_commit(drain2);
+      mbar_wait(drain2, 0, p.limit_ns, p.status);
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int ew = warp - 2;
+    const int ew = warp - 3;
     const int quarter = warp & 3;  // TMEM lanes 32 quarter .. + 31
     const int cg = ew >> 2;        // column group: 16 hidden columns / one 56-column piece
     const int rt = quarter * 32 + lane;
