@@ -60,6 +60,13 @@ def peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+# DRAM bytes (read + write) per GEMM-class launch of this workload, averaged over the 91
+# tc_gemm / mlp_fused launches of one forward, from one ncu capture of the current kernels
+# (the command and numbers are in profiles/gemm_tcgen05_stage2_block_512_b8.md). Must be
+# re-captured, or set to None, whenever those kernels change.
+GEMM_DRAM_BYTES_PER_LAUNCH = 21.62e6
+
+
 def launch_flops(img: int, B: int, fused_mlp: bool = True):
     """Algorithmic FLOPs of every library launch of one backbone forward, in launch order
     (head_dim 56, not the padded 64). Returns list of (kind-class, flops). With fused_mlp,
@@ -336,7 +343,11 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                                               "attention": "mask-unit / global attention"}
                 [dominant],
                 "achieved": dom["tflops"], "peak": tf_sust, "unit": "TFLOP/s",
-                "frac": dom["tflops"] / tf_sust, "traffic": None,
+                "frac": dom["tflops"] / tf_sust,
+                "traffic": GEMM_DRAM_BYTES_PER_LAUNCH if dominant == "gemm" else None,
+                "traffic_note": "dram__bytes_read.sum + dram__bytes_write.sum per GEMM-class "
+                                "launch, ncu, cold caches (profiles/gemm_tcgen05_stage2_block_"
+                                "512_b8.md); algorithmic bytes 40.9e6 per launch",
                 "peak_kind": f"bf16 dense sustained ({peak_src})",
                 "launches_per_step": dom["launches"],
                 "gflop_per_launch": dom["gflop"] / max(dom["launches"], 1),
