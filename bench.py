@@ -67,6 +67,12 @@ def peaks():
 GEMM_DRAM_BYTES_PER_LAUNCH = 21.62e6
 
 
+def reroll_bytes(img: int, B: int):
+    """Algorithmic bytes (read + write, bf16) of the four feature Rerolls, in launch order."""
+    G0 = img // 4
+    return [2 * 2 * B * (G0 >> s) ** 2 * STAGE_DIMS[s] for s in range(4)]
+
+
 def launch_flops(img: int, B: int, fused_mlp: bool = True):
     """Algorithmic FLOPs of every library launch of one backbone forward, in launch order
     (head_dim 56, not the padded 64). Returns list of (kind-class, flops). With fused_mlp,
@@ -331,6 +337,18 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             e["launches"] += 1
             e["ms"] += ms
     step_ms_prof = sum(ms for _, ms in per_launch)
+    rr_ms = [ms for n, ms in per_launch if n == "unroll_reroll"]
+    rr_bytes = reroll_bytes(IMG, B)
+    reroll_hbm = None
+    if len(rr_ms) == len(rr_bytes) and sum(rr_ms) > 0:
+        gbs = sum(rr_bytes) / (sum(rr_ms) * 1e-3) / 1e9
+        big = max(range(len(rr_bytes)), key=lambda i: rr_bytes[i])
+        gbs_big = rr_bytes[big] / (rr_ms[big] * 1e-3) / 1e9
+        reroll_hbm = {"bytes_per_step": sum(rr_bytes), "ms": sum(rr_ms), "gbs": gbs,
+                      "frac_of_hbm": gbs / hbm_gbs, "largest_launch_bytes": rr_bytes[big],
+                      "largest_launch_gbs": gbs_big, "largest_launch_frac": gbs_big / hbm_gbs,
+                      "peak_gbs": hbm_gbs, "note": "event-timed inside the instrumented "
+                      "graph (includes the per-launch event gap)"}
     for e in list(classes.values()) + list(by_kernel.values()):
         e["share"] = e["ms"] / step_ms_prof if step_ms_prof > 0 else None
         e["tflops"] = e["gflop"] / e["ms"] if e["ms"] > 0 else 0.0
@@ -408,6 +426,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "by_kernel": by_kernel,
         "cpu_baseline": cpu,
         "e2e": e2e,
+        "unroll_reroll_hbm": reroll_hbm,
         "clocks": clocks.record(),
         "gpu_launches": n_launches * args.steps,
         "launches_per_step": n_launches,
