@@ -231,6 +231,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     hb.set_option(hb.OPT_FUSED_MLP, 1 if args.mlp == "fused" else 0)
+    hb.set_option(hb.OPT_PDL, 1 if args.pdl == "on" else 0)
     hbm_gbs, tf_burst, tf_sust, peak_src = peaks()
     B = args.batch
 
@@ -417,7 +418,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                    "parallelism": f"replicas x{world} (no data-path collective)",
                    "l2": "flushed before every step (256 MiB write)",
                    "timing": "CUDA-graph replay of the library launches, per-step CUDA events",
-                   "mlp": args.mlp},
+                   "mlp": args.mlp, "pdl": args.pdl},
         "tflops": gflop_per_image * images / (total_ms * 1e-3) * 1e-3,
         "attn_gemm_frac_of_bf16_peak": attn_gemm_gflop / (ms_per_step * 1e-3) / 1e3 / tf_sust,
         "gflop_per_image": gflop_per_image,
@@ -446,6 +447,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--mlp", choices=["fused", "unfused"], default="fused",
                     help="stage-0/1 MLPs as one fused kernel (default) or two GEMMs")
+    ap.add_argument("--pdl", choices=["on", "off"], default="on",
+                    help="programmatic dependent launch between the library's kernels")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

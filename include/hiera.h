@@ -280,10 +280,16 @@ HIERA_API hiera_status hiera_backbone_forward(const hiera_backbone_desc* desc, c
  *                        Summary). 0: the two stand-alone GEMMs with the hidden
  *                        activation in the workspace. Both give the same values (same
  *                        tensor-core K order, same epilogue arithmetic).
+ *   HIERA_OPT_PDL        1 (default): the bf16 path's kernels are launched with programmatic
+ *                        dependent launch, so each one's launch and set-up (barrier init,
+ *                        TMEM allocation, descriptor prefetch) overlap the tail of the
+ *                        kernel before it; every kernel waits (griddepcontrol.wait) for
+ *                        its predecessor's completion before it reads or writes any data
+ *                        a previous kernel touches. 0: ordinary stream-ordered launches.
  * hiera_set_option returns HIERA_ERR_INVALID_ARG for an unknown option or value;
  * hiera_get_option returns the current value (0 for an unknown option).
  * -------------------------------------------------------------------------------- */
-typedef enum { HIERA_OPT_FUSED_MLP = 0, HIERA_OPT_COUNT = 1 } hiera_option;
+typedef enum { HIERA_OPT_FUSED_MLP = 0, HIERA_OPT_PDL = 1, HIERA_OPT_COUNT = 2 } hiera_option;
 HIERA_API hiera_status hiera_set_option(hiera_option opt, int value);
 HIERA_API int hiera_get_option(hiera_option opt);
 

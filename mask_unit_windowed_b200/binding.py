@@ -387,6 +387,7 @@ def kernel_name(kind: int) -> str:
 
 # ----------------------------------------------------------------------------- options
 OPT_FUSED_MLP = 0
+OPT_PDL = 1
 
 
 def set_option(opt: int, value: int):
@@ -397,20 +398,30 @@ def get_option(opt: int) -> int:
     return lib().hiera_get_option(opt)
 
 
-class fused_mlp:
-    """Context manager: run the block MLPs fused (True, the default) or as two GEMMs."""
+class option:
+    """Context manager: set a library option for the duration of a block of calls."""
 
-    def __init__(self, enabled: bool):
-        self.enabled = bool(enabled)
+    def __init__(self, opt: int, value: int):
+        self.opt, self.value = opt, int(value)
 
     def __enter__(self):
-        self._old = get_option(OPT_FUSED_MLP)
-        set_option(OPT_FUSED_MLP, int(self.enabled))
+        self._old = get_option(self.opt)
+        set_option(self.opt, self.value)
         return self
 
     def __exit__(self, *exc):
-        set_option(OPT_FUSED_MLP, self._old)
+        set_option(self.opt, self._old)
         return False
+
+
+def fused_mlp(enabled: bool) -> option:
+    """Run the block MLPs fused (True, the default) or as two GEMMs."""
+    return option(OPT_FUSED_MLP, bool(enabled))
+
+
+def pdl(enabled: bool) -> option:
+    """Launch with programmatic dependent launch (True, the default) or plain launches."""
+    return option(OPT_PDL, bool(enabled))
 
 
 class LaunchProfile:

@@ -596,7 +596,7 @@ void profile_mark(int kind, cudaStream_t stream) {
 }
 
 namespace {
-int g_options[HIERA_OPT_COUNT] = {1};  // HIERA_OPT_FUSED_MLP on
+int g_options[HIERA_OPT_COUNT] = {1, 1};  // fused MLP on, programmatic dependent launch on
 }  // namespace
 
 int g_option(int opt) { return (opt >= 0 && opt < HIERA_OPT_COUNT) ? g_options[opt] : 0; }
@@ -918,7 +918,7 @@ int hiera_profile_end(hiera_stream_t stream) {
 
 hiera_status hiera_set_option(hiera_option opt, int value) {
   if (opt < 0 || opt >= HIERA_OPT_COUNT) return HIERA_ERR_INVALID_ARG;
-  if (opt == HIERA_OPT_FUSED_MLP && value != 0 && value != 1) return HIERA_ERR_INVALID_ARG;
+  if (value != 0 && value != 1) return HIERA_ERR_INVALID_ARG;
   g_options[opt] = value;
   return HIERA_OK;
 }

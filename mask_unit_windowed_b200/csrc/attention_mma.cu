@@ -213,6 +213,8 @@ struct KArgs {
 
 // tiled mode: blockIdx.x = unit (b, w, h), blockIdx.y = 64-row query tile
 __global__ void __launch_bounds__(128) attn_tiled_kernel(const KArgs p) {
+  griddep_wait();  // everything below reads or writes data of earlier kernels
+  griddep_launch_dependents();
   __shared__ __align__(1024) uint8_t smem[8192 + 2 * 2 * 8192];
   const uint32_t sQ = smem_u32(smem);
   const uint32_t sKV = sQ + 8192;  // [buf][K|V] 8 KB each
@@ -261,6 +263,8 @@ __global__ void __launch_bounds__(128) attn_tiled_kernel(const KArgs p) {
 // packed mode: 4 units per CTA, one per warp; Tq <= 16 and Tkv <= KEYS
 template <int KEYS>
 __global__ void __launch_bounds__(128) attn_packed_kernel(const KArgs p) {
+  griddep_wait();  // everything below reads or writes data of earlier kernels
+  griddep_launch_dependents();
   constexpr int WARP_BYTES = 2048 + 2 * KEYS * 128;
   extern __shared__ __align__(1024) uint8_t smem[];  // 4 * WARP_BYTES
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -307,7 +311,7 @@ hiera_status launch_attention_bf16(const AttnArgs& a, cudaStream_t stream) {
   if (p.units <= 0 || a.Tq <= 0 || a.Tkv <= 0) return HIERA_OK;
   profile_mark(a.Tq <= 16 && a.Tkv <= 64 ? K_ATTN_PACKED : K_ATTN_TILED, stream);
   if (a.Tq <= 16 && a.Tkv <= 16) {
-    attn_packed_kernel<16><<<(p.units + 3) / 4, 128, 4 * (2048 + 2 * 16 * 128), stream>>>(p);
+    launch_k(attn_packed_kernel<16>, dim3((p.units + 3) / 4), dim3(128), 4 * (2048 + 2 * 16 * 128), stream, p);
   } else if (a.Tq <= 16 && a.Tkv <= 64) {
     constexpr int bytes = 4 * (2048 + 2 * 64 * 128);
     static bool attr_done[64] = {false};
@@ -319,11 +323,11 @@ hiera_status launch_attention_bf16(const AttnArgs& a, cudaStream_t stream) {
         return HIERA_ERR_CUDA;
       attr_done[dev] = true;
     }
-    attn_packed_kernel<64><<<(p.units + 3) / 4, 128, bytes, stream>>>(p);
+    launch_k(attn_packed_kernel<64>, dim3((p.units + 3) / 4), dim3(128), bytes, stream, p);
   } else {
     dim3 grid(p.units, (a.Tq + 63) / 64);
     if (grid.y > 65535) return HIERA_ERR_SHAPE;
-    attn_tiled_kernel<<<grid, 128, 0, stream>>>(p);
+    launch_k(attn_tiled_kernel, grid, dim3(128), 0, stream, p);
   }
   return cudaGetLastError() == cudaSuccess ? HIERA_OK : HIERA_ERR_CUDA;
 }

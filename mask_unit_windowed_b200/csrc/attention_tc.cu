@@ -114,6 +114,8 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  griddep_wait();  // everything below reads or writes data of earlier kernels
+  griddep_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -398,7 +400,7 @@ hiera_status launch_attention_tc(const AttnArgs& a, cudaStream_t stream) {
   dim3 grid((a.Tq + 2 * QT - 1) / (2 * QT), units);
   if (grid.y > 65535) return HIERA_ERR_SHAPE;
   profile_mark(K_ATTN_TC, stream);
-  attn_tc_kernel<<<grid, 320, SMEM_BYTES, stream>>>(tmQ, tmK, tmV, p);
+  launch_k(attn_tc_kernel, grid, dim3(320), SMEM_BYTES, stream, tmQ, tmK, tmV, p);
   return cudaGetLastError() == cudaSuccess ? HIERA_OK : HIERA_ERR_CUDA;
 }
 

@@ -86,6 +86,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
   }
 }
 
+// Programmatic dependent launch: wait until the grids this one depends on have completed
+// and their memory is visible (a no-op when the launch had no such dependency), and let
+// the next grid of the stream start its launch and set-up.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Orders this thread's prior generic-proxy shared-memory accesses before later
 // async-proxy (TMA / tensor-core) accesses of the same memory.
 __device__ __forceinline__ void fence_proxy_async_smem() {

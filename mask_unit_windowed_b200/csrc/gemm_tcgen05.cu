@@ -136,6 +136,8 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  griddep_wait();  // everything below reads or writes data of earlier kernels
+  griddep_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -577,7 +579,7 @@ hiera_status run(const TcGemmArgs& a, cudaStream_t stream) {
   if (grid > tiles) grid = tiles;
   profile_mark(EPI == EPI_QKV ? K_GEMM_QKV : (EPI == EPI_GELU ? K_GEMM_GELU : K_GEMM_STORE),
                stream);
-  kern<<<grid, 320, C::SMEM_BYTES, stream>>>(tmA, tmB, p);
+  launch_k(kern, dim3(grid), dim3(320), C::SMEM_BYTES, stream, tmA, tmB, p);
   return cudaGetLastError() == cudaSuccess ? HIERA_OK : HIERA_ERR_CUDA;
 }
 

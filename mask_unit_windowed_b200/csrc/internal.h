@@ -79,6 +79,25 @@ bool mlp_fused_supported(int d);
 hiera_status launch_mlp_fused(const MlpArgs& a, cudaStream_t stream);
 int g_option(int opt);      // library options (hiera_set_option)
 
+// Launch on `stream`, with programmatic dependent launch unless HIERA_OPT_PDL is off. A
+// kernel launched this way must execute griddep_wait() (common.cuh) before it reads or
+// writes global memory that another kernel of the stream writes or reads.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                     cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = g_option(HIERA_OPT_PDL) ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
+}
+
 // N-tile width the plain-store GEMM uses for N output columns (N a multiple of 16).
 inline int store_bn(int N) {
   return N % 224 == 0 ? 224 : N % 128 == 0 ? 128 : N % 112 == 0 ? 112 : N % 64 == 0 ? 64

@@ -200,6 +200,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  griddep_wait();  // everything below reads or writes data of earlier kernels
+  griddep_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -603,7 +605,7 @@ hiera_status run_mlp(const MlpArgs& a, cudaStream_t stream) {
   int grid = g_num_sms();
   if (grid > tiles) grid = tiles;
   profile_mark(K_MLP_FUSED, stream);
-  kern<<<grid, THREADS, C::SMEM_BYTES, stream>>>(tmX, tmW1, tmW2, p);
+  launch_k(kern, dim3(grid), dim3(THREADS), C::SMEM_BYTES, stream, tmX, tmW1, tmW2, p);
   return cudaGetLastError() == cudaSuccess ? HIERA_OK : HIERA_ERR_CUDA;
 }
 

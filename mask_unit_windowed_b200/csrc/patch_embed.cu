@@ -130,6 +130,8 @@ __global__ void __launch_bounds__(256, 1) patch_embed_mma_kernel(
     const bf16* __restrict__ img, const bf16* __restrict__ w16, const float* __restrict__ bias,
     const bf16* __restrict__ pos, bf16* __restrict__ out, float2* __restrict__ stats_out,
     int img_side) {
+  griddep_wait();  // everything below reads or writes data of earlier kernels
+  griddep_launch_dependents();
   extern __shared__ __align__(16) uint8_t smem_pe[];
   bf16* sW = reinterpret_cast<bf16*>(smem_pe);                       // [112][WPITCH]
   bf16* sIn = sW + PATCH_CO * WPITCH;                                // [7][IN_PITCH][4]
@@ -268,9 +270,9 @@ hiera_status launch_patch_embed(const void* img, const void* packed, const void*
         return HIERA_ERR_CUDA;
       attr_done[1][dev] = true;
     }
-    patch_embed_mma_kernel<<<grid, 256, MMA_SMEM, stream>>>(
-        static_cast<const bf16*>(img), w16, bias, static_cast<const bf16*>(pos),
-        static_cast<bf16*>(out), stats_out, img_side);
+    launch_k(patch_embed_mma_kernel, grid, dim3(256), MMA_SMEM, stream,
+             static_cast<const bf16*>(img), w16, bias, static_cast<const bf16*>(pos),
+             static_cast<bf16*>(out), stats_out, img_side);
   } else {
     dim3 grid((G + SEG - 1) / SEG, (G + ROWS - 1) / ROWS, B);
     if (grid.y > 65535 || grid.z > 65535) return HIERA_ERR_SHAPE;

@@ -13,6 +13,8 @@ __global__ void __launch_bounds__(256) permute_kernel(const uint4* __restrict__ 
                                                       uint4* __restrict__ dst, int B, int G,
                                                       int L, int chunks_per_row,
                                                       long long total) {
+  griddep_wait();  // everything below reads or writes data of earlier kernels
+  griddep_launch_dependents();
   const int M = G >> L;
   const int N = G * G;
   const long long stride = (long long)gridDim.x * blockDim.x;
@@ -41,13 +43,13 @@ cudaError_t launch_permute(bool unroll, const void* x, void* y, int B, int G, in
   const long long cap = (long long)g_num_sms() * 16;
   if (blocks > cap) blocks = cap;
   profile_mark(K_PERMUTE, stream);
+  const uint4* src = static_cast<const uint4*>(x);
+  uint4* dst = static_cast<uint4*>(y);
   if (unroll)
-    permute_kernel<true><<<(int)blocks, 256, 0, stream>>>(
-        static_cast<const uint4*>(x), static_cast<uint4*>(y), B, G, L, chunks, total);
-  else
-    permute_kernel<false><<<(int)blocks, 256, 0, stream>>>(
-        static_cast<const uint4*>(x), static_cast<uint4*>(y), B, G, L, chunks, total);
-  return cudaGetLastError();
+    return launch_k(permute_kernel<true>, dim3((unsigned)blocks), dim3(256), 0, stream, src,
+                    dst, B, G, L, chunks, total);
+  return launch_k(permute_kernel<false>, dim3((unsigned)blocks), dim3(256), 0, stream, src, dst,
+                  B, G, L, chunks, total);
 }
 
 }  // namespace hiera

@@ -10,6 +10,8 @@ namespace {
 
 __global__ void __launch_bounds__(256) row_partials_bf16_kernel(const bf16* __restrict__ x, int M,
                                                                 int K, float2* __restrict__ out) {
+  griddep_wait();  // everything below reads or writes data of earlier kernels
+  griddep_launch_dependents();
   const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (row >= M) return;
@@ -43,9 +45,10 @@ hiera_status launch_row_partials_bf16(const void* x, int M, int K, float2* out,
   if (K % 8 != 0) return HIERA_ERR_SHAPE;
   const long long threads = (long long)M * 32;
   profile_mark(K_ROW_STATS, stream);
-  row_partials_bf16_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, stream>>>(
-      static_cast<const bf16*>(x), M, K, out);
-  return cudaGetLastError() == cudaSuccess ? HIERA_OK : HIERA_ERR_CUDA;
+  const cudaError_t e =
+      launch_k(row_partials_bf16_kernel, dim3((unsigned)((threads + 255) / 256)), dim3(256), 0,
+               stream, static_cast<const bf16*>(x), M, K, out);
+  return e == cudaSuccess ? HIERA_OK : HIERA_ERR_CUDA;
 }
 
 }  // namespace hiera

@@ -87,8 +87,29 @@ def test_fused_mlp_backbone_bitwise():
         assert torch.equal(a, b)
 
 
+def test_backbone_same_with_and_without_programmatic_launch():
+    """Programmatic dependent launch only changes when kernels start their set-up; every
+    kernel still waits for its predecessor, so the features are bit-identical."""
+    img, B = 64, 2
+    p = syn.backbone_params(64, img, dtype="bf16", affine="random")
+    x = dev(syn.image(64, B, img, dtype="bf16"), "bf16")
+    desc = hb.BackboneDesc(B=B, img=img)
+    w = {"patch_w": dev(p["patch_w"]), "patch_b": dev(p["patch_b"]),
+         "pos_embed": dev(p["pos_embed"]),
+         "blocks": [{k: dev(v) for k, v in b.items()} for b in p["blocks"]]}
+    packed = hb.backbone_pack(desc, w)
+    outs = []
+    for on in (True, False):
+        with hb.pdl(on):
+            outs.append(hb.backbone_forward(desc, packed, x))
+            assert hb.device_status() == 0
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
+
+
 def test_option_api():
     assert hb.get_option(hb.OPT_FUSED_MLP) == 1
+    assert hb.get_option(hb.OPT_PDL) == 1
     with pytest.raises(hb.HieraError):
         hb.set_option(hb.OPT_FUSED_MLP, 2)
     with pytest.raises(hb.HieraError):
