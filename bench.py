@@ -212,8 +212,12 @@ def run_reference(args, rank: int):
             "n_gpus": args.gpus, "steps": steps, "warmup": min(args.warmup, 1),
             "ms_per_step": 1000.0 / value, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"Hiera-B+ backbone forward, {IMG}x{IMG}x4 image, batch 1 "
-                                   "per step, CPU oracle", "img": IMG},
+            "config": {"workload": f"Hiera-B+ backbone forward, {IMG}x{IMG}x4 bf16 images, "
+                                   f"batch {args.batch} per GPU (random-init weights, seed "
+                                   f"{SEED})", "img": IMG, "batch_per_gpu": args.batch,
+                       "global_batch": args.batch,
+                       "sample": "each timed step runs one image of the batch through the "
+                                 "CPU oracle (bf16-valued inputs, fp64 arithmetic)"},
             "cpu_baseline": cpu,
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
