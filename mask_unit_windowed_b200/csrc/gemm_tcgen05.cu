@@ -71,14 +71,16 @@ struct Cfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STG_BYTES = 8 * 32 * 128;  // per epilogue warp: 32 rows x 128 B staging
   static constexpr int STAGES =
-      cmin(8, (227 * 1024 - 1024 - 256 - 2 * BN * 4 - 128 - STG_BYTES) / STAGE_BYTES);
+      cmin(8, (227 * 1024 - 1024 - 256 - EPI_WARPS * BN * 4 - 128 - STG_BYTES) / STAGE_BYTES);
   static constexpr int ACC_STRIDE = BN <= 128 ? 128 : 256;
   static constexpr int TMEM_COLS = 2 * ACC_STRIDE;
   static constexpr int HALF = BN / 2;                    // columns per epilogue thread
   static constexpr int CH = (HALF % 56 == 0) ? 56 : cmin(HALF, 32);  // columns per chunk
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
-  static constexpr int CONST_OFF = BAR_OFF + 256;        // colsum[BN], colconst[BN] (fp32)
-  static constexpr int STG_OFF = (CONST_OFF + 2 * BN * 4 + 127) / 128 * 128;
+  // per epilogue warp: colsum and colconst (fp32) of its half of the tile's columns
+  static constexpr int CONST_OFF = BAR_OFF + 256;
+  static constexpr int CONST_BYTES = EPI_WARPS * 2 * (BN / 2) * 4;
+  static constexpr int STG_OFF = (CONST_OFF + CONST_BYTES + 127) / 128 * 128;
   static constexpr int SMEM_BYTES = STG_OFF + STG_BYTES + 1024;
   static_assert(B_BYTES % 1024 == 0, "W tile must keep 1024-byte alignment");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128");
@@ -103,8 +105,6 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* col_sum = reinterpret_cast<float*>(smem + C::CONST_OFF);
-  float* col_const = col_sum + BN;
   uint8_t* stg_all = smem + C::STG_OFF;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -269,20 +269,33 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
       for (int j = 0; j < 8; ++j) part[j] = j < P ? __ldg(sp + j) : make_float2(0.f, 0.f);
     };
-    // this thread's share of a tile's column constants (BN <= 256 columns, one per thread),
-    // also loaded one tile ahead and staged in shared memory at the tile's start
-    const int etid = ew * 32 + lane;
-    float nsum = 0.f, nconst = 0.f;
+    // This warp's column constants (its half of the tile's columns) live in its own
+    // shared-memory slots, so moving to the next tile needs no barrier with the other
+    // epilogue warps. They are loaded a tile ahead, CPL per lane, and staged at the tile's
+    // start.
+    constexpr int CPL = (HALF + 31) / 32;
+    float* col_sum = reinterpret_cast<float*>(smem + C::CONST_OFF) + ew * 2 * HALF;
+    float* col_const = col_sum + HALF;
+    float nsum[CPL], nconst[CPL];
     auto load_consts = [&](int tile) {
-      const int c = (tile - (tile / n_tiles) * n_tiles) * BN + etid;
-      if (etid < BN) {
-        nsum = FOLD ? __ldg(p.colsum + c) : 0.f;
-        nconst = p.colconst != nullptr ? __ldg(p.colconst + c)
-                 : (p.bias16 != nullptr ? __bfloat162float(p.bias16[c]) : 0.f);
+      const int c0 = (tile - (tile / n_tiles) * n_tiles) * BN + c_begin;
+#pragma unroll
+      for (int k = 0; k < CPL; ++k) {
+        const int i = lane + 32 * k;
+        nsum[k] = 0.f;
+        nconst[k] = 0.f;
+        if (i < HALF) {
+          const int c = c0 + i;
+          nsum[k] = FOLD ? __ldg(p.colsum + c) : 0.f;
+          nconst[k] = p.colconst != nullptr ? __ldg(p.colconst + c)
+                      : (p.bias16 != nullptr ? __bfloat162float(p.bias16[c]) : 0.f);
+        }
       }
     };
-    if ((int)blockIdx.x < num_tiles) {
-      if (FOLD) load_parts(blockIdx.x);
+    // the store epilogue (residual prefetch already holds many registers, few tiles per
+    // CTA) loads them at the tile's start instead
+    if ((int)blockIdx.x < num_tiles && FOLD) {
+      load_parts(blockIdx.x);
       load_consts(blockIdx.x);
     }
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
@@ -317,15 +330,20 @@ __global__ void __launch_bounds__(320, 1)
       // LayerNorm statistics of this row, merged from the producer's partials
       float fa = 1.f, fb = 0.f;  // v = fa * acc + fb * colsum + colconst
       if (FOLD && row_ok) ln_merge_parts(part, p.stats_parts, p.K, p.ln_eps, fa, fb);
-      // per-column constants of this tile into shared memory (loaded a tile ahead)
-      named_bar_sync(1, EPI_THREADS);  // every epilogue thread is done with the last tile's
-      if (etid < BN) {
-        col_sum[etid] = nsum;
-        col_const[etid] = nconst;
+      // this warp's column constants of this tile into its slots (loaded a tile ahead)
+      if (!FOLD) load_consts(tile);
+      __syncwarp();  // every lane is done with the last tile's
+#pragma unroll
+      for (int k = 0; k < CPL; ++k) {
+        const int i = lane + 32 * k;
+        if (i < HALF) {
+          col_sum[i] = nsum[k];
+          col_const[i] = nconst[k];
+        }
       }
-      named_bar_sync(1, EPI_THREADS);
-      if (tile + (int)gridDim.x < num_tiles) {
-        if (FOLD) load_parts(tile + gridDim.x);
+      __syncwarp();
+      if (FOLD && tile + (int)gridDim.x < num_tiles) {
+        load_parts(tile + gridDim.x);
         load_consts(tile + gridDim.x);
       }
       if (!warp_wait(&acc_full[acc], aph, p.limit_ns, p.status, abort_flag)) break;
@@ -343,7 +361,7 @@ __global__ void __launch_bounds__(320, 1)
         float v[CH];
 #pragma unroll
         for (int i = 0; i < CH; ++i) {
-          const int cl = c_begin + c + i;
+          const int cl = c + i;  // column within this warp's half
           float x = FOLD ? fmaf(fa, __uint_as_float(r[i]), fmaf(fb, col_sum[cl], col_const[cl]))
                          : __uint_as_float(r[i]) + col_const[cl];
           if (EPI == EPI_GELU) x = gelu_fast(x);
