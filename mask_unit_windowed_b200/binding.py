@@ -359,6 +359,74 @@ def backbone_forward(desc: BackboneDesc, packed, img, feats=None, workspace=None
     return feats
 
 
+class BackbonePipeline:
+    """Host-to-host inference over consecutive batches on one device.
+
+    For each batch: upload the image from pinned host memory, run hiera_backbone_forward,
+    download the four features into pinned host memory. Uploads, the forward calls and
+    downloads go to three streams with two device buffer sets, so the copies of a batch
+    overlap the compute of its neighbours; the forwards themselves run one after another on
+    the compute stream (they share one workspace).
+
+        pipe = BackbonePipeline(desc, packed)
+        pipe.run(host_images, host_features)   # lists of pinned CPU tensors, one per batch
+        pipe.synchronize()
+    """
+
+    def __init__(self, desc: BackboneDesc, packed: torch.Tensor, device=None):
+        self.desc, self.packed = desc, packed
+        dev = packed.device if device is None else torch.device(device)
+        shape = (desc.B, desc.img, desc.img, 4)
+        self.imgs = [torch.empty(shape, dtype=desc.dtype, device=dev) for _ in range(2)]
+        self.feats = [[torch.empty(s, dtype=desc.dtype, device=dev)
+                       for s in desc.feature_shapes()] for _ in range(2)]
+        self.ws = torch.empty(backbone_workspace_bytes(desc), dtype=torch.uint8, device=dev)
+        self.s_in = torch.cuda.Stream(device=dev)
+        self.s_comp = torch.cuda.Stream(device=dev)
+        self.s_out = torch.cuda.Stream(device=dev)
+        self._ev = {k: [torch.cuda.Event() for _ in range(2)] for k in ("in", "comp", "out")}
+        self._count = 0
+
+    def host_feature_buffers(self):
+        """A set of pinned host tensors shaped like one batch's features."""
+        return [torch.empty(s, dtype=self.desc.dtype, pin_memory=True)
+                for s in self.desc.feature_shapes()]
+
+    def run(self, host_images, host_features, start_event=None, end_event=None):
+        """Enqueue one upload / forward / download per batch. host_features[k] receives the
+        features of host_images[k] (the same set may be passed for several batches: the
+        downloads are ordered). Returns without waiting; see synchronize()."""
+        ev_in, ev_comp, ev_out = self._ev["in"], self._ev["comp"], self._ev["out"]
+        if start_event is not None:
+            start_event.record(self.s_in)
+        for h_img, h_feats in zip(host_images, host_features):
+            i = self._count % 2
+            if self._count >= 2:
+                self.s_in.wait_event(ev_comp[i])    # device image buffer i is free again
+            with torch.cuda.stream(self.s_in):
+                self.imgs[i].copy_(h_img, non_blocking=True)
+            ev_in[i].record(self.s_in)
+            self.s_comp.wait_event(ev_in[i])
+            if self._count >= 2:
+                self.s_comp.wait_event(ev_out[i])   # feature buffers i were downloaded
+            backbone_forward(self.desc, self.packed, self.imgs[i], feats=self.feats[i],
+                             workspace=self.ws, stream=self.s_comp)
+            ev_comp[i].record(self.s_comp)
+            self.s_out.wait_event(ev_comp[i])
+            with torch.cuda.stream(self.s_out):
+                for hf, f in zip(h_feats, self.feats[i]):
+                    hf.copy_(f, non_blocking=True)
+            ev_out[i].record(self.s_out)
+            self._count += 1
+        if end_event is not None:
+            end_event.record(self.s_out)
+
+    def synchronize(self):
+        self.s_out.synchronize()
+        self.s_comp.synchronize()
+        self.s_in.synchronize()
+
+
 # ----------------------------------------------------------------------------- status
 def device_status(stream=None) -> int:
     """Synchronise and return (then clear) the first device-side error code."""

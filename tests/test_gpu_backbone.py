@@ -157,3 +157,23 @@ def test_transition_block_65536_tokens_sampled_rows():
     ref = U.block_forward_rows(x, p, 8, 4, 16, False, rows)
     got = np.stack([y[b, n] for b, n in rows])
     assert rel_l2(got, ref) <= 1e-2
+
+
+def test_backbone_pipeline_host_to_host_bitwise():
+    """binding.BackbonePipeline (uploads, forward and downloads of consecutive batches
+    overlapping on three streams) gives every batch the same features as a plain call."""
+    img, B = 64, 2
+    p = syn.backbone_params(71, img, dtype="bf16", affine="random")
+    desc = hb.BackboneDesc(B=B, img=img)
+    packed = hb.backbone_pack(desc, weights_dev(p, "bf16"))
+    hosts = [torch.from_numpy(syn.image(71 + k, B, img, dtype="bf16")).to(torch.bfloat16)
+             .pin_memory() for k in range(5)]
+    pipe = hb.BackbonePipeline(desc, packed)
+    outs = [pipe.host_feature_buffers() for _ in hosts]
+    pipe.run(hosts, outs)
+    pipe.synchronize()
+    assert hb.device_status() == 0
+    for h, o in zip(hosts, outs):
+        ref = hb.backbone_forward(desc, packed, h.cuda())
+        for a, b in zip(o, ref):
+            assert torch.equal(a, b.cpu())
