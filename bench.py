@@ -61,9 +61,9 @@ def peaks():
 
 
 # DRAM bytes (read + write) per GEMM-class launch of this workload, averaged over the 91
-# tc_gemm / mlp_fused launches of one forward, from one ncu capture of the current kernels
-# (the command and numbers are in profiles/gemm_tcgen05_stage2_block_512_b8.md). Must be
-# re-captured, or set to None, whenever those kernels change.
+# tc_gemm / mlp_fused launches of the first forward, from one ncu capture of the current
+# kernels (dram__bytes_read.sum + dram__bytes_write.sum, cold caches). Must be re-captured,
+# or set to None, whenever those kernels change.
 GEMM_DRAM_BYTES_PER_LAUNCH = 21.61e6
 
 
@@ -369,8 +369,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                 "frac": dom["tflops"] / tf_sust,
                 "traffic": GEMM_DRAM_BYTES_PER_LAUNCH if dominant == "gemm" else None,
                 "traffic_note": "dram__bytes_read.sum + dram__bytes_write.sum per GEMM-class "
-                                "launch, ncu, cold caches (profiles/gemm_tcgen05_stage2_block_"
-                                "512_b8.md); algorithmic bytes 40.9e6 per launch",
+                                "launch, one ncu capture, cold caches; algorithmic bytes "
+                                "40.9e6 per launch",
                 "peak_kind": f"bf16 dense sustained ({peak_src})",
                 "launches_per_step": dom["launches"],
                 "gflop_per_launch": dom["gflop"] / max(dom["launches"], 1),

@@ -8,7 +8,7 @@ in 4 stages, Reroll, stage transitions, MaskUnitAttention, MLP) and section
 "Sub-phase 4a: Core backbone module" (unroll, reroll, undo_windowing,
 MaskUnitAttention, HieraMLP, HieraBlock, HieraBackbone).
 
-Readings taken where the plan is silent (each restated in the design doc):
+Readings taken where the plan is silent:
   * Unroll order: a stage-s grid of side G with L = 3 - s unroll levels and mask-unit
     grid side M = G / 2^L puts spatial (y, x), y = my*2^L + sum_k a_k 2^(k-1),
     x = mx*2^L + sum_k b_k 2^(k-1), at token
