@@ -6,14 +6,15 @@
 //   warp 0      TMA: both Q tiles once, then K (128 keys x 64) and V^T (64 x 128 keys) tiles
 //               through a KV_STAGES-deep ring shared by the two query tiles.
 //   warp 1      TMEM owner and MMA issuer: S_t = Q_t K_j^T (M=128, N=128, K=64) and
-//               O_t += P_t V_j (M=128, N=64, K=128) for t = A, B, interleaved so that the
+//               O_t += P_t V_j (M=128, N=64, K=128; P_t from TMEM) for t = A, B, so that the
 //               tensor core works on one tile while the other tile's softmax runs.
 //   warps 2-5   softmax of tile A, warps 6-9 of tile B, one query row per thread (TMEM lane
 //               = row): row max, then the weights P = 2^(s log2(e)/sqrt(56) - m) on the
 //               MUFU unit, rounded to bf16 with integer operations (the conversion unit
-//               shares the MUFU pipe) into the PV's A operand in shared memory. The running
-//               max is raised, and O rescaled in TMEM, only when a tile's max exceeds it by
-//               more than 2^8, so P entries stay below 256.
+//               shares the MUFU pipe) and stored as bf16 pairs into TMEM next to S and O;
+//               the PV product reads its A operand (P) from there, so P never goes through
+//               shared memory. The running max is raised, and O rescaled in TMEM, only when
+//               a tile's max exceeds it by more than 2^8, so P entries stay below 256.
 // head_dim 56 is padded to 64: q/k channels 56..63 are zero; v^T padding row 56 is one, so
 // column 56 of O accumulates the softmax denominator from the very P values the tensor core
 // used; the output is O[:, :56] / O[:, 56].
@@ -32,14 +33,13 @@ constexpr int Q_BYTES = QT * 128;                // [128 q][64 ch] bf16
 constexpr int K_BYTES = KT * 128;                // [128 keys][64 ch]
 constexpr int V_BYTES = 2 * 64 * 128;            // two [64 ch][64 keys] blocks of V^T
 constexpr int KV_BYTES = K_BYTES + V_BYTES;
-constexpr int P_BYTES = 2 * QT * 128;            // two [128 q][64 keys] blocks
 constexpr int OFF_Q = 0;                         // Q_A, Q_B
 constexpr int OFF_KV = OFF_Q + 2 * Q_BYTES;
-constexpr int OFF_P = OFF_KV + KV_STAGES * KV_BYTES;  // P_A, P_B
-constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
+constexpr int OFF_BAR = OFF_KV + KV_STAGES * KV_BYTES;
 constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;
-constexpr uint32_t TMEM_COLS = 512;              // S_A, S_B [0,256), O_A, O_B [256,384)
+constexpr uint32_t TMEM_COLS = 512;  // S_A, S_B [0,256), O_A, O_B [256,384), P_A, P_B [384,512)
 constexpr uint32_t O_COL = 256;
+constexpr uint32_t P_COL = 384;      // P as bf16 pairs: 128 keys in 64 columns per tile
 constexpr float RESCALE_LOG2 = 8.f;              // raise the running max past 2^8 only
 
 struct AParams {
@@ -196,17 +196,17 @@ __global__ void __launch_bounds__(320, 1)
               break;
             }
             tc_fence_after();
-            const uint64_t pdesc = desc_advance(desc0, (uint32_t)(OFF_P + t * P_BYTES));
+            const uint32_t pa = tmem + P_COL + (uint32_t)(t * 64);  // P_t in TMEM
             const uint32_t od = tmem + O_COL + (uint32_t)(t * 64);
             if (jj == 0)
-              tc_mma_bf16_k<false>(od, pdesc, vdesc, IDESC_O);
+              tc_mma_bf16_ta<false>(od, pa, vdesc, IDESC_O);
             else
-              tc_mma_bf16_k<true>(od, pdesc, vdesc, IDESC_O);
+              tc_mma_bf16_ta<true>(od, pa, vdesc, IDESC_O);
 #pragma unroll
             for (int kk = 1; kk < 8; ++kk) {
               const uint32_t blk = kk >> 2, k4 = kk & 3;
-              tc_mma_bf16_k<true>(od, desc_advance(pdesc, blk * (QT * 128) + 32u * k4),
-                                  desc_advance(vdesc, blk * (64 * 128) + 32u * k4), IDESC_O);
+              tc_mma_bf16_ta<true>(od, pa + 8u * kk,
+                                   desc_advance(vdesc, blk * (64 * 128) + 32u * k4), IDESC_O);
             }
             tc_commit(&o_done[t]);
             tc_commit(&p_free[t]);
@@ -230,7 +230,7 @@ __global__ void __launch_bounds__(320, 1)
     const float thr = RESCALE_LOG2 / sl2;  // in raw score units
     float m_run = -INFINITY;
     bool ok = true;
-    uint8_t* pb = smem + OFF_P + t * P_BYTES + r * 128;
+    const uint32_t p_col = P_COL + (uint32_t)(t * 64);
     for (int j = 0; j < n_tiles; ++j) {
       if (!warp_wait(&s_full[t], (uint32_t)(j & 1), p, abort_flag)) {
         ok = false;
@@ -276,18 +276,17 @@ __global__ void __launch_bounds__(320, 1)
         ok = false;
         break;
       }
+      // P of this row as bf16 pairs straight into TMEM (lane = row), 64 keys per store
 #pragma unroll
-      for (int c = 0; c < KT / 8; ++c) {
-        uint4 pk;
-        uint32_t* w4 = reinterpret_cast<uint32_t*>(&pk);
+      for (int h = 0; h < 2; ++h) {
+        uint32_t pw[32];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float x0 = fmaf(__uint_as_float(sr[8 * c + 2 * u]), sl2, -ms);   // -inf -> 0
-          const float x1 = fmaf(__uint_as_float(sr[8 * c + 2 * u + 1]), sl2, -ms);
-          w4[u] = pack_bf16x2_int(ex2_approx(x0), ex2_approx(x1));
+        for (int u = 0; u < 32; ++u) {
+          const float x0 = fmaf(__uint_as_float(sr[64 * h + 2 * u]), sl2, -ms);   // -inf -> 0
+          const float x1 = fmaf(__uint_as_float(sr[64 * h + 2 * u + 1]), sl2, -ms);
+          pw[u] = pack_bf16x2_int(ex2_approx(x0), ex2_approx(x1));
         }
-        const int blk = c >> 3, cc = c & 7;
-        *reinterpret_cast<uint4*>(pb + blk * (QT * 128) + ((cc ^ (r & 7)) << 4)) = pk;
+        tc_st_32x32b_x32(lane_base + p_col + (uint32_t)(32 * h), pw);
       }
       if (__any_sync(0xffffffffu, resc)) {
         // O_t holds the sum through tile j-1 (its PV completed above): rescale these rows
@@ -307,7 +306,7 @@ __global__ void __launch_bounds__(320, 1)
         }
         tc_wait_st();
       }
-      fence_proxy_async_smem();  // P (generic stores) before the tensor core reads it
+      tc_wait_st();  // P (and any rescaled O) written before the tensor core reads them
       tc_fence_before();
       mbar_arrive(&p_full[t]);
     }

@@ -297,6 +297,26 @@ __device__ __forceinline__ void tc_mma_bf16_k(uint32_t d_tmem, uint64_t a_desc, 
   }
 }
 
+// The same with the A operand in tensor memory: M = 128 rows in the 128 lanes, K along the
+// columns, two 16-bit elements per 32-bit column (one K = 16 step spans 8 columns).
+template <bool ACC>
+__device__ __forceinline__ void tc_mma_bf16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                               uint32_t idesc) {
+  if constexpr (ACC) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.eq.u32 p, 1, 1;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.eq.u32 p, 1, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc)
+        : "memory");
+  }
+}
+
 // Instruction descriptor for kind::f16 with bf16 A/B, fp32 accumulator, both operands
 // K-major: D format bits 4-5 = 1 (f32), A format bits 7-9 = 1 (bf16), B format bits
 // 10-12 = 1 (bf16), N >> 3 in bits 17-22, M >> 4 in bits 24-28.
