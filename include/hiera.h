@@ -136,8 +136,10 @@ HIERA_API hiera_status hiera_linear(const void* x, const void* w, const void* bi
  * hiera_block_pack() converts the weights once into `packed` (caller memory of
  * hiera_block_packed_bytes() bytes): LayerNorm's gamma is folded into the following
  * Linear (W' = W diag(gamma)) together with the column sums of W' and the constant
- * beta W^T + b, so that the forward pass applies LayerNorm inside the GEMM epilogue.
- * The raw weights may be freed after the pack has run.
+ * beta W^T + b, so that the forward pass applies LayerNorm inside the GEMM epilogue
+ * (bf16: from per-row (mean, M2) partials written by the kernel that produced the
+ * LayerNorm's input, merged in the epilogue; x itself is reduced once by a small
+ * statistics kernel). The raw weights may be freed after the pack has run.
  *
  * hiera_block_forward(): x [B, tokens, dim_in] -> y [B, tokens/q_stride, dim_out];
  * workspace of hiera_block_workspace_bytes() bytes holds the intermediates. x, y,
@@ -188,8 +190,9 @@ HIERA_API hiera_status hiera_block_forward(const hiera_block_desc* desc, const v
  * attention runs on the tensor-core kernel: T_q >= 128 and T_kv >= 128; f32 token-major
  * [B, tokens, 4*dim_out] holding q|k|v|proj in [0] and -1 in [1],[2]), [3] merged
  * attention output [B, tokens/q_stride, dim_out], [4] transition residual (or -1), [5] x
- * after the attention residual, [6] MLP hidden [B, tokens/q_stride, 4*dim_out]. Returns
- * HIERA_ERR_SHAPE on a bad desc. */
+ * after the attention residual, [6] MLP hidden [B, tokens/q_stride, 4*dim_out] (left
+ * unwritten when the bf16 MLP runs fused: dim_out 112 or 224 with HIERA_OPT_FUSED_MLP).
+ * Returns HIERA_ERR_SHAPE on a bad desc. */
 HIERA_API hiera_status hiera_block_workspace_layout(const hiera_block_desc* desc, long long offsets[7]);
 
 /* --------------------------------------------------------------------------------
