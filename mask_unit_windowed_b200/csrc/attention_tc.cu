@@ -62,6 +62,26 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   tc_ld_32x32b_x32(taddr, r);
 }
 
+// max(a, b, c) in one instruction (three-input form of max.f32 on sm_100a); the scores
+// are finite or -inf.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Softmax weights p in [0, 1] to bf16x2 by truncation (the high half of each fp32, lo
+// first): one byte permute per pair. The rounding bias this leaves (every weight a
+// fraction of an ulp low, relative 2^-9..2^-8 on average) cancels in the output, because
+// the denominator is the sum of the same bf16 weights (the ones row of V^T), so the
+// normalised result carries only the zero-mean part of the error, of the same size as
+// round-to-nearest's.
+__device__ __forceinline__ uint32_t pack_bf16x2_trunc(float lo, float hi) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(d) : "r"(__float_as_uint(lo)), "r"(__float_as_uint(hi)));
+  return d;
+}
+
 __global__ void __launch_bounds__(320, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const AParams p) {
@@ -253,16 +273,21 @@ __global__ void __launch_bounds__(320, 1)
         for (int i = 0; i < KT; ++i)
           if (i >= kv_valid) sr[i] = __float_as_uint(-INFINITY);
       }
-      // row max with 8 independent chains
+      // row max: 8 independent chains over keys u, u+8, ..., u+120, two new keys per
+      // three-input max
+      static_assert(KT == 128, "max chains cover 16 keys each");
       float mx[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) mx[u] = __uint_as_float(sr[u]);
+      for (int u = 0; u < 8; ++u) {
+        mx[u] = fmax3(__uint_as_float(sr[u]), __uint_as_float(sr[8 + u]),
+                      __uint_as_float(sr[16 + u]));
 #pragma unroll
-      for (int i = 8; i < KT; i += 8)
-#pragma unroll
-        for (int u = 0; u < 8; ++u) mx[u] = fmaxf(mx[u], __uint_as_float(sr[i + u]));
-      const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        for (int k = 3; k < 15; k += 2)
+          mx[u] = fmax3(mx[u], __uint_as_float(sr[8 * k + u]), __uint_as_float(sr[8 * k + 8 + u]));
+        mx[u] = fmaxf(mx[u], __uint_as_float(sr[120 + u]));
+      }
+      const float mt = fmaxf(fmax3(mx[0], mx[1], mx[2]),
+                             fmax3(fmax3(mx[3], mx[4], mx[5]), mx[6], mx[7]));
       float alpha = 1.f;
       bool resc = false;
       if (mt > m_run + thr) {
@@ -284,7 +309,7 @@ __global__ void __launch_bounds__(320, 1)
         for (int u = 0; u < 32; ++u) {
           const float x0 = fmaf(__uint_as_float(sr[64 * h + 2 * u]), sl2, -ms);   // -inf -> 0
           const float x1 = fmaf(__uint_as_float(sr[64 * h + 2 * u + 1]), sl2, -ms);
-          pw[u] = pack_bf16x2_int(ex2_approx(x0), ex2_approx(x1));
+          pw[u] = pack_bf16x2_trunc(ex2_approx(x0), ex2_approx(x1));
         }
         tc_st_32x32b_x32(lane_base + p_col + (uint32_t)(32 * h), pw);
       }

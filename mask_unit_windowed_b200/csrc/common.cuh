@@ -222,16 +222,6 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
-// Two floats to bf16x2 with integer operations only (no conversion unit): round half away
-// from zero in magnitude on the bit pattern (add 0x8000, keep the high half), lo first.
-// -inf stays -inf; finite inputs far below the bf16 range are not expected.
-__device__ __forceinline__ uint32_t pack_bf16x2_int(float lo, float hi) {
-  const uint32_t a = __float_as_uint(lo) + 0x8000u, b = __float_as_uint(hi) + 0x8000u;
-  uint32_t d;
-  asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-
 // 2^x on the MUFU unit (approximate, flush-to-zero), for softmax weights.
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
