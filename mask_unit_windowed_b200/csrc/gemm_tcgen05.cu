@@ -25,7 +25,8 @@
 // half of its tile).
 // Transition pooling: a 4-D tensor map loads, for 32 pooled tokens n, the four rows
 // n + c*T/4 (c = 0..3) interleaved, so the four pooling candidates are adjacent TMEM
-// lanes and the max is two warp shuffles.
+// lanes, hence adjacent rows of the epilogue's staging buffer; the copy-out takes their
+// max on the packed bf16 values.
 #include <mutex>
 
 #include "common.cuh"
@@ -63,6 +64,16 @@ struct KParams {
 };
 
 constexpr int cmin(int a, int b) { return a < b ? a : b; }
+
+// element-wise max of two groups of 8 bf16 (finite values)
+__device__ __forceinline__ uint4 bf16x8_max(uint4 a, uint4 b) {
+  uint4 d;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(d.x) : "r"(a.x), "r"(b.x));
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(d.y) : "r"(a.y), "r"(b.y));
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(d.z) : "r"(a.z), "r"(b.z));
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(d.w) : "r"(a.w), "r"(b.w));
+  return d;
+}
 
 template <int BN>
 struct Cfg {
@@ -367,17 +378,10 @@ __global__ void __launch_bounds__(320, 1)
           if (EPI == EPI_GELU) x = gelu_fast(x);
           v[i] = x;
         }
-        // ---- finish the values of this chunk (pooling / residual)
-        if (EPI == EPI_QKV) {
-          static_assert(EPI != EPI_QKV || CH == 56, "q/k/v chunks are whole heads");
-          if (pool_this) {
-#pragma unroll
-            for (int i = 0; i < CH; ++i) {
-              v[i] = fmaxf(v[i], __shfl_xor_sync(0xffffffffu, v[i], 1));
-              v[i] = fmaxf(v[i], __shfl_xor_sync(0xffffffffu, v[i], 2));
-            }
-          }
-        } else if (EPI == EPI_STORE && has_res) {
+        // ---- finish the values of this chunk (residual; the q / residual pooling of a
+        // transition is taken on the packed values when they are copied out)
+        static_assert(EPI != EPI_QKV || CH == 56, "q/k/v chunks are whole heads");
+        if (EPI == EPI_STORE && has_res) {
 #pragma unroll
           for (int g = 0; g < CH / 8; ++g) {
             const uint4 rr = res[(c / 8 + g) < NV ? (c / 8 + g) : 0];
@@ -469,15 +473,39 @@ __global__ void __launch_bounds__(320, 1)
         __syncwarp();
         // ---- copy out: 8 lanes per row, 4 rows per instruction, whole row segments
         const unsigned long long my_dst = reinterpret_cast<unsigned long long>(dst_row);
+        if (POOLED && pool_this) {
+          // q / residual of a transition: staged rows 4o..4o+3 are the four pooling
+          // candidates of output row o (lanes 4o..4o+3, the first of them the writer). Their
+          // max is taken on the bf16 values; rounding to nearest is monotonic, so the max of
+          // the rounded values is the rounded max of the fp32 values.
 #pragma unroll
-        for (int it = 0; it < 8; ++it) {
-          const int row = it * 4 + (lane >> 3), ch = lane & 7;
-          const unsigned long long d = __shfl_sync(0xffffffffu, my_dst, row);
-          const int ok = __shfl_sync(0xffffffffu, valid ? 1 : 0, row);
-          if (ok && ch < nchunk) {
-            const uint4 val =
-                *reinterpret_cast<const uint4*>(stg + (row << 7) + ((ch ^ (row & 7)) << 4));
-            *reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(d) + ch * 8) = val;
+          for (int it = 0; it < 2; ++it) {
+            const int orow = it * 4 + (lane >> 3), ch = lane & 7;
+            const unsigned long long d = __shfl_sync(0xffffffffu, my_dst, 4 * orow);
+            const int ok = __shfl_sync(0xffffffffu, valid ? 1 : 0, 4 * orow);
+            if (ok && ch < nchunk) {
+              uint4 val = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+              for (int c4 = 0; c4 < 4; ++c4) {
+                const int row = 4 * orow + c4;
+                const uint4 o =
+                    *reinterpret_cast<const uint4*>(stg + (row << 7) + ((ch ^ (row & 7)) << 4));
+                val = c4 == 0 ? o : bf16x8_max(val, o);
+              }
+              *reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(d) + ch * 8) = val;
+            }
+          }
+        } else {
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            const int row = it * 4 + (lane >> 3), ch = lane & 7;
+            const unsigned long long d = __shfl_sync(0xffffffffu, my_dst, row);
+            const int ok = __shfl_sync(0xffffffffu, valid ? 1 : 0, row);
+            if (ok && ch < nchunk) {
+              const uint4 val =
+                  *reinterpret_cast<const uint4*>(stg + (row << 7) + ((ch ^ (row & 7)) << 4));
+              *reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(d) + ch * 8) = val;
+            }
           }
         }
         __syncwarp();
