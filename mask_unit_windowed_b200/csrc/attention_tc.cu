@@ -71,11 +71,11 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 }
 
 // Softmax weights p in [0, 1] to bf16x2 by truncation (the high half of each fp32, lo
-// first): one byte permute per pair. The rounding bias this leaves (every weight a
-// fraction of an ulp low, relative 2^-9..2^-8 on average) cancels in the output, because
-// the denominator is the sum of the same bf16 weights (the ones row of V^T), so the
-// normalised result carries only the zero-mean part of the error, of the same size as
-// round-to-nearest's.
+// first): one byte permute per pair. Truncation leaves every weight a fraction of an ulp
+// low. The denominator is the sum of the same bf16 weights (the ones row of V^T), so for
+// rows with many comparable weights that bias cancels, and the output error is round-to-
+// nearest's. For rows dominated by a few weights it is about twice that, near 2e-3
+// relative.
 __device__ __forceinline__ uint32_t pack_bf16x2_trunc(float lo, float hi) {
   uint32_t d;
   asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(d) : "r"(__float_as_uint(lo)), "r"(__float_as_uint(hi)));
