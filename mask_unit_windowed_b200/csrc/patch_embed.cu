@@ -8,10 +8,12 @@
 // its 128 output columns need (3-pixel halo, zero outside the image); each warp computes 16
 // output pixels x 112 channels over K = 196 (padded to 208) with A fragments gathered
 // straight from the staged input (the (ky, kx, c) ordering keeps every fragment pair in one
-// 4-byte word). The epilogue stages fp32 results per warp in shared memory; a lane per
-// (pixel, 56-channel half) adds bias and pos_embed[raster token], rounds once to bf16,
+// 4-byte word). The epilogue adds bias and pos_embed[raster token] (loaded before the MMA
+// loop) to the accumulator fragments, rounds once to bf16 and stages the rows per warp in
+// the input buffer, which the MMA no longer needs; a lane per (pixel, 56-channel half) then
 // stores the half row at its unrolled position (3 unroll levels) and, when asked, the
-// LayerNorm partial (mean, M2) of the half for block 0's norm1.
+// LayerNorm partial (mean, M2) of the half for block 0's norm1. 79 KB of shared memory
+// per CTA: two CTAs per SM overlap one's loads with the other's MMA.
 // fp32: the same computation in fp32 SIMT (weights fp32 [196][112] in shared memory, 56
 // accumulators per thread).
 #include "common.cuh"
@@ -106,9 +108,12 @@ __global__ void __launch_bounds__(256, 1) patch_embed_kernel(const float* __rest
 constexpr int KP = 208;                 // K padded to 13 k-steps of 16
 constexpr int WPITCH = 216;             // bf16 per weight row in smem (conflict-free fragments)
 constexpr int IN_PITCH = 516;           // pixels per staged input row
-constexpr int OPITCH = 116;             // fp32 per staged output pixel (29 x 16 B: odd)
+constexpr int SPITCH = 120;             // bf16 per staged output pixel (240 B: 16-byte rows)
 constexpr int MMA_ROWS = 4;             // output rows per CTA (weights loaded once)
-constexpr int MMA_SMEM = PATCH_CO * WPITCH * 2 + KSZ * IN_PITCH * CIN * 2 + 8 * 16 * OPITCH * 4;
+constexpr int IN_BYTES = KSZ * IN_PITCH * CIN * 2;
+constexpr int STG_BYTES = 8 * 16 * SPITCH * 2;  // 8 warps x 16 pixels, aliases the input rows
+constexpr int BUF_BYTES = IN_BYTES > STG_BYTES ? IN_BYTES : STG_BYTES;
+constexpr int MMA_SMEM = PATCH_CO * WPITCH * 2 + BUF_BYTES;  // 79 KB: two CTAs per SM
 
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1,
                                                uint32_t a2, uint32_t a3, uint32_t b0,
@@ -126,16 +131,15 @@ __device__ __forceinline__ int in_off(int k, int px) {
   return (ky * IN_PITCH + 4 * px + (rem >> 2)) * CIN + (rem & 3);
 }
 
-__global__ void __launch_bounds__(256, 1) patch_embed_mma_kernel(
+__global__ void __launch_bounds__(256, 2) patch_embed_mma_kernel(
     const bf16* __restrict__ img, const bf16* __restrict__ w16, const float* __restrict__ bias,
     const bf16* __restrict__ pos, bf16* __restrict__ out, float2* __restrict__ stats_out,
     int img_side) {
   griddep_wait();  // everything below reads or writes data of earlier kernels
   griddep_launch_dependents();
   extern __shared__ __align__(16) uint8_t smem_pe[];
-  bf16* sW = reinterpret_cast<bf16*>(smem_pe);                       // [112][WPITCH]
-  bf16* sIn = sW + PATCH_CO * WPITCH;                                // [7][IN_PITCH][4]
-  float* sOut = reinterpret_cast<float*>(sIn + KSZ * IN_PITCH * CIN);  // [8 warps][16][OPITCH]
+  bf16* sW = reinterpret_cast<bf16*>(smem_pe);  // [112][WPITCH]
+  bf16* sIn = sW + PATCH_CO * WPITCH;           // [7][IN_PITCH][4] during the MMA
   const int G = img_side / 4;
   const int M = G / 8;
   const int N = G * G;
@@ -143,17 +147,19 @@ __global__ void __launch_bounds__(256, 1) patch_embed_mma_kernel(
   const int ox0 = blockIdx.x * SEG;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t4 = lane & 3;
+  // after the MMA the input rows are dead: each warp stages its 16 pixels x 112 channels
+  // there, rounded to bf16 ([16][SPITCH])
+  bf16* so = sIn + warp * 16 * SPITCH;
 
   for (int i = tid; i < PATCH_CO * (KP / 8); i += 256) {
     const int co = i / (KP / 8), c8 = i - co * (KP / 8);
     *reinterpret_cast<uint4*>(sW + co * WPITCH + c8 * 8) =
         __ldg(reinterpret_cast<const uint4*>(w16 + co * KP) + c8);
   }
-  float* so = sOut + warp * 16 * OPITCH;
   for (int rr = 0; rr < MMA_ROWS; ++rr) {
     const int oy = blockIdx.y * MMA_ROWS + rr;
     if (oy >= G) break;
-    __syncthreads();  // previous row's readers are done with sIn
+    __syncthreads();  // the previous row's staged outputs have been copied out
     for (int i = tid; i < KSZ * XSPAN; i += 256) {
       const int ky = i / XSPAN, xi = i - ky * XSPAN;
       const int iy = 4 * oy - 3 + ky, ix = 4 * ox0 - 3 + xi;
@@ -161,6 +167,17 @@ __global__ void __launch_bounds__(256, 1) patch_embed_mma_kernel(
       if (iy >= 0 && iy < img_side && ix >= 0 && ix < img_side)
         v = __ldg(reinterpret_cast<const uint2*>(img + (((long long)b * img_side + iy) * img_side + ix) * CIN));
       *reinterpret_cast<uint2*>(sIn + (ky * IN_PITCH + xi) * CIN) = v;
+    }
+    // pos_embed of this lane's two pixels (rows g, g + 8 of the warp's 16) and 28 channels
+    // (8 nt + 2 t4, +1), in flight while the MMA runs
+    uint32_t pw[2][14];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int ox = ox0 + warp * 16 + g + 8 * h;
+      const bf16* pr = pos + (long long)(oy * G + (ox < G ? ox : 0)) * PATCH_CO + 2 * t4;
+#pragma unroll
+      for (int nt = 0; nt < 14; ++nt)
+        pw[h][nt] = __ldg(reinterpret_cast<const unsigned int*>(pr + nt * 8));
     }
     __syncthreads();
     const int px = warp * 16 + g;  // fragment rows g and g + 8
@@ -187,41 +204,31 @@ __global__ void __launch_bounds__(256, 1) patch_embed_mma_kernel(
         mma_bf16_16816(acc[nt], a0, a1, a2, a3, b0, b1);
       }
     }
-    // stage fp32 (+ bias) per warp: pixel rows g, g + 8; channels 8 nt + 2 t4, +1
+    __syncthreads();  // every warp is done reading the input rows
+    // (acc + bias) + pos_embed, rounded once to bf16, staged per pixel row
 #pragma unroll
     for (int nt = 0; nt < 14; ++nt) {
       const int co = nt * 8 + 2 * t4;
       const float b0 = __ldg(bias + co), b1 = __ldg(bias + co + 1);
-      *reinterpret_cast<float2*>(so + g * OPITCH + co) = make_float2(acc[nt][0] + b0, acc[nt][1] + b1);
-      *reinterpret_cast<float2*>(so + (g + 8) * OPITCH + co) =
-          make_float2(acc[nt][2] + b0, acc[nt][3] + b1);
+      *reinterpret_cast<uint32_t*>(so + g * SPITCH + co) =
+          pack_bf16x2((acc[nt][0] + b0) + bf16_lo(pw[0][nt]), (acc[nt][1] + b1) + bf16_hi(pw[0][nt]));
+      *reinterpret_cast<uint32_t*>(so + (g + 8) * SPITCH + co) =
+          pack_bf16x2((acc[nt][2] + b0) + bf16_lo(pw[1][nt]), (acc[nt][3] + b1) + bf16_hi(pw[1][nt]));
     }
     __syncwarp();
-    // lane = (pixel, half): + pos_embed, one rounding, unrolled store, LayerNorm partial
+    // lane = (pixel, half): the half row to its unrolled position, LayerNorm partial
     {
-      const int lp = lane >> 1, half = lane & 1;
+      const int lp = lane & 15, half = lane >> 4;
       const int ox = ox0 + warp * 16 + lp;
       if (ox < G) {
-        const int t = oy * G + ox;
         const int u = unrolled_of_spatial(oy, ox, 3, M);
-        const float* src = so + lp * OPITCH + half * 56;
-        const bf16* pr = pos + (long long)t * PATCH_CO + half * 56;
-        bf16* dst = out + ((long long)b * N + u) * PATCH_CO + half * 56;
+        const uint4* src = reinterpret_cast<const uint4*>(so + lp * SPITCH + half * 56);
+        uint4* dst = reinterpret_cast<uint4*>(out + ((long long)b * N + u) * PATCH_CO + half * 56);
         float vals[56];
 #pragma unroll
         for (int c8 = 0; c8 < 7; ++c8) {
-          const uint4 pv = __ldg(reinterpret_cast<const uint4*>(pr) + c8);
-          const float4 s0 = *reinterpret_cast<const float4*>(src + 8 * c8);
-          const float4 s1 = *reinterpret_cast<const float4*>(src + 8 * c8 + 4);
-          float v8[8] = {s0.x + bf16_lo(pv.x), s0.y + bf16_hi(pv.x), s0.z + bf16_lo(pv.y),
-                         s0.w + bf16_hi(pv.y), s1.x + bf16_lo(pv.z), s1.y + bf16_hi(pv.z),
-                         s1.z + bf16_lo(pv.w), s1.w + bf16_hi(pv.w)};
-          uint4 pk;
-          pk.x = pack_bf16x2(v8[0], v8[1]);
-          pk.y = pack_bf16x2(v8[2], v8[3]);
-          pk.z = pack_bf16x2(v8[4], v8[5]);
-          pk.w = pack_bf16x2(v8[6], v8[7]);
-          reinterpret_cast<uint4*>(dst)[c8] = pk;
+          const uint4 pk = src[c8];
+          dst[c8] = pk;
           vals[8 * c8 + 0] = bf16_lo(pk.x);
           vals[8 * c8 + 1] = bf16_hi(pk.x);
           vals[8 * c8 + 2] = bf16_lo(pk.y);
@@ -243,7 +250,6 @@ __global__ void __launch_bounds__(256, 1) patch_embed_mma_kernel(
         }
       }
     }
-    __syncwarp();
   }
 }
 
