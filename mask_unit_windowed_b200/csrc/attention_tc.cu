@@ -10,7 +10,7 @@
 //               tensor core works on one tile while the other tile's softmax runs.
 //   warps 2-5   softmax of tile A, warps 6-9 of tile B, one query row per thread (TMEM lane
 //               = row): row max, then the weights P = 2^(s log2(e)/sqrt(56) - m) on the
-//               MUFU unit, rounded to bf16 with integer operations (the conversion unit
+//               MUFU unit, cut to bf16 by a byte permute per pair (the conversion unit
 //               shares the MUFU pipe) and stored as bf16 pairs into TMEM next to S and O;
 //               the PV product reads its A operand (P) from there, so P never goes through
 //               shared memory. The running max is raised, and O rescaled in TMEM, only when
