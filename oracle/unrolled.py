@@ -28,9 +28,12 @@ Readings taken where the plan is silent:
 from __future__ import annotations
 
 import math
+import os
+from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
 from scipy.special import erf
+from threadpoolctl import threadpool_limits
 
 LN_EPS = 1e-6
 HEAD_DIM = 56
@@ -122,22 +125,49 @@ def softmax_rows(s):
 
 
 # --------------------------------------------------------------------------- attention
-def mask_unit_attention(xn, qkv_w, qkv_b, attn_proj_w, attn_proj_b, heads, q_stride,
-                        window_tokens, mask_unit_attn, head_dim=HEAD_DIM):
-    """MaskUnitAttention ("Architecture Summary", MaskUnitAttention).
+def attention_core(q, k, v, head_dim=HEAD_DIM, row_chunk=None):
+    """Scaled dot-product attention over the last two axes ("Architecture Summary",
+    MaskUnitAttention: scaled dot-product attention with scale head_dim^-1/2):
+    softmax_rows(q k^T / sqrt(head_dim)) v for q [..., Tq, hd], k and v [..., Tkv, hd].
+
+    row_chunk, if given, evaluates that many query rows at a time. Each query row's
+    softmax only involves its own scores, so this is the same definition; it bounds the
+    host memory of long global attention (16384 queries x 65536 keys at 2048^2)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    scale = 1.0 / math.sqrt(head_dim)
+    Tq = q.shape[-2]
+    if row_chunk is None or Tq <= row_chunk:
+        return softmax_rows((q @ k.swapaxes(-1, -2)) * scale) @ v
+    out = np.empty(q.shape[:-1] + (v.shape[-1],))
+    kt = k.swapaxes(-1, -2)
+
+    def rows(r0):
+        r1 = min(Tq, r0 + row_chunk)
+        out[..., r0:r1, :] = softmax_rows((q[..., r0:r1, :] @ kt) * scale) @ v
+
+    # the chunks are independent; numpy releases the GIL inside its kernels, so host
+    # threads evaluate several at once, each with a single-threaded BLAS (each chunk's
+    # arithmetic is unchanged)
+    with threadpool_limits(1, user_api="blas"), \
+            ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
+        list(ex.map(rows, range(0, Tq, row_chunk)))
+    return out
+
+
+def attention_heads(xn, qkv_w, qkv_b, heads, q_stride, window_tokens, mask_unit_attn,
+                    head_dim=HEAD_DIM, row_chunk=None):
+    """MaskUnitAttention up to the merged heads, before its output proj ("Architecture
+    Summary", MaskUnitAttention).
 
     qkv = Linear(dim_in, 3 dim_out) split per window; at q_stride > 1 the queries are
-    max-pooled over the q_stride axis; scaled dot-product attention with scale
-    head_dim^-1/2 inside each window; heads merged; proj = Linear(dim_out, dim_out).
-
-    window_tokens is the number of key tokens per mask-unit window at the block input;
-    with mask_unit_attn False there is one window holding every token (global).
-    Returns [B, N / q_stride, dim_out].
+    max-pooled over the q_stride axis; scaled dot-product attention inside each window;
+    heads merged. window_tokens is the number of key tokens per mask-unit window at the
+    block input; with mask_unit_attn False there is one window holding every token
+    (global). Returns [B, N / q_stride, heads * head_dim], token j*nW + w, channel
+    h*head_dim + e.
     """
     B, N, _ = xn.shape
-    d_out = attn_proj_w.shape[0]
-    if d_out != heads * head_dim:
-        raise ValueError("dim_out must equal heads * head_dim")
+    d_out = heads * head_dim
     nW = N // window_tokens if mask_unit_attn else 1
     T = N // nW
     qkv = linear(xn, qkv_w, qkv_b)                          # [B, N, 3 d_out]
@@ -146,21 +176,32 @@ def mask_unit_attention(xn, qkv_w, qkv_b, attn_proj_w, attn_proj_b, heads, q_str
     q, k, v = qkv[0], qkv[1], qkv[2]
     if q_stride > 1:
         q = q.reshape(B, heads, nW, q_stride, T // q_stride, head_dim).max(axis=3)
-    scores = (q @ k.swapaxes(-1, -2)) / math.sqrt(head_dim)
-    o = softmax_rows(scores) @ v                            # [B, h, nW, Tq, hd]
+    o = attention_core(q, k, v, head_dim, row_chunk)       # [B, h, nW, Tq, hd]
     Tq = o.shape[3]
-    o = o.transpose(0, 3, 2, 1, 4).reshape(B, Tq * nW, d_out)   # token j*nW + w
+    return o.transpose(0, 3, 2, 1, 4).reshape(B, Tq * nW, d_out)   # token j*nW + w
+
+
+def mask_unit_attention(xn, qkv_w, qkv_b, attn_proj_w, attn_proj_b, heads, q_stride,
+                        window_tokens, mask_unit_attn, head_dim=HEAD_DIM, row_chunk=None):
+    """MaskUnitAttention ("Architecture Summary", MaskUnitAttention): attention_heads
+    followed by proj = Linear(dim_out, dim_out). Returns [B, N / q_stride, dim_out]."""
+    d_out = attn_proj_w.shape[0]
+    if d_out != heads * head_dim:
+        raise ValueError("dim_out must equal heads * head_dim")
+    o = attention_heads(xn, qkv_w, qkv_b, heads, q_stride, window_tokens, mask_unit_attn,
+                        head_dim, row_chunk)
     return linear(o, attn_proj_w, attn_proj_b)
 
 
 # --------------------------------------------------------------------------- block
 def block_forward(x, p, heads, q_stride, window_tokens, mask_unit_attn, eps=LN_EPS,
-                  head_dim=HEAD_DIM):
+                  head_dim=HEAD_DIM, row_chunk=None):
     """HieraBlock (Sub-phase 4a item 7): norm1 -> [proj + max-pool if transition]
     -> attn + residual -> norm2 -> MLP + residual.
 
     `p` holds numpy arrays keyed norm1_w, norm1_b, qkv_w, qkv_b, [proj_w, proj_b],
     attn_proj_w, attn_proj_b, norm2_w, norm2_b, fc1_w, fc1_b, fc2_w, fc2_b.
+    row_chunk: see attention_core.
     """
     x = _f64(x)
     dim_in = x.shape[-1]
@@ -170,7 +211,7 @@ def block_forward(x, p, heads, q_stride, window_tokens, mask_unit_attn, eps=LN_E
         x = max_pool_tokens(linear(xn, p["proj_w"], p["proj_b"]), q_stride)
     x = x + mask_unit_attention(xn, p["qkv_w"], p["qkv_b"], p["attn_proj_w"],
                                 p["attn_proj_b"], heads, q_stride, window_tokens,
-                                mask_unit_attn, head_dim)
+                                mask_unit_attn, head_dim, row_chunk)
     x = x + mlp(layer_norm(x, p["norm2_w"], p["norm2_b"], eps), p["fc1_w"], p["fc1_b"],
                 p["fc2_w"], p["fc2_b"])
     return x
@@ -222,12 +263,12 @@ def stage_ends():
     return ends
 
 
-def backbone_forward(img_nhwc, params, mask_unit_attn_override=None):
+def backbone_forward(img_nhwc, params, mask_unit_attn_override=None, row_chunk=None):
     """HieraBackbone (Sub-phase 4a item 8): patch_embed + pos_embed + unroll + 24 blocks
     + reroll at the stage ends [1, 4, 20, 23]. Returns four NHWC features.
 
     mask_unit_attn_override, if given, is a list of 24 booleans replacing the
-    per-block flag (used for the lagged-flag variant)."""
+    per-block flag (used for the lagged-flag variant). row_chunk: see attention_core."""
     B, H, W, _ = img_nhwc.shape
     G = H // 4
     x = patch_embed(img_nhwc, params["patch_w"], params["patch_b"])
@@ -246,7 +287,7 @@ def backbone_forward(img_nhwc, params, mask_unit_attn_override=None):
         if mua and N % window_tokens:
             raise ValueError("tokens not divisible into mask units")
         x = block_forward(x, params["blocks"][i], cfg["heads"], cfg["q_stride"],
-                          window_tokens, mua)
+                          window_tokens, mua, row_chunk=row_chunk)
         if i in ends:
             Gs = G >> s
             feats.append(reroll(x, Gs, UNROLL_LEVELS - s))

@@ -367,3 +367,36 @@ def test_block_rows_matches_full_block(case):
     part = U.block_forward_rows(x, p, heads, qs, window, mua, rows, head_dim=4)
     for r, (b, n) in enumerate(rows):
         np.testing.assert_allclose(part[r], full[b, n], rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("row_chunk", [1, 7, 64, 99])
+def test_row_chunked_attention_equals_unchunked(row_chunk):
+    """The row-chunked evaluation used for the 2048^2 global stages is the same definition:
+    each query row's softmax involves only its own scores (ragged last chunk included)."""
+    rng = np.random.default_rng(16)
+    q = rng.standard_normal((2, 3, 1, 100, 8)) * 2
+    k = rng.standard_normal((2, 3, 1, 130, 8)) * 2
+    v = rng.standard_normal((2, 3, 1, 130, 8))
+    full = U.attention_core(q, k, v, 8)
+    part = U.attention_core(q, k, v, 8, row_chunk=row_chunk)
+    np.testing.assert_allclose(part, full, rtol=1e-12, atol=1e-14)   # summation order only
+
+
+def test_backbone_row_chunk_equals_plain():
+    p = syn.backbone_params(17, 64, dtype="f32", affine="random")
+    x = syn.image(17, 1, 64)
+    for a, b in zip(U.backbone_forward(x, p), U.backbone_forward(x, p, row_chunk=3)):
+        np.testing.assert_allclose(b, a, rtol=1e-12, atol=1e-13)
+
+
+def test_attention_heads_is_mask_unit_attention_before_proj():
+    """attention_heads (compared per unit against the GPU's attention output) composes with
+    the proj Linear into MaskUnitAttention."""
+    rng = np.random.default_rng(18)
+    xn = rng.standard_normal((2, 64, 8))
+    p = _tiny_block(19, 8, 8, False)
+    o = U.attention_heads(xn, p["qkv_w"], p["qkv_b"], 2, 4, 16, True, head_dim=4)
+    a = U.mask_unit_attention(xn, p["qkv_w"], p["qkv_b"], p["attn_proj_w"], p["attn_proj_b"],
+                              2, 4, 16, True, head_dim=4)
+    np.testing.assert_allclose(U.linear(o, p["attn_proj_w"], p["attn_proj_b"]), a,
+                               rtol=1e-13, atol=1e-14)
