@@ -2,18 +2,23 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-One step = one forward of the whole backbone (patch embedding + pos_embed + Unroll,
-24 blocks, Reroll of the four stage features) over one batch of 8 synthetic images per
-GPU, replayed from a CUDA graph of the library's launches. Inputs are resident in HBM
-when a timed step starts; L2 is flushed (256 MiB write) before every step and the step
-is timed with CUDA events on the launching stream; the timed value sums the K step
-windows and takes the max over ranks. Multi-GPU runs are independent replicas (one
-batch per rank, no collective on the data path): value = all images / max time.
+One forward = the whole backbone (patch embedding + pos_embed + Unroll, 24 blocks, Reroll
+of the four stage features) over one batch of 8 synthetic images per GPU, replayed from a
+CUDA graph of the library's launches. One step = R consecutive forwards (R chosen from the
+warm-up so that the K timed steps last about a second: enough clock samples under load).
+Inputs are resident in HBM when a timed step starts; L2 is flushed (256 MiB write) before
+every step, and inside a step each forward's working set (138 MB of weights plus its
+activations) exceeds the 126 MB L2. Steps are timed with CUDA events on the launching
+stream; the timed value sums the K step windows and takes the max over ranks. Multi-GPU
+runs are independent replicas (one batch per rank, no collective on the data path):
+value = all images / max time.
 
 Rank 0 prints one JSON line with the headline images/s, the roofline of the dominant
-kernel (per-launch CUDA events inside a separately captured graph of the same
-forward), the end-to-end number through the public API with host buffers, SM clocks
-sampled during the timed region, and the CPU oracle timed on a bounded sample.
+kernel (the launch shape with the largest share of the forward, timed with per-launch
+CUDA events inside a separately captured graph of the same forward) against the burst
+bf16 peak, the end-to-end number through the public API with host buffers, SM clocks
+sampled during the timed region, the batch-1 latency of the same forward, the 2048^2
+batch-1 throughput, and the CPU oracle timed on a bounded sample.
 
 --impl reference times the CPU oracle (fp64 numpy, formulation U) on the same metric:
 each step is one 512^2 image through the whole backbone; the number of steps is capped
@@ -60,14 +65,12 @@ def peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
-# DRAM bytes (read + write) per GEMM-class launch of this workload, averaged over the 91
-# tc_gemm / mlp_fused launches of the first forward, from one ncu capture of the current
-# kernels (dram__bytes_read.sum + dram__bytes_write.sum, cold caches). Must be re-captured,
-# or set to None, whenever those kernels change. The GEMM's transition (pooled) epilogue
-# changed after the last capture, so it is None; that capture's figure is reported beside
-# it, labelled as such.
-GEMM_DRAM_BYTES_PER_LAUNCH = None
-GEMM_DRAM_BYTES_LAST_CAPTURE = 21.61e6
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of a kernel shape,
+# from one ncu capture of that kernel alone (three launches of the shape, this workload);
+# the summaries under profiles/ give the commands. Keyed by (kernel kind, GFLOP per launch
+# rounded to 0.01). A shape missing here reports traffic null; an entry must be removed
+# whenever its kernel changes.
+DRAM_BYTES_PER_LAUNCH = {}
 
 
 def reroll_bytes(img: int, B: int):
@@ -116,9 +119,50 @@ def launch_flops(img: int, B: int, fused_mlp: bool = True):
 
 KIND_CLASS = {"patch_embed": "patch_embed", "unroll_reroll": "unroll_reroll",
               "gemm_qkv_lnfold": "gemm", "gemm_fc1_lnfold_gelu": "gemm",
-              "gemm_bias_residual": "gemm", "attention_tiled": "attention",
-              "attention_packed": "attention", "attention_tcgen05": "attention",
-              "mlp_fused": "gemm"}
+              "gemm_bias_residual": "gemm", "attention_window": "attention",
+              "attention_tcgen05": "attention", "mlp_fused": "gemm"}
+
+KIND_DESCRIPTION = {
+    "gemm_qkv_lnfold": "tcgen05 GEMM: norm1 folded, qkv (+ transition proj) with window scatter",
+    "gemm_fc1_lnfold_gelu": "tcgen05 GEMM: norm2 folded, fc1 + GELU",
+    "gemm_bias_residual": "tcgen05 GEMM: attention proj or fc2, + bias + residual",
+    "mlp_fused": "tcgen05 fused MLP (norm2, fc1, GELU, fc2, residual)",
+    "attention_tcgen05": "tcgen05 attention, 128-key tiles (global attention)",
+    "attention_window": "tcgen05 attention, several mask-unit windows per tile",
+}
+
+
+def shape_breakdown(per_launch, flops, tf_burst, tf_sust):
+    """Group launches by (kind, GFLOP per launch): the shapes a forward is made of."""
+    shapes = {}
+    for (n, ms), (c, fl) in zip(per_launch, flops):
+        key = (n, round(fl / 1e9, 2))
+        e = shapes.setdefault(key, {"kind": n, "class": c, "launches": 0, "ms": 0.0,
+                                    "gflop": 0.0})
+        e["launches"] += 1
+        e["ms"] += ms
+        e["gflop"] += fl / 1e9
+    for e in shapes.values():
+        e["tflops"] = e["gflop"] / e["ms"] if e["ms"] > 0 else 0.0
+        e["frac_of_bf16_burst"] = e["tflops"] / tf_burst
+        e["frac_of_bf16_sustained"] = e["tflops"] / tf_sust
+    return shapes
+
+
+def time_steps(graph, stream, flush, steps, replays):
+    """K steps of `replays` graph replays each, L2 flushed before every step; per-step ms."""
+    import torch
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    with torch.cuda.stream(stream):
+        for k in range(steps):
+            flush.fill_(k & 0xFF)
+            starts[k].record(stream)
+            for _ in range(replays):
+                graph.replay()
+            ends[k].record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in zip(starts, ends)]
 
 
 class ClockSampler:
@@ -227,6 +271,59 @@ def run_reference(args, rank: int):
     print(json.dumps(line), flush=True)
 
 
+def _weights_dev(params, dev):
+    import torch
+
+    def t(a):
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev, torch.bfloat16)
+
+    return {"patch_w": t(params["patch_w"]), "patch_b": t(params["patch_b"]),
+            "pos_embed": t(params["pos_embed"]),
+            "blocks": [{k: t(v) for k, v in blk.items()} for blk in params["blocks"]]}
+
+
+def _graph_of(fn, stream):
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def extra_forward_timing(hb, syn, dev, stream, flush, img, B, seed, reps):
+    """ms per forward of the backbone at (img, B), CUDA graph, L2 flushed before each
+    forward, median of `reps`; also returns the algorithmic GFLOP per forward."""
+    import torch
+    params = syn.backbone_params(seed, img, dtype="bf16")
+    desc = hb.BackboneDesc(B=B, img=img)
+    packed = hb.backbone_pack(desc, _weights_dev(params, dev))
+    del params
+    x = torch.from_numpy(syn.image(seed, B, img)).to(dev, torch.bfloat16)
+    feats = [torch.empty(sh, dtype=torch.bfloat16, device=dev) for sh in desc.feature_shapes()]
+    ws = torch.empty(hb.backbone_workspace_bytes(desc), dtype=torch.uint8, device=dev)
+
+    def fwd():
+        hb.backbone_forward(desc, packed, x, feats=feats, workspace=ws)
+
+    with torch.cuda.stream(stream):
+        fwd()
+    torch.cuda.synchronize()
+    if hb.device_status(stream) != 0:
+        raise RuntimeError("device status after the extra forward")
+    g = _graph_of(fwd, stream)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g.replay()
+    ms = sorted(time_steps(g, stream, flush, reps, 1))
+    if hb.device_status(stream) != 0:
+        raise RuntimeError("device status after the extra timing")
+    gflop = sum(fl for _, fl in launch_flops(img, B)) / 1e9
+    del g, packed, ws, feats, x
+    torch.cuda.synchronize()
+    return ms[len(ms) // 2], gflop
+
+
 def run_ours(args, rank: int, world: int, local_rank: int):
     import torch
     import torch.distributed as dist
@@ -244,16 +341,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     # ---- weights and inputs (synthetic, seeded; random-init Hiera-B+)
     params = syn.backbone_params(SEED, IMG, dtype="bf16")
-
-    def t(a):
-        return torch.from_numpy(np.ascontiguousarray(a)).to(dev, torch.bfloat16)
-
-    weights = {"patch_w": t(params["patch_w"]), "patch_b": t(params["patch_b"]),
-               "pos_embed": t(params["pos_embed"]),
-               "blocks": [{k: t(v) for k, v in blk.items()} for blk in params["blocks"]]}
     desc = hb.BackboneDesc(B=B, img=IMG)
-    packed = hb.backbone_pack(desc, weights)
-    del weights
+    packed = hb.backbone_pack(desc, _weights_dev(params, dev))
+    del params
     img_host = torch.from_numpy(syn.image(SEED + rank, B, IMG)).to(torch.bfloat16).pin_memory()
     img = img_host.to(dev)
     feats = [torch.empty(s, dtype=torch.bfloat16, device=dev) for s in desc.feature_shapes()]
@@ -272,10 +362,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         raise RuntimeError(f"device status after warm-up: {hb.status_string(st)}")
 
     # ---- CUDA graph of one forward (the library's launches only)
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        forward()
-    torch.cuda.synchronize()
+    graph = _graph_of(forward, stream)
 
     # ---- instrumented graph: an event before every launch (kernel breakdown / roofline)
     prof = hb.LaunchProfile(capacity=256, stream=stream)
@@ -286,37 +373,32 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     torch.cuda.synchronize()
     n_launches = prof.count
 
-    with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
-            graph.replay()
-    torch.cuda.synchronize()
+    # ---- warm-up steps (one forward each), which also size a step: R forwards such that
+    # the K timed steps last about a second
+    warm = time_steps(graph, stream, flush, max(args.warmup, 3), 1)
+    est_ms = statistics.median(warm)
+    replays = args.replays if args.replays > 0 else \
+        max(1, math.ceil(args.timed_seconds * 1e3 / (args.steps * est_ms)))
 
     # ---- timed region
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local_rank) as clocks:
-        with torch.cuda.stream(stream):
-            for k in range(args.steps):
-                flush.fill_(k & 0xFF)
-                starts[k].record(stream)
-                graph.replay()
-                ends[k].record(stream)
-        torch.cuda.synchronize()
+        step_ms = time_steps(graph, stream, flush, args.steps, replays)
     if world > 1:
         dist.barrier()
-    total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    total_ms = sum(step_ms)
     st = hb.device_status(stream)
     if st != 0:
         raise RuntimeError(f"device status after timing: {hb.status_string(st)}")
     total_ms = replicas.max_over_ranks(total_ms, dev)
-    images = B * args.steps * world
-    value = replicas.job_throughput(B * args.steps, world, total_ms)
+    images = B * replays * args.steps * world
+    value = replicas.job_throughput(B * replays * args.steps, world, total_ms)
     ms_per_step = total_ms / args.steps
+    ms_per_forward = ms_per_step / replays
 
-    # ---- per-kernel breakdown from the instrumented graph (same workload, L2 flushed)
+    # ---- per-launch breakdown from the instrumented graph (same workload, L2 flushed)
     reps = 5
     per_launch = None
     with torch.cuda.stream(stream):
@@ -329,22 +411,48 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                 [(n, a + ms) for (n, a), (_, ms) in zip(per_launch, d)]
     per_launch = [(n, ms / reps) for n, ms in per_launch]
     flops = launch_flops(IMG, B, fused_mlp=hb.get_option(hb.OPT_FUSED_MLP) == 1)
-    classes = {}
-    by_kernel = {}
-    if len(flops) == len(per_launch) and all(KIND_CLASS.get(n) == c for (n, _), (c, _) in
-                                             zip(per_launch, flops)):
-        for (n, ms), (c, fl) in zip(per_launch, flops):
-            for e in (classes.setdefault(c, {"launches": 0, "ms": 0.0, "gflop": 0.0}),
-                      by_kernel.setdefault(n, {"launches": 0, "ms": 0.0, "gflop": 0.0})):
-                e["launches"] += 1
-                e["ms"] += ms
-                e["gflop"] += fl / 1e9
-    else:
-        for n, ms in per_launch:
-            e = classes.setdefault(KIND_CLASS.get(n, n), {"launches": 0, "ms": 0.0, "gflop": 0.0})
+    if len(flops) != len(per_launch) or any(KIND_CLASS.get(n) != c for (n, _), (c, _) in
+                                            zip(per_launch, flops)):
+        raise RuntimeError("the launch sequence differs from the bench's work model")
+    classes, by_kernel = {}, {}
+    for (n, ms), (c, fl) in zip(per_launch, flops):
+        for e in (classes.setdefault(c, {"launches": 0, "ms": 0.0, "gflop": 0.0}),
+                  by_kernel.setdefault(n, {"launches": 0, "ms": 0.0, "gflop": 0.0})):
             e["launches"] += 1
             e["ms"] += ms
+            e["gflop"] += fl / 1e9
     step_ms_prof = sum(ms for _, ms in per_launch)
+    for e in list(classes.values()) + list(by_kernel.values()):
+        e["share"] = e["ms"] / step_ms_prof if step_ms_prof > 0 else None
+        e["tflops"] = e["gflop"] / e["ms"] if e["ms"] > 0 else 0.0
+        e["frac_of_bf16_burst"] = e["tflops"] / tf_burst
+        e["frac_of_bf16_sustained"] = e["tflops"] / tf_sust
+    shapes = shape_breakdown(per_launch, flops, tf_burst, tf_sust)
+    for e in shapes.values():
+        e["share"] = e["ms"] / step_ms_prof if step_ms_prof > 0 else None
+    # dominant kernel: the tensor-core launch shape with the largest share of the forward
+    dom_key = max((k for k, e in shapes.items() if e["class"] in ("gemm", "attention")),
+                  key=lambda k: shapes[k]["ms"])
+    dom = shapes[dom_key]
+    traffic = DRAM_BYTES_PER_LAUNCH.get(dom_key)
+    attn_gemm_gflop = sum(fl for c, fl in flops if c in ("gemm", "attention")) / 1e9
+    roofline = {"bound": "tensor", "achieved": dom["tflops"], "peak": tf_burst,
+                "unit": "TFLOP/s", "frac": dom["tflops"] / tf_burst, "traffic": traffic,
+                "kernel": dom_key[0], "kernel_description": KIND_DESCRIPTION.get(dom_key[0]),
+                "gflop_per_launch": dom_key[1], "launches_per_forward": dom["launches"],
+                "ms_per_launch": dom["ms"] / dom["launches"],
+                "share_of_forward": dom["share"],
+                "peak_kind": f"bf16 dense burst ({peak_src}); the kernels run inside a "
+                             "ms-scale forward, not a seconds-long loop",
+                "peak_sustained": tf_sust, "frac_of_sustained": dom["tflops"] / tf_sust,
+                "traffic_unit": "bytes per launch (dram__bytes_read.sum + "
+                                "dram__bytes_write.sum, one ncu capture of this kernel)",
+                "timing": "per-launch CUDA events in an instrumented graph of the same "
+                          "forward, mean of 5 replays, L2 flushed before each"}
+    shape_list = sorted(({"kernel": k[0], "gflop_per_launch": k[1], **{kk: vv for kk, vv in
+                          e.items() if kk not in ("kind",)}} for k, e in shapes.items()),
+                        key=lambda e: -e["ms"])
+
     rr_ms = [ms for n, ms in per_launch if n == "unroll_reroll"]
     rr_bytes = reroll_bytes(IMG, B)
     reroll_hbm = None
@@ -352,40 +460,14 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         gbs = sum(rr_bytes) / (sum(rr_ms) * 1e-3) / 1e9
         big = max(range(len(rr_bytes)), key=lambda i: rr_bytes[i])
         gbs_big = rr_bytes[big] / (rr_ms[big] * 1e-3) / 1e9
-        reroll_hbm = {"bytes_per_step": sum(rr_bytes), "ms": sum(rr_ms), "gbs": gbs,
+        reroll_hbm = {"bytes_per_forward": sum(rr_bytes), "ms": sum(rr_ms), "gbs": gbs,
                       "frac_of_hbm": gbs / hbm_gbs, "largest_launch_bytes": rr_bytes[big],
                       "largest_launch_gbs": gbs_big, "largest_launch_frac": gbs_big / hbm_gbs,
                       "peak_gbs": hbm_gbs, "note": "event-timed inside the instrumented "
                       "graph (includes the per-launch event gap)"}
-    for e in list(classes.values()) + list(by_kernel.values()):
-        e["share"] = e["ms"] / step_ms_prof if step_ms_prof > 0 else None
-        e["tflops"] = e["gflop"] / e["ms"] if e["ms"] > 0 else 0.0
-        e["frac_of_bf16_sustained"] = e["tflops"] / tf_sust
-    dominant = max((c for c in classes if c in ("gemm", "attention")),
-                   key=lambda c: classes[c]["ms"])
-    dom = classes[dominant]
-    attn_gemm_gflop = sum(fl for c, fl in flops if c in ("gemm", "attention")) / 1e9
-    roofline = {"bound": "tensor", "kernel": {"gemm": "tcgen05 GEMM + fused MLP (all Linear layers)",
-                                              "attention": "mask-unit / global attention"}
-                [dominant],
-                "achieved": dom["tflops"], "peak": tf_sust, "unit": "TFLOP/s",
-                "frac": dom["tflops"] / tf_sust,
-                "traffic": GEMM_DRAM_BYTES_PER_LAUNCH if dominant == "gemm" else None,
-                "traffic_note": "dram__bytes_read.sum + dram__bytes_write.sum per GEMM-class "
-                                "launch, one ncu capture, cold caches; algorithmic bytes "
-                                "40.9e6 per launch; null: the transition GEMMs' epilogue "
-                                "changed after the capture (shared-memory work only, same "
-                                "global loads and stores)",
-                "traffic_last_capture": (GEMM_DRAM_BYTES_LAST_CAPTURE if dominant == "gemm"
-                                         else None),
-                "peak_kind": f"bf16 dense sustained ({peak_src})",
-                "launches_per_step": dom["launches"],
-                "gflop_per_launch": dom["gflop"] / max(dom["launches"], 1),
-                "ms_per_launch": dom["ms"] / max(dom["launches"], 1)}
 
     # ---- Unroll / Reroll alone: a stage-0 tensor of 32 images (235 MB, both directions 470 MB,
     # far beyond the 126 MB L2), 10 launches back to back between two events
-    rr_alone = None
     G0 = IMG // 4
     xs = torch.randn(32, G0 * G0, 112, device=dev).to(torch.bfloat16)
     ys = torch.empty_like(xs)
@@ -437,14 +519,32 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         e2e = {"value": replicas.job_throughput(B * n, world, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": img_host.numel() * img_host.element_size(),
                "d2h_bytes_per_step": sum(f.numel() * f.element_size() for f in host_feats),
-               "steps": n,
+               "steps": n, "images_per_step": B,
                "api": "binding.BackbonePipeline: pinned H2D image, hiera_backbone_forward, "
                       "pinned D2H of the four features per step, copies overlapping "
                       "neighbouring steps",
                "l2": "not flushed; per-step working set > L2"}
         del pipe
 
-    del graph, pgraph
+    del graph, pgraph, packed, ws, feats
+    torch.cuda.synchronize()
+
+    # ---- other workloads of the same forward (one GPU each, not part of the headline):
+    # batch-1 latency at 512^2 and batch-1 throughput at 2048^2
+    extra = {}
+    if not args.no_extra:
+        ms1, gf1 = extra_forward_timing(hb, syn, dev, stream, flush, IMG, 1, SEED, 30)
+        extra["latency_512_b1"] = {"ms_per_forward": ms1, "images_per_s": 1e3 / ms1,
+                                   "tflops": gf1 / ms1, "gflop_per_forward": gf1,
+                                   "timing": "CUDA graph, L2 flushed before each forward, "
+                                             "median of 30"}
+        ms5, gf5 = extra_forward_timing(hb, syn, dev, stream, flush, 2048, 1, 4, 10)
+        extra["throughput_2048_b1"] = {"ms_per_forward": ms5, "images_per_s": 1e3 / ms5,
+                                       "tflops": gf5 / ms5, "gflop_per_forward": gf5,
+                                       "frac_of_bf16_burst": gf5 / ms5 / tf_burst,
+                                       "timing": "CUDA graph, L2 flushed before each "
+                                                 "forward, median of 10"}
+
     if rank != 0:
         return
     cpu = None
@@ -456,27 +556,35 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     gflop_per_image = sum(fl for _, fl in flops) / B / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": f"Hiera-B+ backbone forward, {IMG}x{IMG}x4 bf16 images, "
                                f"batch {B} per GPU (random-init weights, seed {SEED})",
                    "img": IMG, "batch_per_gpu": B, "global_batch": B * world,
+                   "forwards_per_step": replays, "images_per_step_per_gpu": B * replays,
                    "parallelism": f"replicas x{world} (no data-path collective)",
-                   "l2": "flushed before every step (256 MiB write)",
+                   "l2": "flushed before every step (256 MiB write); within a step each "
+                         "forward's working set (138 MB of weights + activations) exceeds L2",
                    "timing": "CUDA-graph replay of the library launches, per-step CUDA events",
                    "mlp": args.mlp, "pdl": args.pdl},
+        "ms_per_forward": ms_per_forward,
+        "timed_seconds": total_ms / 1e3,
         "tflops": gflop_per_image * images / (total_ms * 1e-3) * 1e-3,
-        "attn_gemm_frac_of_bf16_peak": attn_gemm_gflop / (ms_per_step * 1e-3) / 1e3 / tf_sust,
+        "attn_gemm_frac_of_bf16_peak": attn_gemm_gflop / (ms_per_forward * 1e-3) / 1e3 / tf_burst,
+        "attn_gemm_frac_of_bf16_sustained": attn_gemm_gflop / (ms_per_forward * 1e-3) / 1e3
+        / tf_sust,
         "gflop_per_image": gflop_per_image,
         "roofline": roofline,
         "kernels": classes,
         "by_kernel": by_kernel,
+        "by_shape": shape_list,
         "cpu_baseline": cpu,
         "e2e": e2e,
         "unroll_reroll_hbm": reroll_hbm,
+        "extra_workloads": extra,
         "clocks": clocks.record(),
-        "gpu_launches": n_launches * args.steps,
-        "launches_per_step": n_launches,
+        "gpu_launches": n_launches * replays * args.steps,
+        "launches_per_forward": n_launches,
     }
     print(json.dumps(line), flush=True)
 
@@ -484,8 +592,14 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--replays", type=int, default=0,
+                    help="forwards per timed step (0: chosen so the timed region lasts "
+                         "--timed-seconds)")
+    ap.add_argument("--timed-seconds", type=float, default=1.2)
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the batch-1 latency and 2048^2 throughput measurements")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--batch", type=int, default=BATCH)
     ap.add_argument("--e2e-steps", type=int, default=30)

@@ -186,14 +186,37 @@ HIERA_API hiera_status hiera_block_forward(const hiera_block_desc* desc, const v
 
 /* Byte offsets of the block's intermediates inside its workspace, for inspection:
  * [0] q, [1] k, [2] v (head-major: bf16 [B][windows][heads][T][64] with channels 56..63
- * zero, except that v is stored transposed, [B][windows][heads][64][T], when the block's
- * attention runs on the tensor-core kernel: T_q >= 128 and T_kv >= 128; f32 token-major
- * [B, tokens, 4*dim_out] holding q|k|v|proj in [0] and -1 in [1],[2]), [3] merged
+ * zero, except v's channel 56, which holds 1.0 (the layout hiera_attention() takes); f32
+ * token-major [B, tokens, 4*dim_out] holding q|k|v|proj in [0] and -1 in [1],[2]), [3] merged
  * attention output [B, tokens/q_stride, dim_out], [4] transition residual (or -1), [5] x
  * after the attention residual, [6] MLP hidden [B, tokens/q_stride, 4*dim_out] (left
  * unwritten when the bf16 MLP runs fused: dim_out 112 or 224 with HIERA_OPT_FUSED_MLP).
  * Returns HIERA_ERR_SHAPE on a bad desc. */
 HIERA_API hiera_status hiera_block_workspace_layout(const hiera_block_desc* desc, long long offsets[7]);
+
+/* --------------------------------------------------------------------------------
+ * Attention core of MaskUnitAttention ("Architecture Summary", MaskUnitAttention:
+ * scaled dot-product attention per mask-unit window, or over all tokens, then the heads
+ * merged before proj), on the head-major q/k/v the block's qkv projection writes.
+ *
+ *   o[b, j*windows + w, h*56 + e] = sum_t softmax_t(q_j . k_t / sqrt(56)) v_t[e]
+ *
+ * for every image b, window w, head h and query j < Tq, over the window's Tkv keys t.
+ * All tensors are bf16:
+ *   q  [B][windows][heads][Tq][64]   channels 56..63 zero (head_dim 56, padded);
+ *   k  [B][windows][heads][Tkv][64]  channels 56..63 zero;
+ *   v  [B][windows][heads][Tkv][64]  channel 56 = 1.0 and 57..63 zero (the kernels sum the
+ *                                    softmax denominator through that channel);
+ *   o  [B, Tq*windows, heads*56]     written; token j*windows + w, channel h*56 + e.
+ * Queries are already max-pooled where the block pools them (Tq = Tkv / q_stride). The
+ * softmax is max-subtracted in fp32 with fp32 accumulation; the weights enter the P V
+ * product as bf16. Windows of 4..64 keys (a power of two) with Tq = Tkv or Tkv / 4 run
+ * several windows per tensor-core tile; every other size runs the 128-key-tile kernel.
+ * Any B, windows, heads >= 1 with B*windows*heads*max(Tq, Tkv) <= 2^31.
+ * -------------------------------------------------------------------------------- */
+HIERA_API hiera_status hiera_attention(const void* q, const void* k, const void* v, void* o,
+                                       int B, int windows, int heads, int Tq, int Tkv,
+                                       hiera_stream_t stream);
 
 /* --------------------------------------------------------------------------------
  * Allocation-free variant of hiera_block_forward (no counterpart on the pages: it exists
@@ -219,6 +242,9 @@ HIERA_API hiera_status hiera_block_workspace_layout(const hiera_block_desc* desc
  * byte a call reads was written earlier in the same call.
  * -------------------------------------------------------------------------------- */
 #define HIERA_STATIC_SCRATCH_BYTES ((size_t)32 << 20)
+/* The size of that array as compiled into the library (HIERA_STATIC_SCRATCH_BYTES), for
+ * callers that load the library without this header. */
+HIERA_API size_t hiera_static_scratch_bytes(void);
 HIERA_API hiera_status hiera_block_forward_noalloc(const hiera_block_desc* desc,
                                                    const void* packed, const void* x, void* y,
                                                    hiera_stream_t stream);

@@ -101,6 +101,8 @@ def lib() -> ctypes.CDLL:
             "hiera_debug_timeout_probe": ([I, P], I),
             "hiera_debug_gelu": ([P, P, I, P], I),
             "hiera_block_forward_noalloc": ([ctypes.POINTER(BlockDescC), P, P, P, P], I),
+            "hiera_static_scratch_bytes": ([], S),
+            "hiera_attention": ([P, P, P, P, I, I, I, I, I, P], I),
             "hiera_profile_begin": ([ctypes.POINTER(ctypes.c_void_p), I,
                                      ctypes.POINTER(ctypes.c_int)], I),
             "hiera_profile_end": ([P], I),
@@ -144,30 +146,66 @@ def _need(t: torch.Tensor, name: str):
         raise ValueError(f"{name} must be a contiguous CUDA tensor")
 
 
+def _expect(t: torch.Tensor, name: str, shape, dtype, device=None):
+    """Reject a tensor whose shape, dtype or device differs from what the C call will
+    assume: the library sizes every copy from the descriptor alone, so a mismatched
+    tensor would be read or written past its end."""
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    _need(t, name)
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def _expect_bytes(t: torch.Tensor, name: str, nbytes: int, device=None):
+    have = t.numel() * t.element_size()
+    if have < nbytes:
+        raise ValueError(f"{name} holds {have} bytes, needs {nbytes}")
+    _need(t, name)
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
 # ----------------------------------------------------------------------------- Unroll / Reroll
 def unroll(x: torch.Tensor, G: int, levels: int, out=None, stream=None) -> torch.Tensor:
-    _need(x, "x")
     B, N, C = x.shape
+    if N != G * G:
+        raise ValueError(f"x has shape {tuple(x.shape)}: {N} tokens, expected G*G = {G * G}")
+    _need(x, "x")
     out = torch.empty_like(x) if out is None else out
+    _expect_bytes(out, "out", x.numel() * x.element_size(), x.device)
     _check(lib().hiera_unroll(_ptr(x), _ptr(out), B, G, C, levels, _dt(x), _stream(stream)),
            "hiera_unroll")
     return out
 
 
 def reroll(x: torch.Tensor, G: int, levels: int, out=None, stream=None) -> torch.Tensor:
-    _need(x, "x")
     B, N, C = x.shape
+    if N != G * G:
+        raise ValueError(f"x has shape {tuple(x.shape)}: {N} tokens, expected G*G = {G * G}")
+    _need(x, "x")
     out = torch.empty((B, G, G, C), dtype=x.dtype, device=x.device) if out is None else out
+    _expect_bytes(out, "out", x.numel() * x.element_size(), x.device)
     _check(lib().hiera_reroll(_ptr(x), _ptr(out), B, G, C, levels, _dt(x), _stream(stream)),
            "hiera_reroll")
     return out
 
 
 def linear(x, w, bias=None, residual=None, out=None, stream=None) -> torch.Tensor:
-    _need(x, "x")
     M, K = x.shape
     N = w.shape[0]
+    if tuple(w.shape) != (N, K):
+        raise ValueError(f"w has shape {tuple(w.shape)}, expected {(N, K)}")
+    _need(x, "x")
+    _expect(w, "w", (N, K), x.dtype, x.device)
+    if bias is not None:
+        _expect(bias, "bias", (N,), x.dtype, x.device)
+    if residual is not None:
+        _expect(residual, "residual", (M, N), x.dtype, x.device)
     out = torch.empty((M, N), dtype=x.dtype, device=x.device) if out is None else out
+    _expect(out, "out", (M, N), x.dtype, x.device)
     _check(lib().hiera_linear(_ptr(x), _ptr(w), _ptr(bias), _ptr(residual), _ptr(out), M, N, K,
                               _dt(x), _stream(stream)), "hiera_linear")
     return out
@@ -243,35 +281,79 @@ def block_pack(desc: BlockDesc, weights: dict, device="cuda", stream=None) -> to
     return packed
 
 
+def _check_block_args(desc: BlockDesc, packed, x, out):
+    """Shapes, dtypes and devices of a block call against its descriptor (before any
+    launch): every shape first, then where the tensors live."""
+    out_shape = (desc.B, desc.out_tokens, desc.dim_out)
+    for t, name, shape in ((x, "x", (desc.B, desc.tokens, desc.dim_in)), (out, "out", out_shape)):
+        if t is not None and (tuple(t.shape) != shape or t.dtype != desc.dtype):
+            raise ValueError(f"{name} is {tuple(t.shape)} {t.dtype}, expected {shape} "
+                             f"{desc.dtype}: shape or dtype mismatch")
+    _expect(x, "x", (desc.B, desc.tokens, desc.dim_in), desc.dtype)
+    _expect_bytes(packed, "packed", block_packed_bytes(desc), x.device)
+    if out is not None:
+        _expect(out, "out", out_shape, desc.dtype, x.device)
+
+
 def block_forward(desc: BlockDesc, packed: torch.Tensor, x: torch.Tensor, out=None,
                   workspace=None, stream=None) -> torch.Tensor:
-    _need(x, "x")
+    _check_block_args(desc, packed, x, out)
     d = desc.c()
     if out is None:
         out = torch.empty((desc.B, desc.out_tokens, desc.dim_out), dtype=x.dtype,
                           device=x.device)
     if workspace is None:
         workspace = torch.empty(block_workspace_bytes(desc), dtype=torch.uint8, device=x.device)
+    _expect_bytes(workspace, "workspace", block_workspace_bytes(desc), x.device)
     _check(lib().hiera_block_forward(ctypes.byref(d), _ptr(packed), _ptr(x), _ptr(out),
-                                     _ptr(workspace), workspace.numel(), _stream(stream)),
+                                     _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                     _stream(stream)),
            "hiera_block_forward")
     return out
 
 
-STATIC_SCRATCH_BYTES = 32 << 20
+def static_scratch_bytes() -> int:
+    """Size of the library's static scratch array (hiera_static_scratch_bytes)."""
+    return int(lib().hiera_static_scratch_bytes())
 
 
 def block_forward_noalloc(desc: BlockDesc, packed: torch.Tensor, x: torch.Tensor, out=None,
                           stream=None) -> torch.Tensor:
     """hiera_block_forward_noalloc: the block forward with the library's static scratch
     (for callers that cannot allocate a workspace); `out` may be preallocated."""
-    _need(x, "x")
+    _check_block_args(desc, packed, x, out)
     d = desc.c()
     if out is None:
         out = torch.empty((desc.B, desc.out_tokens, desc.dim_out), dtype=x.dtype,
                           device=x.device)
     _check(lib().hiera_block_forward_noalloc(ctypes.byref(d), _ptr(packed), _ptr(x), _ptr(out),
                                              _stream(stream)), "hiera_block_forward_noalloc")
+    return out
+
+
+# ----------------------------------------------------------------------------- attention core
+def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out=None,
+              stream=None) -> torch.Tensor:
+    """hiera_attention on head-major q [B, windows, heads, Tq, 64], k and v
+    [B, windows, heads, Tkv, 64] (bf16; q/k channels 56..63 zero, v channel 56 = 1 and
+    57..63 zero). Returns the merged [B, Tq * windows, heads * 56] output."""
+    if q.dim() != 5 or k.dim() != 5:
+        raise ValueError("q, k, v must be [B, windows, heads, T, 64]")
+    B, nW, heads, Tq, _ = q.shape
+    Tkv = k.shape[3]
+    for t, name, T in ((q, "q", Tq), (k, "k", Tkv), (v, "v", Tkv)):
+        if tuple(t.shape) != (B, nW, heads, T, 64) or t.dtype != torch.bfloat16:
+            raise ValueError(f"{name} is {tuple(t.shape)} {t.dtype}: shape or dtype mismatch "
+                             f"(expected {(B, nW, heads, T, 64)} bf16)")
+    _expect(q, "q", (B, nW, heads, Tq, 64), torch.bfloat16)
+    _expect(k, "k", (B, nW, heads, Tkv, 64), torch.bfloat16, q.device)
+    _expect(v, "v", (B, nW, heads, Tkv, 64), torch.bfloat16, q.device)
+    shape = (B, Tq * nW, heads * 56)
+    if out is None:
+        out = torch.empty(shape, dtype=torch.bfloat16, device=q.device)
+    _expect(out, "out", shape, torch.bfloat16, q.device)
+    _check(lib().hiera_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, nW, heads, Tq, Tkv,
+                                 _stream(stream)), "hiera_attention")
     return out
 
 
@@ -288,7 +370,11 @@ def patch_embed(img, packed_patch, pos_embed, out=None, stream=None) -> torch.Te
     _need(img, "img")
     B, H, W, _ = img.shape
     G = H // 4
+    _expect(img, "img", (B, H, H, 4), img.dtype)
+    _expect_bytes(packed_patch, "packed_patch", PATCH_PACKED_BYTES, img.device)
+    _expect(pos_embed, "pos_embed", (G * G, 112), img.dtype, img.device)
     out = torch.empty((B, G * G, 112), dtype=img.dtype, device=img.device) if out is None else out
+    _expect(out, "out", (B, G * G, 112), img.dtype, img.device)
     _check(lib().hiera_patch_embed(_ptr(img), _ptr(packed_patch), _ptr(pos_embed), _ptr(out), B,
                                    H, _dt(img), _stream(stream)), "hiera_patch_embed")
     return out
@@ -344,17 +430,24 @@ def backbone_pack(desc: BackboneDesc, weights: dict, device="cuda", stream=None)
 
 def backbone_forward(desc: BackboneDesc, packed, img, feats=None, workspace=None,
                      stream=None):
-    _need(img, "img")
+    _expect(img, "img", (desc.B, desc.img, desc.img, 4), desc.dtype)
+    _expect_bytes(packed, "packed", backbone_packed_bytes(desc), img.device)
     d = desc.c()
     if feats is None:
         feats = [torch.empty(s, dtype=img.dtype, device=img.device)
                  for s in desc.feature_shapes()]
+    if len(feats) != 4:
+        raise ValueError("feats must hold four tensors")
+    for i, (f, shp) in enumerate(zip(feats, desc.feature_shapes())):
+        _expect(f, f"feats[{i}]", shp, desc.dtype, img.device)
     if workspace is None:
         workspace = torch.empty(backbone_workspace_bytes(desc), dtype=torch.uint8,
                                 device=img.device)
+    _expect_bytes(workspace, "workspace", backbone_workspace_bytes(desc), img.device)
     fp = (ctypes.c_void_p * 4)(*[f.data_ptr() for f in feats])
     _check(lib().hiera_backbone_forward(ctypes.byref(d), _ptr(packed), _ptr(img), fp,
-                                        _ptr(workspace), workspace.numel(), _stream(stream)),
+                                        _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                        _stream(stream)),
            "hiera_backbone_forward")
     return feats
 

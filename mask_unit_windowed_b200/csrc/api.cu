@@ -6,6 +6,8 @@
 
 #include <algorithm>
 #include <mutex>
+#include <set>
+#include <utility>
 
 #include "common.cuh"
 #include "internal.h"
@@ -256,8 +258,6 @@ hiera_status forward_bf16(const Geom& g, const uint8_t* packed, const void* x, v
   a.Tq = g.Tq;
   a.Tkv = g.Tkv;
   a.pooled = g.qs == 4;
-  const bool tc_attn = attention_tc_supported(g.Tq, g.Tkv);
-  a.vt = tc_attn ? 1 : 0;
   HIERA_TRY(launch_tc_gemm(EPI_QKV, a, st));
   // (a7, a8) attention core, heads merged
   AttnArgs at{};
@@ -271,7 +271,7 @@ hiera_status forward_bf16(const Geom& g, const uint8_t* packed, const void* x, v
   at.Tq = g.Tq;
   at.Tkv = g.Tkv;
   at.d_out = g.d_out;
-  HIERA_TRY(tc_attn ? launch_attention_tc(at, st) : launch_attention_bf16(at, st));
+  HIERA_TRY(launch_attention(at, st));
   // (a9) attention proj + residual
   TcGemmArgs pj{};
   pj.M = (int)qrows;
@@ -565,6 +565,20 @@ int g_num_sms() {
 
 unsigned int* g_status_ptr() { return dev_info().status; }
 
+bool ensure_smem_attr(const void* kern, int bytes) {
+  static std::mutex mu;
+  static std::set<std::pair<const void*, int>> done;  // (kernel, device)
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  std::lock_guard<std::mutex> lk(mu);
+  if (done.count({kern, dev})) return true;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+      cudaSuccess)
+    return false;
+  done.insert({kern, dev});
+  return true;
+}
+
 namespace {
 // Under stream capture a plain cudaEventRecord only orders the capture; the external
 // flag makes it an event-record node that re-records on every graph replay.
@@ -759,6 +773,8 @@ hiera_status hiera_block_forward(const hiera_block_desc* desc, const void* packe
                 : forward_f32(g, (const uint8_t*)packed, x, y, (uint8_t*)workspace, st);
 }
 
+size_t hiera_static_scratch_bytes(void) { return HIERA_STATIC_SCRATCH_BYTES; }
+
 hiera_status hiera_block_forward_noalloc(const hiera_block_desc* desc, const void* packed,
                                          const void* x, void* y, hiera_stream_t stream) {
   Geom g;
@@ -772,6 +788,29 @@ hiera_status hiera_block_forward_noalloc(const hiera_block_desc* desc, const voi
   const cudaStream_t st = (cudaStream_t)stream;
   return g.bf16 ? forward_bf16(g, (const uint8_t*)packed, x, y, (uint8_t*)scratch, st)
                 : forward_f32(g, (const uint8_t*)packed, x, y, (uint8_t*)scratch, st);
+}
+
+hiera_status hiera_attention(const void* q, const void* k, const void* v, void* o, int B,
+                             int windows, int heads, int Tq, int Tkv, hiera_stream_t stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return HIERA_ERR_INVALID_ARG;
+  if (B < 1 || windows < 1 || heads < 1 || Tq < 1 || Tkv < 1) return HIERA_ERR_INVALID_ARG;
+  if ((long long)B * windows * heads * std::max(Tq, Tkv) > (1ll << 31)) return HIERA_ERR_SHAPE;
+  if ((long long)heads * 56 > (1 << 20)) return HIERA_ERR_SHAPE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return HIERA_ERR_ALIGNMENT;
+  HIERA_TRY(check_device());
+  AttnArgs at{};
+  at.q = q;
+  at.k = k;
+  at.v = v;
+  at.o = o;
+  at.B = B;
+  at.nW = windows;
+  at.heads = heads;
+  at.Tq = Tq;
+  at.Tkv = Tkv;
+  at.d_out = heads * 56;
+  return launch_attention(at, (cudaStream_t)stream);
 }
 
 hiera_status hiera_patch_pack(const void* patch_w, const void* patch_b, void* packed,
@@ -928,9 +967,9 @@ int hiera_get_option(hiera_option opt) { return g_option(opt); }
 const char* hiera_kernel_name(int kind) {
   static const char* names[K_COUNT] = {
       "patch_embed", "unroll_reroll", "gemm_qkv_lnfold", "gemm_fc1_lnfold_gelu",
-      "gemm_bias_residual", "attention_tiled", "attention_packed", "f32_gemm",
-      "f32_attention", "f32_row_stats", "pack", "timeout_probe", "row_stats",
-      "attention_tcgen05", "mlp_fused"};
+      "gemm_bias_residual", "attention_window", "f32_gemm", "f32_attention",
+      "f32_row_stats", "pack", "timeout_probe", "row_stats", "attention_tcgen05",
+      "mlp_fused"};
   return (kind >= 0 && kind < K_COUNT) ? names[kind] : "unknown";
 }
 

@@ -3,7 +3,7 @@
 // scaled dot-product attention over all tokens, heads merged before proj).
 //
 // One CTA = two 128-row query tiles (A and B) of one (image, window, head) unit:
-//   warp 0      TMA: both Q tiles once, then K (128 keys x 64) and V^T (64 x 128 keys) tiles
+//   warp 0      TMA: both Q tiles once, then K and V tiles (128 keys x 64 channels each)
 //               through a KV_STAGES-deep ring shared by the two query tiles.
 //   warp 1      TMEM owner and MMA issuer: S_t = Q_t K_j^T (M=128, N=128, K=64) and
 //               O_t += P_t V_j (M=128, N=64, K=128; P_t from TMEM) for t = A, B, so that the
@@ -15,9 +15,12 @@
 //               the PV product reads its A operand (P) from there, so P never goes through
 //               shared memory. The running max is raised, and O rescaled in TMEM, only when
 //               a tile's max exceeds it by more than 2^8, so P entries stay below 256.
-// head_dim 56 is padded to 64: q/k channels 56..63 are zero; v^T padding row 56 is one, so
-// column 56 of O accumulates the softmax denominator from the very P values the tensor core
-// used; the output is O[:, :56] / O[:, 56].
+// head_dim 56 is padded to 64: q/k channels 56..63 are zero; v's padding channel 56 is one,
+// so column 56 of O accumulates the softmax denominator from the very P values the tensor core
+// used; the output is O[:, :56] / O[:, 56]. V is read in its natural [keys][channels] layout
+// as an MN-major B operand (channels contiguous), so no transposed copy of v exists.
+// Any Tq and Tkv work: query rows and keys past the ends are zero-filled by TMA, masked keys
+// take no part in the softmax and rows past Tq are not stored.
 #include <math.h>
 
 #include "common.cuh"
@@ -31,7 +34,7 @@ constexpr int KT = 128;          // keys per tile
 constexpr int KV_STAGES = 4;
 constexpr int Q_BYTES = QT * 128;                // [128 q][64 ch] bf16
 constexpr int K_BYTES = KT * 128;                // [128 keys][64 ch]
-constexpr int V_BYTES = 2 * 64 * 128;            // two [64 ch][64 keys] blocks of V^T
+constexpr int V_BYTES = KT * 128;                // [128 keys][64 ch]
 constexpr int KV_BYTES = K_BYTES + V_BYTES;
 constexpr int OFF_Q = 0;                         // Q_A, Q_B
 constexpr int OFF_KV = OFF_Q + 2 * Q_BYTES;
@@ -72,7 +75,7 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 
 // Softmax weights p in [0, 1] to bf16x2 by truncation (the high half of each fp32, lo
 // first): one byte permute per pair. Truncation leaves every weight a fraction of an ulp
-// low. The denominator is the sum of the same bf16 weights (the ones row of V^T), so for
+// low. The denominator is the sum of the same bf16 weights (v's ones channel), so for
 // rows with many comparable weights that bias cancels, and the output error is round-to-
 // nearest's. For rows dominated by a few weights it is about twice that, near 2e-3
 // relative.
@@ -102,8 +105,8 @@ __global__ void __launch_bounds__(320, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int unit = blockIdx.y;
-  const int q0 = blockIdx.x * 2 * QT;
+  const int unit = blockIdx.x;
+  const int q0 = blockIdx.y * 2 * QT;
   const int n_tiles = (p.Tkv + KT - 1) / KT;
 
   if (threadIdx.x == 0) {
@@ -158,10 +161,8 @@ __global__ void __launch_bounds__(320, 1)
       if (lane == 0) mbar_arrive_expect_tx(&kv_full[s], KV_BYTES);
       __syncwarp();
       if (lane == rr) tma_load_3d(st, &tmK, &kv_full[s], 0, j * KT, unit);
-      if (lane == ((rr + 1) & 7)) tma_load_3d(st + K_BYTES, &tmV, &kv_full[s], j * KT, 0, unit);
-      if (lane == ((rr + 2) & 7))
-        tma_load_3d(st + K_BYTES + 64 * 128, &tmV, &kv_full[s], j * KT + 64, 0, unit);
-      rr = (rr + 3) & 7;
+      if (lane == ((rr + 1) & 7)) tma_load_3d(st + K_BYTES, &tmV, &kv_full[s], 0, j * KT, unit);
+      rr = (rr + 2) & 7;
       ++issued;
     }
     if (lane == 0) {
@@ -176,7 +177,7 @@ __global__ void __launch_bounds__(320, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, KT);
-      constexpr uint32_t IDESC_O = idesc_bf16_f32(128, 64);
+      constexpr uint32_t IDESC_O = idesc_bf16_f32(128, 64) | IDESC_B_MN_MAJOR;
       const uint64_t desc0 = smem_desc_sw128(smem_u32(smem));
       bool ok = mbar_wait(q_full, 0, p.limit_ns, p.status, abort_flag);
       tc_fence_after();
@@ -209,7 +210,7 @@ __global__ void __launch_bounds__(320, 1)
         }
         if (j >= 1) {
           const int jj = j - 1, s2 = jj % KV_STAGES;
-          const uint64_t vdesc = desc_advance(desc0, (uint32_t)(OFF_KV + s2 * KV_BYTES + K_BYTES));
+          const uint64_t vdesc = smem_desc_sw128_mn64(smem_u32(smem + OFF_KV + s2 * KV_BYTES + K_BYTES));
           for (int t = 0; t < 2 && ok; ++t) {
             if (!mbar_wait(&p_full[t], (uint32_t)(jj & 1), p.limit_ns, p.status, abort_flag)) {
               ok = false;
@@ -222,12 +223,10 @@ __global__ void __launch_bounds__(320, 1)
               tc_mma_bf16_ta<false>(od, pa, vdesc, IDESC_O);
             else
               tc_mma_bf16_ta<true>(od, pa, vdesc, IDESC_O);
+            // K step kk covers keys 16kk..16kk+15: two 8-row groups of the swizzled V tile
 #pragma unroll
-            for (int kk = 1; kk < 8; ++kk) {
-              const uint32_t blk = kk >> 2, k4 = kk & 3;
-              tc_mma_bf16_ta<true>(od, pa + 8u * kk,
-                                   desc_advance(vdesc, blk * (64 * 128) + 32u * k4), IDESC_O);
-            }
+            for (int kk = 1; kk < 8; ++kk)
+              tc_mma_bf16_ta<true>(od, pa + 8u * kk, desc_advance(vdesc, 2048u * kk), IDESC_O);
             tc_commit(&o_done[t]);
             tc_commit(&p_free[t]);
           }
@@ -377,12 +376,11 @@ __global__ void __launch_bounds__(320, 1)
 
 }  // namespace
 
-bool attention_tc_supported(int Tq, int Tkv) { return Tq >= 128 && Tkv >= 128 && Tkv % 8 == 0; }
-
 hiera_status launch_attention_tc(const AttnArgs& a, cudaStream_t stream) {
-  const int units = a.B * a.nW * a.heads;
-  if (units <= 0) return HIERA_OK;
-  if (!attention_tc_supported(a.Tq, a.Tkv)) return HIERA_ERR_SHAPE;
+  const long long units_ll = (long long)a.B * a.nW * a.heads;
+  if (units_ll <= 0 || a.Tq <= 0 || a.Tkv <= 0) return HIERA_OK;
+  if (units_ll > (1ll << 30)) return HIERA_ERR_SHAPE;
+  const int units = (int)units_ll;
   CUtensorMap tmQ, tmK, tmV;
   {
     cuuint64_t dims[3] = {64, (cuuint64_t)a.Tq, (cuuint64_t)units};
@@ -397,9 +395,9 @@ hiera_status launch_attention_tc(const AttnArgs& a, cudaStream_t stream) {
     if (!encode_tmap_bf16_sw128(&tmK, a.k, 3, dims, str, box)) return HIERA_ERR_CUDA;
   }
   {
-    cuuint64_t dims[3] = {(cuuint64_t)a.Tkv, 64, (cuuint64_t)units};
-    cuuint64_t str[2] = {(cuuint64_t)a.Tkv * 2, (cuuint64_t)a.Tkv * 128};
-    cuuint32_t box[3] = {64, 64, 1};
+    cuuint64_t dims[3] = {64, (cuuint64_t)a.Tkv, (cuuint64_t)units};
+    cuuint64_t str[2] = {128, (cuuint64_t)a.Tkv * 128};
+    cuuint32_t box[3] = {64, KT, 1};
     if (!encode_tmap_bf16_sw128(&tmV, a.v, 3, dims, str, box)) return HIERA_ERR_CUDA;
   }
   AParams p;
@@ -412,16 +410,9 @@ hiera_status launch_attention_tc(const AttnArgs& a, cudaStream_t stream) {
   p.o = static_cast<bf16*>(a.o);
   p.limit_ns = g_wait_limit_ns();
   p.status = g_status_ptr();
-  static bool attr_done[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_done[dev]) {
-    if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SMEM_BYTES) != cudaSuccess)
-      return HIERA_ERR_CUDA;
-    attr_done[dev] = true;
-  }
-  dim3 grid((a.Tq + 2 * QT - 1) / (2 * QT), units);
+  if (!ensure_smem_attr(reinterpret_cast<const void*>(attn_tc_kernel), SMEM_BYTES))
+    return HIERA_ERR_CUDA;
+  dim3 grid(units, (a.Tq + 2 * QT - 1) / (2 * QT));
   if (grid.y > 65535) return HIERA_ERR_SHAPE;
   profile_mark(K_ATTN_TC, stream);
   launch_k(attn_tc_kernel, grid, dim3(320), SMEM_BYTES, stream, tmQ, tmK, tmV, p);

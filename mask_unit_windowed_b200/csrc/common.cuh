@@ -249,6 +249,19 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
   return d;
 }
 
+// The same for an MN-major operand tile 64 elements (one 128-byte swizzle atom) wide: rows of
+// K, 8-row groups 1024 B apart. The stride to a next atom along MN is never used at this
+// width; both offset fields hold 1024 B.
+__device__ __forceinline__ uint64_t smem_desc_sw128_mn64(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)(1024u >> 4) << 16;
+  d |= (uint64_t)(1024u >> 4) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)2u << 61;
+  return d;
+}
+
 // A descriptor with its start address advanced by `bytes` (a multiple of 16, staying inside
 // shared memory, so the 14-bit address field cannot carry into the next field): only the
 // low word changes, one 32-bit add instead of rebuilding the descriptor.
@@ -303,6 +316,12 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
          ((uint32_t)(M >> 4) << 24);
 }
+
+// Instruction-descriptor bit 16: the B operand is MN-major (its N elements contiguous in
+// shared memory, K along the 128-byte-swizzled rows) instead of K-major. With N = 64 bf16
+// (one 128-byte swizzle atom wide) the shared-memory descriptor is the same as for a K-major
+// tile: 8-row groups 1024 bytes apart.
+constexpr uint32_t IDESC_B_MN_MAJOR = 1u << 16;
 
 // ------------------------------------------------------------------ small numeric helpers
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

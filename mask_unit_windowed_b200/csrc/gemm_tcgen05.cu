@@ -54,7 +54,6 @@ struct KParams {
   bf16* v;
   bf16* r;
   int tokens, nW, heads, d_out, Tq, Tkv;
-  int vt;  // 1: v written transposed, [B][nW][heads][64][Tkv]
   uint64_t limit_ns;
   unsigned int* status;
   const float2* stats_in;  // FOLD: [M][stats_parts] partial (mean, M2) of A's rows
@@ -395,23 +394,6 @@ __global__ void __launch_bounds__(320, 1)
             v[8 * g + 7] += bf16_hi(rr.w);
           }
         }
-        if (EPI == EPI_QKV && which == 2 && p.vt) {
-          // v for the tensor-core attention, transposed: channel-major rows of Tkv keys.
-          // Padding row 56 holds ones, so the P V product also yields each query row's
-          // softmax denominator; rows 57..63 are zero. Lanes hold consecutive tokens, so
-          // each store instruction covers a run of keys.
-          if (writer) {
-            const int h = (n0 - 2 * p.d_out + c_begin + c) / 56;
-            const int w = tok % p.nW, j = tok / p.nW;
-            bf16* base = p.v + (((long long)b * p.nW + w) * p.heads + h) * 64 * (long long)p.Tkv + j;
-#pragma unroll
-            for (int e = 0; e < 56; ++e) base[(long long)e * p.Tkv] = __float2bfloat16_rn(v[e]);
-            base[56LL * p.Tkv] = __float2bfloat16_rn(1.f);
-#pragma unroll
-            for (int e = 57; e < 64; ++e) base[(long long)e * p.Tkv] = __float2bfloat16_rn(0.f);
-          }
-          continue;
-        }
         // ---- destination of this lane's row for this chunk
         bf16* dst_row = nullptr;
         bool valid = row_ok;
@@ -453,9 +435,12 @@ __global__ void __launch_bounds__(320, 1)
             v[8 * g + 7] = bf16_hi(pk.w);
           }
         }
+        // channels 56..63 of a head row: zero padding for q and k; for v, channel 56 holds
+        // 1.0 (bf16 0x3F80) so that the attention's P V product also yields each query
+        // row's softmax denominator
         if (EPI == EPI_QKV && CH == 56)
           *reinterpret_cast<uint4*>(stg + (lane << 7) + ((7 ^ (lane & 7)) << 4)) =
-              make_uint4(0u, 0u, 0u, 0u);
+              make_uint4(which == 2 ? 0x3F80u : 0u, 0u, 0u, 0u);
         if (EPI == EPI_STORE && p.stats_out != nullptr && row_ok) {
           float s = 0.f;
 #pragma unroll
@@ -600,7 +585,6 @@ hiera_status run(const TcGemmArgs& a, cudaStream_t stream) {
   p.d_out = a.d_out;
   p.Tq = a.Tq;
   p.Tkv = a.Tkv;
-  p.vt = a.vt;
   p.limit_ns = g_wait_limit_ns();
   p.status = g_status_ptr();
   p.stats_in = static_cast<const float2*>(a.stats_in);
@@ -609,15 +593,7 @@ hiera_status run(const TcGemmArgs& a, cudaStream_t stream) {
   p.stats_out_parts = a.stats_out_parts;
 
   auto kern = tc_gemm_kernel<BN, EPI, FOLD, POOLED>;
-  static bool attr_done[64] = {false};  // per device
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_done[dev]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
-        cudaSuccess)
-      return HIERA_ERR_CUDA;
-    attr_done[dev] = true;
-  }
+  if (!ensure_smem_attr(reinterpret_cast<const void*>(kern), C::SMEM_BYTES)) return HIERA_ERR_CUDA;
   const int m_tiles = POOLED ? (a.M / 4 + 31) / 32 : (a.M + BM - 1) / BM;
   const int tiles = m_tiles * (a.N / BN);
   if (tiles == 0) return HIERA_OK;

@@ -16,8 +16,8 @@ unsigned int* g_status_ptr();            // device address of the status word (c
 // kernel ids reported by the launch profiler (hiera_profile_begin)
 enum KernelId {
   K_PATCH_EMBED = 0, K_PERMUTE = 1, K_GEMM_QKV = 2, K_GEMM_GELU = 3, K_GEMM_STORE = 4,
-  K_ATTN_TILED = 5, K_ATTN_PACKED = 6, K_F32_GEMM = 7, K_F32_ATTN = 8, K_F32_STATS = 9,
-  K_PACK = 10, K_PROBE = 11, K_ROW_STATS = 12, K_ATTN_TC = 13, K_MLP_FUSED = 14, K_COUNT = 15
+  K_ATTN_WIN = 5, K_F32_GEMM = 6, K_F32_ATTN = 7, K_F32_STATS = 8, K_PACK = 9, K_PROBE = 10,
+  K_ROW_STATS = 11, K_ATTN_TC = 12, K_MLP_FUSED = 13, K_COUNT = 14
 };
 void profile_mark(int kind, cudaStream_t stream);  // no-op unless a session is open
 
@@ -45,14 +45,13 @@ struct TcGemmArgs {
   void* out;
   const void* residual;
   int ldo;
-  // EPI_QKV: scatter into head-major q/k/v [B][nW][heads][T][64] (+ pooled residual r)
+  // EPI_QKV: scatter into head-major q/k/v [B][nW][heads][T][64], channels 56..63 zero
+  // except v's channel 56 = 1 (+ pooled residual r)
   void* q;
   void* k;
   void* v;
   void* r;                // transition residual [B, tokens/4, d_out] (columns 3*d_out..)
   int tokens, nW, heads, d_out, Tq, Tkv;
-  int vt;                 // 1: write v transposed, [B][nW][heads][64][Tkv] with padding row
-                          //    56 = 1 (tensor-core attention)
   int pooled;             // 1: rows n, n+T/4, n+T/2, n+3T/4 of each image loaded together and
                           //    q / r columns max-pooled over them (q_stride 4)
 };
@@ -110,19 +109,26 @@ inline int store_stats_parts(int N) { return 2 * (N / store_bn(N)); }
 hiera_status launch_row_partials_bf16(const void* x, int M, int K, float2* out,
                                       cudaStream_t stream);
 
-// ---------------------------------------------------------------- attention (bf16, mma.sync)
+// ---------------------------------------------------------------- attention (bf16, tcgen05)
 struct AttnArgs {
-  const void* q;  // [B][nW][heads][Tq][64]
-  const void* k;  // [B][nW][heads][Tkv][64]
-  const void* v;
+  const void* q;  // [B][nW][heads][Tq][64], channels 56..63 zero
+  const void* k;  // [B][nW][heads][Tkv][64], channels 56..63 zero
+  const void* v;  // [B][nW][heads][Tkv][64], channel 56 = 1, 57..63 zero
   void* o;        // [B][Tq*nW][d_out], token j*nW + w, channel h*56 + e
   int B, nW, heads, Tq, Tkv, d_out;
 };
-hiera_status launch_attention_bf16(const AttnArgs& a, cudaStream_t stream);
-// Tensor-core (tcgen05) attention for Tq >= 128 and Tkv >= 128: q/k as above, v transposed
-// [B][nW][heads][64][Tkv] with row 56 = 1 (a.v), Tkv a multiple of 8.
-bool attention_tc_supported(int Tq, int Tkv);
+// Small mask-unit windows (Tkv a power of two in 4..64, Tq = Tkv or Tkv / 4): several units
+// per 128-row tile, one exact softmax pass.
+bool attention_win_supported(int Tq, int Tkv);
+hiera_status launch_attention_win(const AttnArgs& a, cudaStream_t stream);
+// Any Tq, Tkv: 128-key tiles with an online softmax (global attention).
 hiera_status launch_attention_tc(const AttnArgs& a, cudaStream_t stream);
+// The windowed kernel where it applies, else the general one.
+hiera_status launch_attention(const AttnArgs& a, cudaStream_t stream);
+
+// Raise `kern`'s dynamic shared-memory limit to `bytes` on the current device, once per
+// (kernel, device); thread-safe. False if the runtime refused.
+bool ensure_smem_attr(const void* kern, int bytes);
 
 // TMA descriptor of a bf16 tensor with 128-byte swizzle (cuTensorMapEncodeTiled).
 bool encode_tmap_bf16_sw128(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,

@@ -592,15 +592,7 @@ hiera_status run_mlp(const MlpArgs& a, cudaStream_t stream) {
   p.limit_ns = g_wait_limit_ns();
   p.status = g_status_ptr();
   auto kern = mlp_fused_kernel<D>;
-  static bool attr_done[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_done[dev]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
-        cudaSuccess)
-      return HIERA_ERR_CUDA;
-    attr_done[dev] = true;
-  }
+  if (!ensure_smem_attr(reinterpret_cast<const void*>(kern), C::SMEM_BYTES)) return HIERA_ERR_CUDA;
   const int tiles = (a.M + BM - 1) / BM;
   int grid = g_num_sms();
   if (grid > tiles) grid = tiles;

@@ -263,32 +263,20 @@ hiera_status launch_patch_embed(const void* img, const void* packed, const void*
   const float* wt = reinterpret_cast<const float*>(pk);
   const float* bias = reinterpret_cast<const float*>(pk + PATCH_OFF_BIAS);
   const bf16* w16 = reinterpret_cast<const bf16*>(pk + PATCH_OFF_W16);
-  static bool attr_done[2][64] = {{false}};
-  int dev = 0;
-  cudaGetDevice(&dev);
   profile_mark(K_PATCH_EMBED, stream);
   if (dtype_bf16) {
     dim3 grid((G + SEG - 1) / SEG, (G + MMA_ROWS - 1) / MMA_ROWS, B);
     if (grid.y > 65535 || grid.z > 65535) return HIERA_ERR_SHAPE;
-    if (dev < 64 && !attr_done[1][dev]) {
-      if (cudaFuncSetAttribute(patch_embed_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               MMA_SMEM) != cudaSuccess)
-        return HIERA_ERR_CUDA;
-      attr_done[1][dev] = true;
-    }
+    if (!ensure_smem_attr(reinterpret_cast<const void*>(patch_embed_mma_kernel), MMA_SMEM))
+      return HIERA_ERR_CUDA;
     launch_k(patch_embed_mma_kernel, grid, dim3(256), MMA_SMEM, stream,
              static_cast<const bf16*>(img), w16, bias, static_cast<const bf16*>(pos),
              static_cast<bf16*>(out), stats_out, img_side);
   } else {
     dim3 grid((G + SEG - 1) / SEG, (G + ROWS - 1) / ROWS, B);
     if (grid.y > 65535 || grid.z > 65535) return HIERA_ERR_SHAPE;
-    if (dev < 64 && !attr_done[0][dev]) {
-      if (cudaFuncSetAttribute(patch_embed_kernel,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               SMEM_TOTAL) != cudaSuccess)
-        return HIERA_ERR_CUDA;
-      attr_done[0][dev] = true;
-    }
+    if (!ensure_smem_attr(reinterpret_cast<const void*>(patch_embed_kernel), SMEM_TOTAL))
+      return HIERA_ERR_CUDA;
     patch_embed_kernel<<<grid, 256, SMEM_TOTAL, stream>>>(
         static_cast<const float*>(img), wt, bias, static_cast<const float*>(pos),
         static_cast<float*>(out), img_side);

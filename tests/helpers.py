@@ -29,3 +29,20 @@ def max_abs(got, ref):
 
 def block_weights_dev(p, dtype):
     return {k: dev(v, dtype) for k, v in p.items()}
+
+
+def row_rel_l2(got, ref):
+    """rel-L2 of every row (last axis) of got against ref."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    return np.linalg.norm(got - ref, axis=-1) / np.maximum(np.linalg.norm(ref, axis=-1), 1e-30)
+
+
+def unit_rel_l2(o_got, o_ref, B, Tq, nW, heads, hd=56):
+    """rel-L2 of every (image, window, head) unit of a merged attention output
+    [B, Tq * nW, heads * hd] (token j * nW + w, channel h * hd + e): [B, nW, heads]."""
+    g = np.asarray(o_got, np.float64).reshape(B, Tq, nW, heads, hd)
+    r = np.asarray(o_ref, np.float64).reshape(B, Tq, nW, heads, hd)
+    num = np.sqrt(((g - r) ** 2).sum(axis=(1, 4)))
+    den = np.maximum(np.sqrt((r ** 2).sum(axis=(1, 4))), 1e-30)
+    return num / den

@@ -72,3 +72,53 @@ def test_workspace_and_pack_sizes():
     bb = hb.BackboneDesc(B=1, img=512)
     assert hb.backbone_packed_bytes(bb) > 2 * 69_000_000
     assert hb.backbone_workspace_bytes(bb) > 2 * 16384 * 112 * 2
+
+
+def test_attention_entry_rejects_bad_arguments_before_any_launch():
+    L = hb.lib()
+    a, b = ctypes.c_void_p(1 << 20), ctypes.c_void_p(2 << 20)
+    assert L.hiera_attention(None, a, a, b, 1, 1, 1, 64, 64, None) == 1
+    assert L.hiera_attention(a, a, a, b, 0, 1, 1, 64, 64, None) == 1
+    assert L.hiera_attention(a, a, a, b, 1, 1, 1, 64, 0, None) == 1
+    misaligned = ctypes.c_void_p((1 << 20) + 8)
+    assert L.hiera_attention(a, misaligned, a, b, 1, 1, 1, 64, 64, None) == 4
+    assert L.hiera_attention(a, a, a, b, 1 << 16, 1 << 10, 8, 64, 64, None) == 2
+
+
+def test_static_scratch_size_matches_header():
+    """The binding reads the scratch size from the library; it must equal the header's
+    HIERA_STATIC_SCRATCH_BYTES, so tests of the size limit test the real boundary."""
+    import re
+    with open(hb.HEADER) as f:
+        m = re.search(r"#define HIERA_STATIC_SCRATCH_BYTES \(\(size_t\)(\d+) << (\d+)\)", f.read())
+    assert m is not None
+    assert hb.static_scratch_bytes() == int(m.group(1)) << int(m.group(2))
+
+
+def test_binding_rejects_mismatched_tensors_before_any_launch():
+    """Shapes and dtypes are compared with the descriptor before the C call: a tensor that
+    does not match would otherwise be read or written past its end."""
+    import torch
+    d = hb.BlockDesc(B=2, tokens=256, dim_in=112, dim_out=112, heads=2)
+    packed = torch.empty(hb.block_packed_bytes(d), dtype=torch.uint8)
+    with pytest.raises(ValueError, match="shape"):
+        hb.block_forward(d, packed, torch.empty(2, 128, 112, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="dtype"):
+        hb.block_forward(d, packed, torch.empty(2, 256, 112, dtype=torch.float32))
+    with pytest.raises(ValueError, match="shape"):
+        hb.block_forward_noalloc(d, packed, torch.empty(2, 256, 112, dtype=torch.bfloat16),
+                                 out=torch.empty(2, 256, 224, dtype=torch.bfloat16))
+    bb = hb.BackboneDesc(B=1, img=64)
+    with pytest.raises(ValueError, match="shape"):
+        hb.backbone_forward(bb, packed, torch.empty(1, 64, 64, 3, dtype=torch.bfloat16))
+    q = torch.empty(1, 4, 2, 64, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="shape"):
+        hb.attention(q, torch.empty(1, 4, 2, 64, 56, dtype=torch.bfloat16), q)
+    with pytest.raises(ValueError, match="shape"):
+        hb.unroll(torch.empty(1, 60, 112, dtype=torch.bfloat16), 8, 3)
+    with pytest.raises(ValueError, match="shape"):
+        hb.linear(torch.empty(4, 16, dtype=torch.bfloat16),
+                  torch.empty(32, 8, dtype=torch.bfloat16))
+    # shapes right, but host tensors: still refused before the library is called
+    with pytest.raises(ValueError, match="CUDA"):
+        hb.block_forward(d, packed, torch.empty(2, 256, 112, dtype=torch.bfloat16))

@@ -1,9 +1,10 @@
 """Hiera-B+ backbone through the C ABI against the fp64 oracle.
 
-bf16 mode: rel-L2 <= 3e-2 per feature after the full backbone; fp32 mode: max-abs
-<= 1e-4 relative to the feature scale. At 2048^2 the oracle cannot evaluate the global
-stages; mask-unit-local stages 0-1 are checked exactly on sampled mask units (each one's
-receptive field is its own 32x32-pixel patch plus the 3-pixel convolution halo).
+bf16 mode: rel-L2 <= 3e-2 per feature after the full backbone, and every feature pixel
+(its channel vector) within PIXEL_BOUND rel-L2, so that a fault confined to a few mask
+units or one image is not diluted by the rest of the map. fp32 mode: max-abs <= 1e-4 on
+every feature element. At 2048^2 the oracle runs the global stages with its row-chunked
+attention (same definition, bounded host memory).
 """
 
 import numpy as np
@@ -14,11 +15,23 @@ from mask_unit_windowed_b200 import binding as hb
 from mask_unit_windowed_b200 import synthetic as syn
 from oracle import unrolled as U
 
-from helpers import TORCH_DT, dev, host, max_abs, rel_l2
+from helpers import TORCH_DT, dev, host, max_abs, rel_l2, row_rel_l2
 
 pytestmark = pytest.mark.gpu
 
 BF16_REL_L2 = 3e-2
+PIXEL_BOUND = 3e-2   # the per-feature tolerance, held by every pixel (measured: <= 1.8e-2)
+F32_MAX_ABS = 1e-4
+
+
+def check_feature(s, f, r, bound=BF16_REL_L2, pixel_bound=PIXEL_BOUND):
+    assert f.shape == r.shape
+    assert np.isfinite(f).all()
+    px = row_rel_l2(f, r)
+    worst = np.unravel_index(np.argmax(px), px.shape)
+    print(f"stage {s}: rel-L2 {rel_l2(f, r):.3e}, max pixel rel-L2 {px.max():.3e} at {worst}")
+    assert rel_l2(f, r) <= bound, (s, rel_l2(f, r))
+    assert px.max() <= pixel_bound, (s, px.max(), worst)
 
 
 def weights_dev(p, dtype):
@@ -43,8 +56,7 @@ def test_backbone_bf16_small(img, B):
     feats, p, x, *_ = run_backbone(img, B, "bf16", 31, "random")
     ref = U.backbone_forward(x, p)
     for s, (f, r) in enumerate(zip(feats, ref)):
-        assert f.shape == r.shape
-        assert rel_l2(f, r) <= BF16_REL_L2, (s, rel_l2(f, r))
+        check_feature(s, f, r)
 
 
 def test_backbone_bf16_lagged_mask_unit_flag():
@@ -52,14 +64,18 @@ def test_backbone_bf16_lagged_mask_unit_flag():
     flags = [True] * 6 + [False] * 18
     ref = U.backbone_forward(x, p, mask_unit_attn_override=flags)
     for s, (f, r) in enumerate(zip(feats, ref)):
-        assert rel_l2(f, r) <= BF16_REL_L2, (s, rel_l2(f, r))
+        check_feature(s, f, r)
 
 
-def test_backbone_f32_small():
-    feats, p, x, *_ = run_backbone(64, 1, "f32", 33, "random")
+@pytest.mark.parametrize("img", [64, 128])
+def test_backbone_f32(img):
+    """fp32 mode (fp32 SIMT arithmetic throughout): every feature element within an
+    absolute 1e-4 of the fp64 oracle after all 24 blocks."""
+    feats, p, x, *_ = run_backbone(img, 1, "f32", 33, "random")
     ref = U.backbone_forward(x, p)
     for s, (f, r) in enumerate(zip(feats, ref)):
-        assert max_abs(f, r) <= 1e-4 * max(1.0, np.abs(r).max()), (s, max_abs(f, r))
+        print(f"stage {s}: max-abs {max_abs(f, r):.3e}, max |ref| {np.abs(r).max():.3f}")
+        assert max_abs(f, r) <= F32_MAX_ABS, (s, max_abs(f, r))
 
 
 def test_cfg4_backbone_512_bf16():
@@ -70,7 +86,7 @@ def test_cfg4_backbone_512_bf16():
     shapes = [(1, 128, 128, 112), (1, 64, 64, 224), (1, 32, 32, 448), (1, 16, 16, 896)]
     for s, (f, r) in enumerate(zip(feats, ref)):
         assert f.shape == shapes[s]
-        assert rel_l2(f, r) <= BF16_REL_L2, (s, rel_l2(f, r))
+        check_feature(s, f, r)
 
 
 def test_batch_rows_independent_bitwise():
@@ -88,44 +104,16 @@ def test_batch_rows_independent_bitwise():
             assert torch.equal(a[i:i + 1], b), (i, s, diff)
 
 
-def _oracle_mask_unit_stages01(x_img, p, my, mx, G0):
-    """Stages 0-1 of one mask unit (8x8 stage-0 tokens) from its padded pixel patch."""
-    img = x_img.shape[1]
-    pad = np.zeros((1, img + 6, img + 6, 4))
-    pad[:, 3:3 + img, 3:3 + img] = x_img
-    crop = pad[:, 32 * my:32 * my + 38, 32 * mx:32 * mx + 38]       # halo included
-    tok = U.patch_embed(crop, p["patch_w"], p["patch_b"], pad=0)    # [1, 64, 112] raster 8x8
-    ys, xs = np.meshgrid(np.arange(8) + 8 * my, np.arange(8) + 8 * mx, indexing="ij")
-    tok = tok + np.asarray(p["pos_embed"], np.float64)[(ys * G0 + xs).reshape(-1)][None]
-    t = U.unroll(tok, 8, 3)
-    sched = U.block_schedule()
-    feats = []
-    for i in range(5):
-        c = sched[i]
-        window = (64 >> (2 * c["stage"])) * c["q_stride"]
-        t = U.block_forward(t, p["blocks"][i], c["heads"], c["q_stride"], window, True)
-        if i == 1:
-            feats.append(U.reroll(t, 8, 3)[0])
-        if i == 4:
-            feats.append(U.reroll(t, 4, 2)[0])
-    return feats
-
-
-def test_cfg5_backbone_2048_sampled_mask_units():
+def test_cfg5_backbone_2048_all_features():
     """Hiera-B+ at 2048x2048x4, bf16, batch 1 (262144 stage-0 tokens, 4096 mask units,
-    global attention over 16384 tokens in stage 2): stage 0 and 1 features of sampled
-    mask units against the oracle; stage 2 and 3 features finite."""
+    global attention over 16384 tokens in stage 2 and block 5's 16384 pooled queries
+    against 65536 keys): all four features against the oracle (row-chunked attention)."""
     feats, p, x, *_ = run_backbone(2048, 1, "bf16", 4, "init")
-    G0 = 512
-    x64 = np.asarray(x, np.float64)
-    for my, mx in [(0, 0), (63, 63), (0, 63), (17, 41), (40, 3)]:
-        f0, f1 = _oracle_mask_unit_stages01(x64, p, my, mx, G0)
-        g0 = feats[0][0, 8 * my:8 * my + 8, 8 * mx:8 * mx + 8]
-        g1 = feats[1][0, 4 * my:4 * my + 4, 4 * mx:4 * mx + 4]
-        assert rel_l2(g0, f0) <= BF16_REL_L2, rel_l2(g0, f0)
-        assert rel_l2(g1, f1) <= BF16_REL_L2, rel_l2(g1, f1)
-    assert np.isfinite(feats[2]).all() and np.isfinite(feats[3]).all()
-    assert feats[2].shape == (1, 128, 128, 448) and feats[3].shape == (1, 64, 64, 896)
+    ref = U.backbone_forward(x, p, row_chunk=256)
+    shapes = [(1, 512, 512, 112), (1, 256, 256, 224), (1, 128, 128, 448), (1, 64, 64, 896)]
+    for s, (f, r) in enumerate(zip(feats, ref)):
+        assert f.shape == shapes[s]
+        check_feature(s, f, r)
 
 
 def test_global_block_16384_tokens_sampled_rows():

@@ -21,13 +21,22 @@ def test_timeout_probe_reports_and_recovers():
 
 
 def test_workspace_too_small_rejected():
+    """Both layers refuse a workspace smaller than hiera_block_workspace_bytes(): the
+    binding before the call, the library itself (HIERA_ERR_WORKSPACE) when called directly,
+    and nothing is launched."""
+    import ctypes
     desc = hb.BlockDesc(B=1, tokens=256, dim_in=112, dim_out=112, heads=2)
     x = torch.zeros(1, 256, 112, device="cuda", dtype=torch.bfloat16)
+    y = torch.zeros(1, 256, 112, device="cuda", dtype=torch.bfloat16)
     packed = torch.zeros(hb.block_packed_bytes(desc), dtype=torch.uint8, device="cuda")
     ws = torch.empty(16, dtype=torch.uint8, device="cuda")
-    with pytest.raises(hb.HieraError) as e:
+    with pytest.raises(ValueError, match="workspace"):
         hb.block_forward(desc, packed, x, workspace=ws)
-    assert e.value.code == 5
+    d = desc.c()
+    code = hb.lib().hiera_block_forward(ctypes.byref(d), packed.data_ptr(), x.data_ptr(),
+                                        y.data_ptr(), ws.data_ptr(), 16, None)
+    assert code == 5
+    assert hb.device_status() == 0
 
 
 def test_tensor_core_path_gelu_within_error_bound():

@@ -39,7 +39,7 @@ def _rel_l2(a, b):
 ])
 def test_noalloc_matches_workspace_entry_point_twice(dtype, args):
     desc, packed, x = _case(dtype, *args)
-    assert hb.block_workspace_bytes(desc) <= hb.STATIC_SCRATCH_BYTES
+    assert hb.block_workspace_bytes(desc) <= hb.static_scratch_bytes()
     ref = hb.block_forward(desc, packed, x)
     for _ in range(2):   # the second call finds the first call's data in the scratch
         y = hb.block_forward_noalloc(desc, packed, x)
@@ -54,7 +54,7 @@ def test_noalloc_matches_workspace_entry_point_twice(dtype, args):
 
 def test_noalloc_rejects_blocks_larger_than_the_static_scratch():
     desc, packed, x = _case("bf16", 8, 1024, 448, 448, 8, 1, 1, False, 54)
-    assert hb.block_workspace_bytes(desc) > hb.STATIC_SCRATCH_BYTES
+    assert hb.block_workspace_bytes(desc) > hb.static_scratch_bytes()
     with pytest.raises(hb.HieraError) as e:
         hb.block_forward_noalloc(desc, packed, x)
     assert e.value.code == 5   # HIERA_ERR_WORKSPACE
