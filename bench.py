@@ -585,6 +585,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "clocks": clocks.record(),
         "gpu_launches": n_launches * replays * args.steps,
         "launches_per_forward": n_launches,
+        "per_launch": [[n, round(fl / 1e9, 3), round(ms * 1e3, 2)]
+                       for (n, ms), (_, fl) in zip(per_launch, flops)],
     }
     print(json.dumps(line), flush=True)
 

@@ -5,8 +5,9 @@
 // A window holds at most 64 keys (stage 0: 64 keys and 64 queries; the stage-1 transition:
 // 64 keys, 16 pooled queries; stage 1: 16 and 16), so one 128-key tile holds the keys of
 // U = 128 / TKV whole (image, window, head) units and the softmax is a single exact pass,
-// with no running max. A tile stacks the U units' queries in R = U * TQ rows and their keys
-// in 128 columns:
+// with no running max. A tile stacks the U units' queries in U row slots (TQ rows each, or
+// 32 rows of which TQ are used when TQ < 32 <= TKV, so that a warp never holds two units'
+// keys) and their keys in 128 columns:
 //   S = Q K^T     M = 128, N = 128, K = 64: unit i's rows meet every unit's keys, and only
 //                 the diagonal block [i*TQ, +TQ) x [i*TKV, +TKV) is used;
 //   P             per row, 2^(s*log2(e)/sqrt(56) - m) over its own unit's keys and exactly 0
@@ -74,10 +75,16 @@ template <int TQ, int TKV>
 struct WinCfg {
   static_assert(TKV >= 4 && TKV <= 64 && (TKV & (TKV - 1)) == 0, "window keys");
   static_assert(TQ == TKV || TQ * 4 == TKV, "q_stride 1 or 4");
-  static constexpr int U = 128 / TKV;                         // units per tile
-  static constexpr int R = U * TQ;                            // query rows per tile
-  static constexpr int CW = TQ >= 32 ? TKV : TKV * 32 / TQ;   // S columns one warp reads
+  // Rows per unit: TQ, or a 32-row slot (one unit per warp, TQ rows used) when a unit has
+  // fewer than 32 queries but 32 or more keys, so that no warp reads two units' keys.
+  static constexpr bool SLOT = TQ < 32 && TKV >= 32;
+  static constexpr int SR = SLOT ? 32 : TQ;
+  static constexpr int U = (128 / SR < 128 / TKV) ? 128 / SR : 128 / TKV;  // units per tile
+  static constexpr int R = U * SR;                            // tile rows in use
+  static constexpr int CW = SR >= 32 ? TKV : TKV * 32 / TQ;   // S columns one warp reads
+  static constexpr int Q_TX = U * TQ * 128;                   // Q bytes per tile
   static_assert(CW >= 32 && CW <= 128 && 128 % CW == 0, "warp column window");
+  static_assert(U * TKV <= 128 && R <= 128, "tile");
 };
 
 template <int TQ, int TKV>
@@ -85,7 +92,7 @@ __global__ void __launch_bounds__(320, 1)
     attn_win_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const WParams p) {
   using C = WinCfg<TQ, TKV>;
-  constexpr int U = C::U, R = C::R, CW = C::CW;
+  constexpr int U = C::U, R = C::R, CW = C::CW, SR = C::SR;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t* smem = smem_raw + pad;
@@ -145,11 +152,16 @@ __global__ void __launch_bounds__(320, 1)
         break;
       }
       uint8_t* st = smem + s * WSTAGE_BYTES;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&full[s], R * 128 + 2 * WK_BYTES);
-        tma_load_2d(st, &tmQ, &full[s], 0, tile * R);
-      }
+      if (lane == 0) mbar_arrive_expect_tx(&full[s], C::Q_TX + 2 * WK_BYTES);
       __syncwarp();
+      if constexpr (C::SLOT) {
+        // unit u's TQ query rows into its 32-row slot (4 KB apart: the swizzle pattern of
+        // every slot starts on a 1024-byte boundary)
+        if (lane >= 3 && lane < 3 + U)
+          tma_load_2d(st + (lane - 3) * SR * 128, &tmQ, &full[s], 0, (tile * U + lane - 3) * TQ);
+      } else {
+        if (lane == 0) tma_load_2d(st, &tmQ, &full[s], 0, tile * R);
+      }
       if (lane == 1) tma_load_2d(st + WQ_BYTES, &tmK, &full[s], 0, tile * 128);
       if (lane == 2) tma_load_2d(st + WQ_BYTES + WK_BYTES, &tmV, &full[s], 0, tile * 128);
       ++issued;
@@ -220,8 +232,8 @@ __global__ void __launch_bounds__(320, 1)
     const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
     const int r = quarter * 32 + lane;       // tile row
     const bool warp_rows = quarter * 32 < R; // warp-uniform: this warp holds rows of the tile
-    const int c0 = ((quarter * 32) / TQ) * TKV;  // first S column this warp reads
-    const int my_chunk = ((r / TQ) * TKV - c0) / TKV;  // this row's keys: chunk my_chunk of
+    const int c0 = ((quarter * 32) / SR) * TKV;  // first S column this warp reads
+    const int my_chunk = ((r / SR) * TKV - c0) / TKV;  // this row's keys: chunk my_chunk of
                                                         // TKV columns of the warp's window
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     const uint32_t sb = lane_base + (uint32_t)(256 * g), ob = sb + 128u;
@@ -299,9 +311,9 @@ __global__ void __launch_bounds__(320, 1)
       }
       tc_fence_before();
       mbar_arrive(&t_free[g]);  // buffer g may take the S of tile t+2
-      const int unit = tile * U + r / TQ;
-      if (warp_rows && r < R && unit < p.units) {
-        const int j = r % TQ;
+      const int unit = tile * U + r / SR;
+      const int j = r % SR;
+      if (warp_rows && r < R && j < TQ && unit < p.units) {
         const int h = unit % p.heads;
         const int w = (unit / p.heads) % p.nW;
         const int bimg = unit / (p.heads * p.nW);
@@ -336,7 +348,7 @@ hiera_status run_win(const AttnArgs& a, cudaStream_t stream) {
   {
     cuuint64_t dims[2] = {64, (cuuint64_t)(units * TQ)};
     cuuint64_t str[1] = {128};
-    cuuint32_t box[2] = {64, (cuuint32_t)C::R};
+    cuuint32_t box[2] = {64, (cuuint32_t)(C::SLOT ? TQ : C::R)};
     if (!encode_tmap_bf16_sw128(&tmQ, a.q, 2, dims, str, box)) return HIERA_ERR_CUDA;
   }
   {

@@ -95,6 +95,7 @@ struct Cfg {
   static_assert(B_BYTES % 1024 == 0, "W tile must keep 1024-byte alignment");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128");
   static_assert(HALF % CH == 0 && CH % 8 == 0, "epilogue chunking");
+  static_assert(CONST_OFF % 16 == 0 && (HALF * 4) % 16 == 0, "16-byte constant loads");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
@@ -284,6 +285,8 @@ __global__ void __launch_bounds__(320, 1)
     // epilogue warps. They are loaded a tile ahead, CPL per lane, and staged at the tile's
     // start.
     constexpr int CPL = (HALF + 31) / 32;
+    // (16-byte aligned: CONST_OFF and HALF * 4 are multiples of 16, and so is every chunk
+    // start c * 4)
     float* col_sum = reinterpret_cast<float*>(smem + C::CONST_OFF) + ew * 2 * HALF;
     float* col_const = col_sum + HALF;
     float nsum[CPL], nconst[CPL];
@@ -369,13 +372,30 @@ __global__ void __launch_bounds__(320, 1)
         uint32_t r[CH];
         tmem_load<CH>(tbase + (uint32_t)c, r);
         float v[CH];
+        // the column constants of this chunk, four per 16-byte shared-memory load (every
+        // lane reads the same address: one broadcast per load)
+        const float4* cs4 = reinterpret_cast<const float4*>(col_sum + c);
+        const float4* cc4 = reinterpret_cast<const float4*>(col_const + c);
 #pragma unroll
-        for (int i = 0; i < CH; ++i) {
-          const int cl = c + i;  // column within this warp's half
-          float x = FOLD ? fmaf(fa, __uint_as_float(r[i]), fmaf(fb, col_sum[cl], col_const[cl]))
-                         : __uint_as_float(r[i]) + col_const[cl];
-          if (EPI == EPI_GELU) x = gelu_fast(x);
-          v[i] = x;
+        for (int g = 0; g < CH / 4; ++g) {
+          const float4 k4 = cc4[g];
+          const float kc[4] = {k4.x, k4.y, k4.z, k4.w};
+          float sc[4] = {0.f, 0.f, 0.f, 0.f};
+          if (FOLD) {
+            const float4 s4 = cs4[g];
+            sc[0] = s4.x;
+            sc[1] = s4.y;
+            sc[2] = s4.z;
+            sc[3] = s4.w;
+          }
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i = 4 * g + e;
+            float x = FOLD ? fmaf(fa, __uint_as_float(r[i]), fmaf(fb, sc[e], kc[e]))
+                           : __uint_as_float(r[i]) + kc[e];
+            if (EPI == EPI_GELU) x = gelu_fast(x);
+            v[i] = x;
+          }
         }
         // ---- finish the values of this chunk (residual; the q / residual pooling of a
         // transition is taken on the packed values when they are copied out)
