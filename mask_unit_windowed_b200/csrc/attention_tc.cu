@@ -5,16 +5,20 @@
 // One CTA = two 128-row query tiles (A and B) of one (image, window, head) unit:
 //   warp 0      TMA: both Q tiles once, then K and V tiles (128 keys x 64 channels each)
 //               through a KV_STAGES-deep ring shared by the two query tiles.
-//   warp 1      TMEM owner and MMA issuer: S_t = Q_t K_j^T (M=128, N=128, K=64) and
-//               O_t += P_t V_j (M=128, N=64, K=128; P_t from TMEM) for t = A, B, so that the
-//               tensor core works on one tile while the other tile's softmax runs.
+//   warp 1      TMEM owner and MMA issuer: S_t(j) = Q_t K_j^T (M=128, N=128, K=64) and
+//               O_t += P_t(j) V_j (M=128, N=64, K=128; P_t(j) read from TMEM) for t = A, B.
 //   warps 2-5   softmax of tile A, warps 6-9 of tile B, one query row per thread (TMEM lane
 //               = row): row max, then the weights P = 2^(s log2(e)/sqrt(56) - m) on the
-//               MUFU unit, cut to bf16 by a byte permute per pair (the conversion unit
-//               shares the MUFU pipe) and stored as bf16 pairs into TMEM next to S and O;
-//               the PV product reads its A operand (P) from there, so P never goes through
-//               shared memory. The running max is raised, and O rescaled in TMEM, only when
-//               a tile's max exceeds it by more than 2^8, so P entries stay below 256.
+//               MUFU unit, cut to bf16 by a byte permute per pair, stored as bf16 pairs over
+//               the S columns they came from; the PV product reads its A operand (P) from
+//               there, so P never goes through shared memory. The running max is raised, and
+//               O rescaled in TMEM, only when a tile's max exceeds it by more than 2^8, so P
+//               entries stay below 256.
+// TMEM holds three S/P buffers and the two O accumulators. Slot k = 2j + t (tile t, key tile
+// j) uses buffer k mod 3, so a softmax warpgroup never waits for its own previous P V
+// product before writing the next weights: buffer k mod 3 was last used by slot k - 3 (the
+// other tile), whose P V the MMA thread issues before S of slot k (issue order S_A(j),
+// P_A(j-1) V, S_B(j), P_B(j-1) V; the tensor core executes one thread's MMAs in order).
 // head_dim 56 is padded to 64: q/k channels 56..63 are zero; v's padding channel 56 is one,
 // so column 56 of O accumulates the softmax denominator from the very P values the tensor core
 // used; the output is O[:, :56] / O[:, 56]. V is read in its natural [keys][channels] layout
@@ -40,9 +44,8 @@ constexpr int OFF_Q = 0;                         // Q_A, Q_B
 constexpr int OFF_KV = OFF_Q + 2 * Q_BYTES;
 constexpr int OFF_BAR = OFF_KV + KV_STAGES * KV_BYTES;
 constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;
-constexpr uint32_t TMEM_COLS = 512;  // S_A, S_B [0,256), O_A, O_B [256,384), P_A, P_B [384,512)
-constexpr uint32_t O_COL = 256;
-constexpr uint32_t P_COL = 384;      // P as bf16 pairs: 128 keys in 64 columns per tile
+constexpr uint32_t TMEM_COLS = 512;  // S/P buffers at 0, 128, 256; O_A, O_B at 384, 448
+constexpr uint32_t O_COL = 384;      // P as bf16 pairs: 128 keys in the first 64 columns
 constexpr float RESCALE_LOG2 = 8.f;              // raise the running max past 2^8 only
 
 struct AParams {
@@ -95,12 +98,10 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;
   uint64_t* kv_empty = kv_full + KV_STAGES;
-  uint64_t* s_full = kv_empty + KV_STAGES;  // [2]: one per query tile
-  uint64_t* s_free = s_full + 2;
-  uint64_t* p_full = s_free + 2;
-  uint64_t* p_free = p_full + 2;
-  uint64_t* o_done = p_free + 2;
-  uint64_t* drain = o_done + 2;
+  uint64_t* s_full = kv_empty + KV_STAGES;  // [3]: per S/P buffer
+  uint64_t* p_full = s_full + 3;            // [3]
+  uint64_t* o_done = p_full + 3;            // [tile][key-tile parity]: that P V has completed
+  uint64_t* drain = o_done + 4;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -115,13 +116,11 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
-    for (int t = 0; t < 2; ++t) {
-      mbar_init(&s_full[t], 1);
-      mbar_init(&s_free[t], 128);
-      mbar_init(&p_full[t], 128);
-      mbar_init(&p_free[t], 1);
-      mbar_init(&o_done[t], 1);
+    for (int i = 0; i < 3; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 128);
     }
+    for (int i = 0; i < 4; ++i) mbar_init(&o_done[i], 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -179,6 +178,40 @@ __global__ void __launch_bounds__(320, 1)
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, KT);
       constexpr uint32_t IDESC_O = idesc_bf16_f32(128, 64) | IDESC_B_MN_MAJOR;
       const uint64_t desc0 = smem_desc_sw128(smem_u32(smem));
+      // S of slot k = 2j + t into buffer k mod 3
+      auto issue_s = [&](int j, int t) {
+        const int k = 2 * j + t, buf = k % 3;
+        const uint64_t kdesc = desc_advance(desc0, (uint32_t)(OFF_KV + (j % KV_STAGES) * KV_BYTES));
+        const uint64_t qdesc = desc_advance(desc0, (uint32_t)(OFF_Q + t * Q_BYTES));
+        const uint32_t sd = tmem + (uint32_t)(128 * buf);
+        tc_mma_bf16_k<false>(sd, qdesc, kdesc, IDESC_S);
+#pragma unroll
+        for (int kk = 1; kk < 4; ++kk)
+          tc_mma_bf16_k<true>(sd, desc_advance(qdesc, 32u * kk), desc_advance(kdesc, 32u * kk),
+                              IDESC_S);
+        tc_commit(&s_full[buf]);
+      };
+      // P of slot k = 2j + t (buffer k mod 3) times V_j into O_t, once the weights are in
+      auto issue_pv = [&](int j, int t) -> bool {
+        const int k = 2 * j + t, buf = k % 3;
+        if (!mbar_wait(&p_full[buf], (uint32_t)((k / 3) & 1), p.limit_ns, p.status, abort_flag))
+          return false;
+        tc_fence_after();
+        const uint64_t vdesc =
+            smem_desc_sw128_mn64(smem_u32(smem + OFF_KV + (j % KV_STAGES) * KV_BYTES + K_BYTES));
+        const uint32_t pa = tmem + (uint32_t)(128 * buf);
+        const uint32_t od = tmem + O_COL + (uint32_t)(t * 64);
+        if (j == 0)
+          tc_mma_bf16_ta<false>(od, pa, vdesc, IDESC_O);
+        else
+          tc_mma_bf16_ta<true>(od, pa, vdesc, IDESC_O);
+        // K step kk covers keys 16kk..16kk+15: two 8-row groups of the swizzled V tile
+#pragma unroll
+        for (int kk = 1; kk < 8; ++kk)
+          tc_mma_bf16_ta<true>(od, pa + 8u * kk, desc_advance(vdesc, 2048u * kk), IDESC_O);
+        tc_commit(&o_done[2 * t + (j & 1)]);
+        return true;
+      };
       bool ok = mbar_wait(q_full, 0, p.limit_ns, p.status, abort_flag);
       tc_fence_after();
       for (int j = 0; ok && j <= n_tiles; ++j) {
@@ -189,49 +222,20 @@ __global__ void __launch_bounds__(320, 1)
             ok = false;
             break;
           }
-          const uint64_t kdesc = desc_advance(desc0, (uint32_t)(OFF_KV + s * KV_BYTES));
-          for (int t = 0; t < 2 && ok; ++t) {
-            // the softmax of tile t has read S_t(j-1) out of TMEM
-            if (j >= 1 && !mbar_wait(&s_free[t], (uint32_t)((j - 1) & 1), p.limit_ns, p.status,
-                                     abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint64_t qdesc = desc_advance(desc0, (uint32_t)(OFF_Q + t * Q_BYTES));
-            tc_mma_bf16_k<false>(tmem + (uint32_t)(t * KT), qdesc, kdesc, IDESC_S);
-#pragma unroll
-            for (int kk = 1; kk < 4; ++kk)
-              tc_mma_bf16_k<true>(tmem + (uint32_t)(t * KT), desc_advance(qdesc, 32u * kk),
-                                  desc_advance(kdesc, 32u * kk), IDESC_S);
-            tc_commit(&s_full[t]);
-          }
-          if (!ok) break;
+          tc_fence_after();
+          issue_s(j, 0);  // buffer of slot 2j - 3 (P_B(j-2) V issued last iteration)
         }
+        if (j >= 1 && !issue_pv(j - 1, 0)) {
+          ok = false;
+          break;
+        }
+        if (j < n_tiles) issue_s(j, 1);  // buffer of slot 2j - 2 (P_A(j-1) V just issued)
         if (j >= 1) {
-          const int jj = j - 1, s2 = jj % KV_STAGES;
-          const uint64_t vdesc = smem_desc_sw128_mn64(smem_u32(smem + OFF_KV + s2 * KV_BYTES + K_BYTES));
-          for (int t = 0; t < 2 && ok; ++t) {
-            if (!mbar_wait(&p_full[t], (uint32_t)(jj & 1), p.limit_ns, p.status, abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t pa = tmem + P_COL + (uint32_t)(t * 64);  // P_t in TMEM
-            const uint32_t od = tmem + O_COL + (uint32_t)(t * 64);
-            if (jj == 0)
-              tc_mma_bf16_ta<false>(od, pa, vdesc, IDESC_O);
-            else
-              tc_mma_bf16_ta<true>(od, pa, vdesc, IDESC_O);
-            // K step kk covers keys 16kk..16kk+15: two 8-row groups of the swizzled V tile
-#pragma unroll
-            for (int kk = 1; kk < 8; ++kk)
-              tc_mma_bf16_ta<true>(od, pa + 8u * kk, desc_advance(vdesc, 2048u * kk), IDESC_O);
-            tc_commit(&o_done[t]);
-            tc_commit(&p_free[t]);
+          if (!issue_pv(j - 1, 1)) {
+            ok = false;
+            break;
           }
-          if (!ok) break;
-          tc_commit(&kv_empty[s2]);
+          tc_commit(&kv_empty[(j - 1) % KV_STAGES]);
         }
       }
       if (!ok) *abort_flag = 1;
@@ -244,14 +248,20 @@ __global__ void __launch_bounds__(320, 1)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-    const uint32_t s_col = (uint32_t)(t * KT), o_col = O_COL + (uint32_t)(t * 64);
+    const uint32_t o_col = O_COL + (uint32_t)(t * 64);
     const float sl2 = p.sl2;
     const float thr = RESCALE_LOG2 / sl2;  // in raw score units
     float m_run = -INFINITY;
     bool ok = true;
-    const uint32_t p_col = P_COL + (uint32_t)(t * 64);
+    // o_done[t][j & 1] completes once per two key tiles; waiting on key tile j-2's phase at
+    // key tile j keeps every wait at most one phase behind (P_t(j) V cannot have run yet)
+    auto wait_pv = [&](int jj) -> bool {
+      return warp_wait(&o_done[2 * t + (jj & 1)], (uint32_t)((jj >> 1) & 1), p, abort_flag);
+    };
     for (int j = 0; j < n_tiles; ++j) {
-      if (!warp_wait(&s_full[t], (uint32_t)(j & 1), p, abort_flag)) {
+      const int k = 2 * j + t, buf = k % 3;
+      const uint32_t s_col = (uint32_t)(128 * buf);
+      if (!warp_wait(&s_full[buf], (uint32_t)((k / 3) & 1), p, abort_flag)) {
         ok = false;
         break;
       }
@@ -264,8 +274,6 @@ __global__ void __launch_bounds__(320, 1)
       tc_wait_ld();
 #pragma unroll
       for (int i = 0; i < KT; ++i) asm volatile("" : "+r"(sr[i]));
-      tc_fence_before();
-      mbar_arrive(&s_free[t]);  // S_t may be overwritten from here on
       const int kv_valid = min(KT, p.Tkv - j * KT);
       if (kv_valid < KT) {  // ragged last tile: masked keys take no part
 #pragma unroll
@@ -281,8 +289,8 @@ __global__ void __launch_bounds__(320, 1)
         mx[u] = fmax3(__uint_as_float(sr[u]), __uint_as_float(sr[8 + u]),
                       __uint_as_float(sr[16 + u]));
 #pragma unroll
-        for (int k = 3; k < 15; k += 2)
-          mx[u] = fmax3(mx[u], __uint_as_float(sr[8 * k + u]), __uint_as_float(sr[8 * k + 8 + u]));
+        for (int c = 3; c < 15; c += 2)
+          mx[u] = fmax3(mx[u], __uint_as_float(sr[8 * c + u]), __uint_as_float(sr[8 * c + 8 + u]));
         mx[u] = fmaxf(mx[u], __uint_as_float(sr[120 + u]));
       }
       const float mt = fmaxf(fmax3(mx[0], mx[1], mx[2]),
@@ -295,12 +303,13 @@ __global__ void __launch_bounds__(320, 1)
         resc = j > 0;
       }
       const float ms = m_run * sl2;
-      // P_t and O_t are free once the PV of tile j-1 has completed
-      if (j >= 1 && !warp_wait(&p_free[t], (uint32_t)((j - 1) & 1), p, abort_flag)) {
+      // bookkeeping: P_t(j-2) V was issued before S_t(j), which has completed
+      if (j >= 2 && !wait_pv(j - 2)) {
         ok = false;
         break;
       }
-      // P of this row as bf16 pairs straight into TMEM (lane = row), 64 keys per store
+      // P of this row as bf16 pairs over the S columns just read (lane = row), 64 keys per
+      // store
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t pw[32];
@@ -310,10 +319,14 @@ __global__ void __launch_bounds__(320, 1)
           const float x1 = fmaf(__uint_as_float(sr[64 * h + 2 * u + 1]), sl2, -ms);
           pw[u] = pack_bf16x2_trunc(ex2_approx(x0), ex2_approx(x1));
         }
-        tc_st_32x32b_x32(lane_base + p_col + (uint32_t)(32 * h), pw);
+        tc_st_32x32b_x32(lane_base + s_col + (uint32_t)(32 * h), pw);
       }
       if (__any_sync(0xffffffffu, resc)) {
-        // O_t holds the sum through tile j-1 (its PV completed above): rescale these rows
+        // O_t holds the sum through tile j-1 once that P V has completed: rescale these rows
+        if (!wait_pv(j - 1)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         const float f = resc ? alpha : 1.f;
 #pragma unroll
@@ -332,11 +345,14 @@ __global__ void __launch_bounds__(320, 1)
       }
       tc_wait_st();  // P (and any rescaled O) written before the tensor core reads them
       tc_fence_before();
-      mbar_arrive(&p_full[t]);
+      mbar_arrive(&p_full[buf]);
     }
-    // ---- normalise and store this row: merged head layout, token j*nW + w. The PV of tile
-    // n-2 is complete (p_free above), so o_done's phase n-1 is the one pending.
-    if (ok && warp_wait(&o_done[t], (uint32_t)((n_tiles - 1) & 1), p, abort_flag)) {
+    // ---- normalise and store this row: merged head layout, token j*nW + w, once the last
+    // two P V products have completed
+    bool done = ok;
+    if (done && n_tiles >= 2) done = wait_pv(n_tiles - 2);
+    if (done) done = wait_pv(n_tiles - 1);
+    if (done) {
       tc_fence_after();
       uint32_t ov[64];
       tmem_ld32(lane_base + o_col, *reinterpret_cast<uint32_t(*)[32]>(&ov[0]));
@@ -346,7 +362,7 @@ __global__ void __launch_bounds__(320, 1)
       for (int i = 0; i < 64; ++i) asm volatile("" : "+r"(ov[i]));
       const int qrow = q0 + t * QT + r;
       if (qrow < p.Tq) {
-        const float inv = 1.f / __uint_as_float(ov[56]);  // softmax denominator (ones row of v)
+        const float inv = 1.f / __uint_as_float(ov[56]);  // softmax denominator (ones channel)
         const int h = unit % p.heads;
         const int w = (unit / p.heads) % p.nW;
         const int bimg = unit / (p.heads * p.nW);
