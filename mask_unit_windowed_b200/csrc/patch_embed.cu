@@ -3,17 +3,11 @@
 // [B, N, C]; a learned pos_embed (1, N, 112) is added; Unroll permutes the tokens).
 // Padding 3, so an img x img image gives a (img/4) x (img/4) token grid.
 //
-// bf16: an implicit GEMM on the tensor cores (mma.sync m16n8k16, fp32 accumulation): a CTA
-// holds the weight as bf16 [112][208] in shared memory and, per output row, the 7 input rows
-// its 128 output columns need (3-pixel halo, zero outside the image); each warp computes 16
-// output pixels x 112 channels over K = 196 (padded to 208) with A fragments gathered
-// straight from the staged input (the (ky, kx, c) ordering keeps every fragment pair in one
-// 4-byte word). The epilogue adds bias and pos_embed[raster token] (loaded before the MMA
-// loop) to the accumulator fragments, rounds once to bf16 and stages the rows per warp in
-// the input buffer, which the MMA no longer needs; a lane per (pixel, 56-channel half) then
-// stores the half row at its unrolled position (3 unroll levels) and, when asked, the
-// LayerNorm partial (mean, M2) of the half for block 0's norm1. 79 KB of shared memory
-// per CTA: two CTAs per SM overlap one's loads with the other's MMA.
+// bf16: an implicit GEMM on the tcgen05 tensor cores with fp32 accumulation in TMEM (see
+// patch_embed_tc_kernel below): im2col tiles built in shared memory from the NHWC image,
+// the weight TMA-loaded once per CTA, bias and pos_embed added in the epilogue with one
+// rounding to bf16, the rows stored at their unrolled positions (3 unroll levels) together
+// with the LayerNorm partials (mean, M2 per 56-channel half) for block 0's norm1.
 // fp32: the same computation in fp32 SIMT (weights fp32 [196][112] in shared memory, 56
 // accumulators per thread).
 #include "common.cuh"
@@ -105,151 +99,262 @@ __global__ void __launch_bounds__(256, 1) patch_embed_kernel(const float* __rest
 }
 
 // ---------------------------------------------------------------- bf16 tensor-core path
-constexpr int KP = 208;                 // K padded to 13 k-steps of 16
-constexpr int WPITCH = 216;             // bf16 per weight row in smem (conflict-free fragments)
-constexpr int IN_PITCH = 516;           // pixels per staged input row
-constexpr int SPITCH = 120;             // bf16 per staged output pixel (240 B: 16-byte rows)
-constexpr int MMA_ROWS = 4;             // output rows per CTA (weights loaded once)
-constexpr int IN_BYTES = KSZ * IN_PITCH * CIN * 2;
-constexpr int STG_BYTES = 8 * 16 * SPITCH * 2;  // 8 warps x 16 pixels, aliases the input rows
-constexpr int BUF_BYTES = IN_BYTES > STG_BYTES ? IN_BYTES : STG_BYTES;
-constexpr int MMA_SMEM = PATCH_CO * WPITCH * 2 + BUF_BYTES;  // 79 KB: two CTAs per SM
+// Implicit GEMM on the 5th-generation tensor cores. A tile is 128 consecutive output
+// pixels of one output row (oy, ox0 .. ox0 + 127) of one image:
+//   A [128 pixels][K = 208]   im2col rows, k = (ky * 7 + kx) * 4 + c for k < 196, zero for
+//                             196 <= k < 208; built in shared memory by four warps, one
+//                             pixel row per thread, in the 128-byte-swizzled K-major layout
+//                             (four 64-column blocks); double-buffered
+//   W [112][208]              the packed bf16 weight, TMA-loaded once per CTA
+//   D [128][112] fp32         13 tcgen05.mma (M = 128, N = 112, K = 16) into one of two TMEM
+//                             accumulators
+// The epilogue warps (TMEM lane = pixel) add the bias and pos_embed[raster token] in fp32,
+// round once to bf16, store the two 56-channel halves at the pixel's unrolled position
+// (3 unroll levels) and, when asked, the LayerNorm partial (mean, M2) of each half for
+// block 0's norm1.
+// Roles (320 threads, persistent CTAs, tiles strided over the grid): warp 0 weight TMA,
+// warp 1 TMEM owner and MMA issuer, warps 2-5 im2col, warps 6-9 epilogue.
+constexpr int KP = 208;                       // K padded to 13 steps of 16
+constexpr int PE_KB = 4;                      // 64-column k-blocks of A and W
+constexpr int PE_A_BYTES = PE_KB * 128 * 128; // one A buffer (64 KB)
+constexpr int PE_W_BYTES = PE_KB * PATCH_CO * 128;  // 4 x 14 KB
+constexpr int PE_OFF_A = 0;
+constexpr int PE_OFF_W = 2 * PE_A_BYTES;
+constexpr int PE_OFF_BIAS = PE_OFF_W + PE_W_BYTES;
+constexpr int PE_OFF_BAR = PE_OFF_BIAS + PATCH_CO * 4;
+constexpr int PE_SMEM = PE_OFF_BAR + 128 + 1024;
+static_assert((PATCH_CO * 128) % 1024 == 0, "W k-blocks keep 1024-byte alignment");
 
-__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1,
-                                               uint32_t a2, uint32_t a3, uint32_t b0,
-                                               uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
+struct PeParams {
+  const bf16* img;
+  const float* bias;
+  const bf16* pos;
+  bf16* out;
+  float2* stats_out;
+  int img_side, G, M, segs, tiles;
+  uint64_t limit_ns;
+  unsigned int* status;
+};
 
-// element offset of (k, local pixel px) in the staged input [ky][x][c]; k even
-__device__ __forceinline__ int in_off(int k, int px) {
-  const int ky = k / 28, rem = k - 28 * ky;
-  return (ky * IN_PITCH + 4 * px + (rem >> 2)) * CIN + (rem & 3);
-}
+__global__ void __launch_bounds__(320, 1)
+    patch_embed_tc_kernel(const __grid_constant__ CUtensorMap tmW, const PeParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  uint8_t* smem = smem_raw + pad;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + PE_OFF_BAR);
+  uint64_t* w_full = bars;
+  uint64_t* a_full = bars + 1;     // [2] count 128: the im2col warps wrote buffer b
+  uint64_t* a_empty = a_full + 2;  // [2] the MMAs reading buffer b completed
+  uint64_t* acc_full = a_empty + 2;
+  uint64_t* acc_empty = acc_full + 2;  // [2] count 128: the epilogue read accumulator a
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* s_bias = reinterpret_cast<float*>(smem + PE_OFF_BIAS);
 
-__global__ void __launch_bounds__(256, 2) patch_embed_mma_kernel(
-    const bf16* __restrict__ img, const bf16* __restrict__ w16, const float* __restrict__ bias,
-    const bf16* __restrict__ pos, bf16* __restrict__ out, float2* __restrict__ stats_out,
-    int img_side) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_local = (int)blockIdx.x < p.tiles
+                          ? (p.tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(w_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&a_full[i], 128);
+      mbar_init(&a_empty[i], 1);
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmW);
+  }
+  if (warp == 1) {
+    tc_alloc(tmem_slot, 256);
+    tc_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
   griddep_wait();  // everything below reads or writes data of earlier kernels
   griddep_launch_dependents();
-  extern __shared__ __align__(16) uint8_t smem_pe[];
-  bf16* sW = reinterpret_cast<bf16*>(smem_pe);  // [112][WPITCH]
-  bf16* sIn = sW + PATCH_CO * WPITCH;           // [7][IN_PITCH][4] during the MMA
-  const int G = img_side / 4;
-  const int M = G / 8;
-  const int N = G * G;
-  const int b = blockIdx.z;
-  const int ox0 = blockIdx.x * SEG;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g = lane >> 2, t4 = lane & 3;
-  // after the MMA the input rows are dead: each warp stages its 16 pixels x 112 channels
-  // there, rounded to bf16 ([16][SPITCH])
-  bf16* so = sIn + warp * 16 * SPITCH;
 
-  for (int i = tid; i < PATCH_CO * (KP / 8); i += 256) {
-    const int co = i / (KP / 8), c8 = i - co * (KP / 8);
-    *reinterpret_cast<uint4*>(sW + co * WPITCH + c8 * 8) =
-        __ldg(reinterpret_cast<const uint4*>(w16 + co * KP) + c8);
-  }
-  for (int rr = 0; rr < MMA_ROWS; ++rr) {
-    const int oy = blockIdx.y * MMA_ROWS + rr;
-    if (oy >= G) break;
-    __syncthreads();  // the previous row's staged outputs have been copied out
-    for (int i = tid; i < KSZ * XSPAN; i += 256) {
-      const int ky = i / XSPAN, xi = i - ky * XSPAN;
-      const int iy = 4 * oy - 3 + ky, ix = 4 * ox0 - 3 + xi;
-      uint2 v = make_uint2(0u, 0u);
-      if (iy >= 0 && iy < img_side && ix >= 0 && ix < img_side)
-        v = __ldg(reinterpret_cast<const uint2*>(img + (((long long)b * img_side + iy) * img_side + ix) * CIN));
-      *reinterpret_cast<uint2*>(sIn + (ky * IN_PITCH + xi) * CIN) = v;
+  // the tile's image, output row and first output column
+  auto tile_pos = [&](int tile, int& b, int& oy, int& ox0) {
+    const int seg = tile % p.segs, row = tile / p.segs;
+    b = row / p.G;
+    oy = row - b * p.G;
+    ox0 = seg * 128;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ weights (once)
+    if (lane == 0 && n_local > 0) {
+      mbar_arrive_expect_tx(w_full, PE_W_BYTES);
+      for (int kb = 0; kb < PE_KB; ++kb)
+        tma_load_2d(smem + PE_OFF_W + kb * PATCH_CO * 128, &tmW, w_full, kb * 64, 0);
+      mbar_wait(w_full, 0, p.limit_ns, p.status);  // landed before the CTA can exit
     }
-    // pos_embed of this lane's two pixels (rows g, g + 8 of the warp's 16) and 28 channels
-    // (8 nt + 2 t4, +1), in flight while the MMA runs
-    uint32_t pw[2][14];
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && n_local > 0) {
+      constexpr uint32_t IDESC = idesc_bf16_f32(128, PATCH_CO);
+      bool ok = mbar_wait(w_full, 0, p.limit_ns, p.status, abort_flag);
+      const uint64_t adesc0 = smem_desc_sw128(smem_u32(smem + PE_OFF_A));
+      const uint64_t wdesc0 = smem_desc_sw128(smem_u32(smem + PE_OFF_W));
+      for (int t = 0; ok && t < n_local; ++t) {
+        const int b = t & 1;
+        if (!mbar_wait(&a_full[b], (uint32_t)((t >> 1) & 1), p.limit_ns, p.status, abort_flag) ||
+            !mbar_wait(&acc_empty[b], (uint32_t)(((t >> 1) & 1) ^ 1), p.limit_ns, p.status,
+                       abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(128 * b);
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int ox = ox0 + warp * 16 + g + 8 * h;
-      const bf16* pr = pos + (long long)(oy * G + (ox < G ? ox : 0)) * PATCH_CO + 2 * t4;
-#pragma unroll
-      for (int nt = 0; nt < 14; ++nt)
-        pw[h][nt] = __ldg(reinterpret_cast<const unsigned int*>(pr + nt * 8));
-    }
-    __syncthreads();
-    const int px = warp * 16 + g;  // fragment rows g and g + 8
-    float acc[14][4];
-#pragma unroll
-    for (int nt = 0; nt < 14; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-#pragma unroll 1
-    for (int ks = 0; ks < KP / 16; ++ks) {
-      const int kA = 16 * ks + 2 * t4, kB = kA + 8;
-      uint32_t a0 = 0, a1 = 0, a2 = 0, a3 = 0;
-      if (kA < PATCH_K) {
-        a0 = *reinterpret_cast<const uint32_t*>(sIn + in_off(kA, px));
-        a1 = *reinterpret_cast<const uint32_t*>(sIn + in_off(kA, px + 8));
+        for (int st = 0; st < KP / 16; ++st) {
+          const int kb = st >> 2, kk = st & 3;
+          const uint64_t ad = desc_advance(adesc0, (uint32_t)(b * PE_A_BYTES + kb * 16384 + 32 * kk));
+          const uint64_t wd = desc_advance(wdesc0, (uint32_t)(kb * PATCH_CO * 128 + 32 * kk));
+          if (st == 0)
+            tc_mma_bf16_k<false>(d, ad, wd, IDESC);
+          else
+            tc_mma_bf16_k<true>(d, ad, wd, IDESC);
+        }
+        tc_commit(&a_empty[b]);
+        tc_commit(&acc_full[b]);
       }
-      if (kB < PATCH_K) {
-        a2 = *reinterpret_cast<const uint32_t*>(sIn + in_off(kB, px));
-        a3 = *reinterpret_cast<const uint32_t*>(sIn + in_off(kB, px + 8));
-      }
-#pragma unroll
-      for (int nt = 0; nt < 14; ++nt) {
-        const bf16* wr = sW + (nt * 8 + g) * WPITCH;
-        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(wr + kA);
-        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(wr + kB);
-        mma_bf16_16816(acc[nt], a0, a1, a2, a3, b0, b1);
-      }
+      if (!ok) *abort_flag = 1;
+      tc_commit(drain);
+      mbar_wait(drain, 0, p.limit_ns, p.status);
     }
-    __syncthreads();  // every warp is done reading the input rows
-    // (acc + bias) + pos_embed, rounded once to bf16, staged per pixel row
-#pragma unroll
-    for (int nt = 0; nt < 14; ++nt) {
-      const int co = nt * 8 + 2 * t4;
-      const float b0 = __ldg(bias + co), b1 = __ldg(bias + co + 1);
-      *reinterpret_cast<uint32_t*>(so + g * SPITCH + co) =
-          pack_bf16x2((acc[nt][0] + b0) + bf16_lo(pw[0][nt]), (acc[nt][1] + b1) + bf16_hi(pw[0][nt]));
-      *reinterpret_cast<uint32_t*>(so + (g + 8) * SPITCH + co) =
-          pack_bf16x2((acc[nt][2] + b0) + bf16_lo(pw[1][nt]), (acc[nt][3] + b1) + bf16_hi(pw[1][nt]));
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ im2col (one pixel per thread)
+    const int px = (warp - 2) * 32 + lane;  // pixel of the tile = row of A
+    const uint32_t sw = (uint32_t)(px & 7);
+    // the padding columns 196..207 (k-block 3, 16-byte chunks 0..1 after the first 4
+    // elements) stay zero: the weight is zero there too, but stale shared memory could hold
+    // a NaN pattern, and 0 * NaN would not vanish
+    for (int b = 0; b < 2; ++b) {
+      uint8_t* row = smem + PE_OFF_A + b * PE_A_BYTES + 3 * 16384 + px * 128;
+      *reinterpret_cast<uint2*>(row + ((0u ^ sw) << 4) + 8) = make_uint2(0u, 0u);
+      *reinterpret_cast<uint4*>(row + ((1u ^ sw) << 4)) = make_uint4(0u, 0u, 0u, 0u);
     }
-    __syncwarp();
-    // lane = (pixel, half): the half row to its unrolled position, LayerNorm partial
-    {
-      const int lp = lane & 15, half = lane >> 4;
-      const int ox = ox0 + warp * 16 + lp;
-      if (ox < G) {
-        const int u = unrolled_of_spatial(oy, ox, 3, M);
-        const uint4* src = reinterpret_cast<const uint4*>(so + lp * SPITCH + half * 56);
-        uint4* dst = reinterpret_cast<uint4*>(out + ((long long)b * N + u) * PATCH_CO + half * 56);
+    for (int t = 0; t < n_local; ++t) {
+      const int tile = (int)blockIdx.x + t * (int)gridDim.x;
+      const int b = t & 1;
+      if (!warp_wait(&a_empty[b], (uint32_t)(((t >> 1) & 1) ^ 1), p.limit_ns, p.status,
+                     abort_flag))
+        break;
+      int bi, oy, ox0;
+      tile_pos(tile, bi, oy, ox0);
+      const int ix0 = 4 * (ox0 + px) - 3;  // first image column of this pixel's window
+      uint8_t* arow = smem + PE_OFF_A + b * PE_A_BYTES + px * 128;
+      const bf16* ib = p.img + (long long)bi * p.img_side * p.img_side * CIN;
+#pragma unroll
+      for (int ky = 0; ky < KSZ; ++ky) {
+        const int iy = 4 * oy - 3 + ky;
+        const bool row_in = iy >= 0 && iy < p.img_side;
+        const bf16* irow = ib + (long long)(row_in ? iy : 0) * p.img_side * CIN;
+#pragma unroll
+        for (int kx = 0; kx < KSZ; ++kx) {
+          const int ix = ix0 + kx;
+          uint2 v = make_uint2(0u, 0u);
+          if (row_in && ix >= 0 && ix < p.img_side)
+            v = __ldg(reinterpret_cast<const uint2*>(irow + (long long)ix * CIN));
+          const int k = (ky * KSZ + kx) * CIN;             // compile-time after unrolling
+          const int kb = k >> 6, kc = k & 63;
+          *reinterpret_cast<uint2*>(arow + kb * 16384 + ((((uint32_t)(kc >> 3)) ^ sw) << 4) +
+                                    (kc & 7) * 2) = v;
+        }
+      }
+      fence_proxy_async_smem();  // generic-proxy writes before the tensor core reads them
+      mbar_arrive(&a_full[b]);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (pixel per thread)
+    const int quarter = warp & 3;
+    const int px = quarter * 32 + lane;
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    for (int i = threadIdx.x - 192; i < PATCH_CO; i += 128) s_bias[i] = __ldg(p.bias + i);
+    named_bar_sync(1, 128);
+    const int N = p.G * p.G;
+    for (int t = 0; t < n_local; ++t) {
+      const int tile = (int)blockIdx.x + t * (int)gridDim.x;
+      const int b = t & 1;
+      int bi, oy, ox0;
+      tile_pos(tile, bi, oy, ox0);
+      const int ox = ox0 + px;
+      const bool valid = ox < p.G;
+      // pos_embed of this pixel (raster token), in flight while the MMA runs
+      uint4 pos4[14];
+      const uint4* pr = reinterpret_cast<const uint4*>(
+          p.pos + (long long)(oy * p.G + (valid ? ox : 0)) * PATCH_CO);
+#pragma unroll
+      for (int i = 0; i < 14; ++i) pos4[i] = __ldg(pr + i);
+      if (!warp_wait(&acc_full[b], (uint32_t)((t >> 1) & 1), p.limit_ns, p.status, abort_flag))
+        break;
+      tc_fence_after();
+      const int u = unrolled_of_spatial(oy, valid ? ox : 0, 3, p.M);
+      bf16* dst = p.out + ((long long)bi * N + u) * PATCH_CO;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t r[56];
+        tmem_load<56>(lane_base + (uint32_t)(128 * b + 56 * half), r);
+        if (half == 1) {
+          tc_fence_before();
+          mbar_arrive(&acc_empty[b]);  // accumulator b may take tile t + 2
+        }
         float vals[56];
+        uint4 pk[7];
 #pragma unroll
         for (int c8 = 0; c8 < 7; ++c8) {
-          const uint4 pk = src[c8];
-          dst[c8] = pk;
-          vals[8 * c8 + 0] = bf16_lo(pk.x);
-          vals[8 * c8 + 1] = bf16_hi(pk.x);
-          vals[8 * c8 + 2] = bf16_lo(pk.y);
-          vals[8 * c8 + 3] = bf16_hi(pk.y);
-          vals[8 * c8 + 4] = bf16_lo(pk.z);
-          vals[8 * c8 + 5] = bf16_hi(pk.z);
-          vals[8 * c8 + 6] = bf16_lo(pk.w);
-          vals[8 * c8 + 7] = bf16_hi(pk.w);
+          const uint4 pp = pos4[half * 7 + c8];
+          const uint32_t pw[4] = {pp.x, pp.y, pp.z, pp.w};
+          float f[8];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = half * 56 + c8 * 8 + 2 * e;
+            f[2 * e] = (__uint_as_float(r[c8 * 8 + 2 * e]) + s_bias[c]) + bf16_lo(pw[e]);
+            f[2 * e + 1] = (__uint_as_float(r[c8 * 8 + 2 * e + 1]) + s_bias[c + 1]) + bf16_hi(pw[e]);
+          }
+          pk[c8] = pack8(f);
+          vals[8 * c8 + 0] = bf16_lo(pk[c8].x);
+          vals[8 * c8 + 1] = bf16_hi(pk[c8].x);
+          vals[8 * c8 + 2] = bf16_lo(pk[c8].y);
+          vals[8 * c8 + 3] = bf16_hi(pk[c8].y);
+          vals[8 * c8 + 4] = bf16_lo(pk[c8].z);
+          vals[8 * c8 + 5] = bf16_hi(pk[c8].z);
+          vals[8 * c8 + 6] = bf16_lo(pk[c8].w);
+          vals[8 * c8 + 7] = bf16_hi(pk[c8].w);
         }
-        if (stats_out != nullptr) {
-          float s = 0.f;
+        if (valid) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + half * 56);
 #pragma unroll
-          for (int j = 0; j < 56; ++j) s += vals[j];
-          const float mean = s * (1.f / 56.f);
-          float m2 = 0.f;
+          for (int c8 = 0; c8 < 7; ++c8) d4[c8] = pk[c8];
+          if (p.stats_out != nullptr) {
+            float sm = 0.f;
 #pragma unroll
-          for (int j = 0; j < 56; ++j) m2 = fmaf(vals[j] - mean, vals[j] - mean, m2);
-          stats_out[((long long)b * N + u) * 2 + half] = make_float2(mean, m2);
+            for (int j = 0; j < 56; ++j) sm += vals[j];
+            const float mean = sm * (1.f / 56.f);
+            float m2 = 0.f;
+#pragma unroll
+            for (int j = 0; j < 56; ++j) m2 = fmaf(vals[j] - mean, vals[j] - mean, m2);
+            p.stats_out[((long long)bi * N + u) * 2 + half] = make_float2(mean, m2);
+          }
         }
       }
     }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tc_dealloc(tmem, 256);
   }
 }
 
@@ -265,13 +370,32 @@ hiera_status launch_patch_embed(const void* img, const void* packed, const void*
   const bf16* w16 = reinterpret_cast<const bf16*>(pk + PATCH_OFF_W16);
   profile_mark(K_PATCH_EMBED, stream);
   if (dtype_bf16) {
-    dim3 grid((G + SEG - 1) / SEG, (G + MMA_ROWS - 1) / MMA_ROWS, B);
-    if (grid.y > 65535 || grid.z > 65535) return HIERA_ERR_SHAPE;
-    if (!ensure_smem_attr(reinterpret_cast<const void*>(patch_embed_mma_kernel), MMA_SMEM))
+    CUtensorMap tmW;
+    {
+      cuuint64_t dims[2] = {(cuuint64_t)PATCH_KP, (cuuint64_t)PATCH_CO};
+      cuuint64_t str[1] = {(cuuint64_t)PATCH_KP * 2};
+      cuuint32_t box[2] = {64, (cuuint32_t)PATCH_CO};
+      if (!encode_tmap_bf16_sw128(&tmW, w16, 2, dims, str, box)) return HIERA_ERR_CUDA;
+    }
+    PeParams pp;
+    pp.img = static_cast<const bf16*>(img);
+    pp.bias = bias;
+    pp.pos = static_cast<const bf16*>(pos);
+    pp.out = static_cast<bf16*>(out);
+    pp.stats_out = stats_out;
+    pp.img_side = img_side;
+    pp.G = G;
+    pp.M = G / 8;
+    pp.segs = (G + 127) / 128;
+    const long long tiles = (long long)B * G * pp.segs;
+    if (tiles > (1ll << 30)) return HIERA_ERR_SHAPE;
+    pp.tiles = (int)tiles;
+    pp.limit_ns = g_wait_limit_ns();
+    pp.status = g_status_ptr();
+    if (!ensure_smem_attr(reinterpret_cast<const void*>(patch_embed_tc_kernel), PE_SMEM))
       return HIERA_ERR_CUDA;
-    launch_k(patch_embed_mma_kernel, grid, dim3(256), MMA_SMEM, stream,
-             static_cast<const bf16*>(img), w16, bias, static_cast<const bf16*>(pos),
-             static_cast<bf16*>(out), stats_out, img_side);
+    const int grid = (int)(tiles < g_num_sms() ? tiles : g_num_sms());
+    launch_k(patch_embed_tc_kernel, dim3(grid), dim3(320), PE_SMEM, stream, tmW, pp);
   } else {
     dim3 grid((G + SEG - 1) / SEG, (G + ROWS - 1) / ROWS, B);
     if (grid.y > 65535 || grid.z > 65535) return HIERA_ERR_SHAPE;
