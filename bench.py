@@ -79,10 +79,11 @@ def reroll_bytes(img: int, B: int):
     return [2 * 2 * B * (G0 >> s) ** 2 * STAGE_DIMS[s] for s in range(4)]
 
 
-def launch_flops(img: int, B: int, fused_mlp: bool = True):
+def launch_flops(img: int, B: int, fused_mlp: bool = True, fused_attn: bool = True):
     """Algorithmic FLOPs of every library launch of one backbone forward, in launch order
     (head_dim 56, not the padded 64). Returns list of (kind-class, flops). With fused_mlp,
-    the MLPs of dims 112 and 224 are one launch (fc1 + fc2 FLOPs)."""
+    the MLPs of dims 112 and 224 are one launch (fc1 + fc2 FLOPs); with fused_attn, the
+    stage-0 blocks' qkv, attention and proj are one launch (class attn_block)."""
     G0 = img // 4
     out = [("patch_embed", 2.0 * B * G0 * G0 * 112 * 196)]
     prev = STAGE_DIMS[0]
@@ -102,9 +103,15 @@ def launch_flops(img: int, B: int, fused_mlp: bool = True):
             tkv = n_in // nW
             tq = tkv // (4 if trans else 1)
             n1 = 3 * d + (d if trans else 0)
-            out.append(("gemm", 2.0 * B * n_in * d_in * n1))
-            out.append(("attention", 4.0 * B * STAGE_HEADS[s] * nW * tq * tkv * HD))
-            out.append(("gemm", 2.0 * B * nq * d * d))
+            qkv = 2.0 * B * n_in * d_in * n1
+            attn = 4.0 * B * STAGE_HEADS[s] * nW * tq * tkv * HD
+            proj = 2.0 * B * nq * d * d
+            if fused_attn and s == 0 and nW % 2 == 0:
+                out.append(("attn_block", qkv + attn + proj))
+            else:
+                out.append(("gemm", qkv))
+                out.append(("attention", attn))
+                out.append(("gemm", proj))
             if fused_mlp and d in (112, 224):
                 out.append(("gemm", 4.0 * B * nq * d * 4 * d))
             else:
@@ -120,7 +127,9 @@ def launch_flops(img: int, B: int, fused_mlp: bool = True):
 KIND_CLASS = {"patch_embed": "patch_embed", "unroll_reroll": "unroll_reroll",
               "gemm_qkv_lnfold": "gemm", "gemm_fc1_lnfold_gelu": "gemm",
               "gemm_bias_residual": "gemm", "attention_window": "attention",
-              "attention_tcgen05": "attention", "mlp_fused": "gemm"}
+              "attention_tcgen05": "attention", "mlp_fused": "gemm",
+              "attention_block_fused": "attn_block"}
+TENSOR_CLASSES = ("gemm", "attention", "attn_block")
 
 KIND_DESCRIPTION = {
     "gemm_qkv_lnfold": "tcgen05 GEMM: norm1 folded, qkv (+ transition proj) with window scatter",
@@ -129,6 +138,8 @@ KIND_DESCRIPTION = {
     "mlp_fused": "tcgen05 fused MLP (norm2, fc1, GELU, fc2, residual)",
     "attention_tcgen05": "tcgen05 attention, 128-key tiles (global attention)",
     "attention_window": "tcgen05 attention, several mask-unit windows per tile",
+    "attention_block_fused": "stage-0 attention half in one kernel (norm1, qkv, windowed "
+                             "attention, proj, residual; tcgen05)",
 }
 
 
@@ -336,6 +347,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     dev = torch.device("cuda", local_rank)
     hb.set_option(hb.OPT_FUSED_MLP, 1 if args.mlp == "fused" else 0)
     hb.set_option(hb.OPT_PDL, 1 if args.pdl == "on" else 0)
+    hb.set_option(hb.OPT_FUSED_ATTN, 1 if args.attn == "fused" else 0)
     hbm_gbs, tf_burst, tf_sust, peak_src = peaks()
     B = args.batch
 
@@ -410,7 +422,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             per_launch = [(n, ms) for n, ms in d] if per_launch is None else \
                 [(n, a + ms) for (n, a), (_, ms) in zip(per_launch, d)]
     per_launch = [(n, ms / reps) for n, ms in per_launch]
-    flops = launch_flops(IMG, B, fused_mlp=hb.get_option(hb.OPT_FUSED_MLP) == 1)
+    flops = launch_flops(IMG, B, fused_mlp=hb.get_option(hb.OPT_FUSED_MLP) == 1,
+                         fused_attn=hb.get_option(hb.OPT_FUSED_ATTN) == 1)
     if len(flops) != len(per_launch) or any(KIND_CLASS.get(n) != c for (n, _), (c, _) in
                                             zip(per_launch, flops)):
         raise RuntimeError("the launch sequence differs from the bench's work model")
@@ -431,11 +444,11 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     for e in shapes.values():
         e["share"] = e["ms"] / step_ms_prof if step_ms_prof > 0 else None
     # dominant kernel: the tensor-core launch shape with the largest share of the forward
-    dom_key = max((k for k, e in shapes.items() if e["class"] in ("gemm", "attention")),
+    dom_key = max((k for k, e in shapes.items() if e["class"] in TENSOR_CLASSES),
                   key=lambda k: shapes[k]["ms"])
     dom = shapes[dom_key]
     traffic = DRAM_BYTES_PER_LAUNCH.get(dom_key)
-    attn_gemm_gflop = sum(fl for c, fl in flops if c in ("gemm", "attention")) / 1e9
+    attn_gemm_gflop = sum(fl for c, fl in flops if c in TENSOR_CLASSES) / 1e9
     roofline = {"bound": "tensor", "achieved": dom["tflops"], "peak": tf_burst,
                 "unit": "TFLOP/s", "frac": dom["tflops"] / tf_burst, "traffic": traffic,
                 "kernel": dom_key[0], "kernel_description": KIND_DESCRIPTION.get(dom_key[0]),
@@ -566,7 +579,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                    "l2": "flushed before every step (256 MiB write); within a step each "
                          "forward's working set (138 MB of weights + activations) exceeds L2",
                    "timing": "CUDA-graph replay of the library launches, per-step CUDA events",
-                   "mlp": args.mlp, "pdl": args.pdl},
+                   "mlp": args.mlp, "pdl": args.pdl, "attn": args.attn},
         "ms_per_forward": ms_per_forward,
         "timed_seconds": total_ms / 1e3,
         "tflops": gflop_per_image * images / (total_ms * 1e-3) * 1e-3,
@@ -611,6 +624,9 @@ def main():
                     help="stage-0/1 MLPs as one fused kernel (default) or two GEMMs")
     ap.add_argument("--pdl", choices=["on", "off"], default="on",
                     help="programmatic dependent launch between the library's kernels")
+    ap.add_argument("--attn", choices=["fused", "unfused"], default="fused",
+                    help="stage-0 attention half (norm1, qkv, attention, proj) as one kernel "
+                         "(default) or three")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

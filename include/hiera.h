@@ -315,10 +315,24 @@ HIERA_API hiera_status hiera_backbone_forward(const hiera_backbone_desc* desc, c
  *                        kernel before it; every kernel waits (griddepcontrol.wait) for
  *                        its predecessor's completion before it reads or writes any data
  *                        a previous kernel touches. 0: ordinary stream-ordered launches.
+ *   HIERA_OPT_FUSED_ATTN 1 (default): for bf16 stage-0 blocks (dim 112, 2 heads, mask-unit
+ *                        windows of 64 tokens, no pooling, an even number of windows), norm1
+ *                        + qkv + windowed attention + proj + residual run as one kernel with
+ *                        q, k, v and the attention output kept on chip (the attention half
+ *                        of the plan's HieraBlock, Sub-phase 4a item 7); workspace slots
+ *                        [0]-[3] of hiera_block_workspace_layout are then left unwritten.
+ *                        0: the separate qkv GEMM, attention and proj GEMM. The two agree
+ *                        to rounding (the fused P V product sums the window's keys in
+ *                        another order).
  * hiera_set_option returns HIERA_ERR_INVALID_ARG for an unknown option or value;
  * hiera_get_option returns the current value (0 for an unknown option).
  * -------------------------------------------------------------------------------- */
-typedef enum { HIERA_OPT_FUSED_MLP = 0, HIERA_OPT_PDL = 1, HIERA_OPT_COUNT = 2 } hiera_option;
+typedef enum {
+  HIERA_OPT_FUSED_MLP = 0,
+  HIERA_OPT_PDL = 1,
+  HIERA_OPT_FUSED_ATTN = 2,
+  HIERA_OPT_COUNT = 3
+} hiera_option;
 HIERA_API hiera_status hiera_set_option(hiera_option opt, int value);
 HIERA_API int hiera_get_option(hiera_option opt);
 

@@ -549,6 +549,7 @@ def kernel_name(kind: int) -> str:
 # ----------------------------------------------------------------------------- options
 OPT_FUSED_MLP = 0
 OPT_PDL = 1
+OPT_FUSED_ATTN = 2
 
 
 def set_option(opt: int, value: int):
@@ -578,6 +579,13 @@ class option:
 def fused_mlp(enabled: bool) -> option:
     """Run the block MLPs fused (True, the default) or as two GEMMs."""
     return option(OPT_FUSED_MLP, bool(enabled))
+
+
+def fused_attention(enabled: bool) -> option:
+    """Run the stage-0 blocks' attention half (norm1, qkv, windowed attention, proj,
+    residual) as one kernel (True, the default) or as the separate kernels, which also write
+    q, k, v and the attention output to the workspace."""
+    return option(OPT_FUSED_ATTN, bool(enabled))
 
 
 def pdl(enabled: bool) -> option:

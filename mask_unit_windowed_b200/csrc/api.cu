@@ -219,21 +219,15 @@ bool weights_aligned(const hiera_block_weights* w) {
   return true;
 }
 
-// stats_x: partial (mean, M2) of x's rows from x's producer ([rows][parts_x]), or nullptr
-// to compute them here; stats_y: where to write y's partials for the next LayerNorm
-// ([qrows][store_stats_parts(d_out)]), or nullptr.
-hiera_status forward_bf16(const Geom& g, const uint8_t* packed, const void* x, void* y,
-                          uint8_t* ws, cudaStream_t st, const float2* stats_x = nullptr,
-                          int parts_x = 0, float2* stats_y = nullptr) {
+// (a3-a9) norm1 + qkv (+ transition proj) with window scatter and q / r pooling, attention,
+// heads merged, proj + residual: x1 and its norm2 partials in the workspace, as separate
+// kernels (q, k, v and the attention output pass through the workspace).
+hiera_status attention_half_unfused(const Geom& g, const uint8_t* packed, const void* x,
+                                    uint8_t* ws, cudaStream_t st, const float2* stats_x,
+                                    int parts_x, int parts_out) {
   const PackLayout P = pack_layout(g);
   const WsLayout W = ws_layout(g);
   const long long rows = (long long)g.B * g.tokens, qrows = (long long)g.B * g.Nq;
-  if (stats_x == nullptr) {
-    HIERA_TRY(launch_row_partials_bf16(x, (int)rows, g.d_in, (float2*)(ws + W.st1), st));
-    stats_x = (const float2*)(ws + W.st1);
-    parts_x = 1;
-  }
-  const int parts_out = store_stats_parts(g.d_out);
   // (a3-a6, a8 folded) norm1 + qkv (+ transition proj) with window scatter and q / r pooling
   TcGemmArgs a{};
   a.M = (int)rows;
@@ -285,7 +279,49 @@ hiera_status forward_bf16(const Geom& g, const uint8_t* packed, const void* x, v
   pj.ldo = g.d_out;
   pj.stats_out = ws + W.st2;
   pj.stats_out_parts = parts_out;
-  HIERA_TRY(launch_tc_gemm(EPI_STORE, pj, st));
+  return launch_tc_gemm(EPI_STORE, pj, st);
+}
+
+// stats_x: partial (mean, M2) of x's rows from x's producer ([rows][parts_x]), or nullptr
+// to compute them here; stats_y: where to write y's partials for the next LayerNorm
+// ([qrows][store_stats_parts(d_out)]), or nullptr.
+hiera_status forward_bf16(const Geom& g, const uint8_t* packed, const void* x, void* y,
+                          uint8_t* ws, cudaStream_t st, const float2* stats_x = nullptr,
+                          int parts_x = 0, float2* stats_y = nullptr) {
+  const PackLayout P = pack_layout(g);
+  const WsLayout W = ws_layout(g);
+  const long long rows = (long long)g.B * g.tokens, qrows = (long long)g.B * g.Nq;
+  if (stats_x == nullptr) {
+    HIERA_TRY(launch_row_partials_bf16(x, (int)rows, g.d_in, (float2*)(ws + W.st1), st));
+    stats_x = (const float2*)(ws + W.st1);
+    parts_x = 1;
+  }
+  const int parts_out = store_stats_parts(g.d_out);
+  const bool fused_attn =
+      g_option(HIERA_OPT_FUSED_ATTN) &&
+      attention_block_supported(g.B, g.tokens, g.d_in, g.d_out, g.heads, g.qs, g.Tkv,
+                                g.nW > 1 ? 1 : 0) &&
+      parts_out == 2;
+  if (fused_attn) {
+    // (a3-a9) norm1 + qkv + windowed attention + heads merged + proj + residual, one kernel
+    AttnBlockArgs ab{};
+    ab.B = g.B;
+    ab.tokens = g.tokens;
+    ab.x = x;
+    ab.stats_in = stats_x;
+    ab.stats_parts = parts_x;
+    ab.ln_eps = g.eps;
+    ab.w1 = packed + P.W1;
+    ab.colsum1 = (const float*)(packed + P.s1);
+    ab.colconst1 = (const float*)(packed + P.c1);
+    ab.wo = packed + P.Wo;
+    ab.bias_o = (const float*)(packed + P.bo);
+    ab.x1 = ws + W.x1;
+    ab.stats_out = ws + W.st2;
+    HIERA_TRY(launch_attention_block(ab, st));
+  } else {
+    HIERA_TRY(attention_half_unfused(g, packed, x, ws, st, stats_x, parts_x, parts_out));
+  }
   if (g_option(HIERA_OPT_FUSED_MLP) && mlp_fused_supported(g.d_out) && parts_out == 2) {
     // (a10-a12) norm2 + fc1 + GELU + fc2 + residual in one kernel, hidden kept on chip
     MlpArgs ml{};
@@ -610,7 +646,8 @@ void profile_mark(int kind, cudaStream_t stream) {
 }
 
 namespace {
-int g_options[HIERA_OPT_COUNT] = {1, 1};  // fused MLP on, programmatic dependent launch on
+int g_options[HIERA_OPT_COUNT] = {1, 1, 1};  // fused MLP, programmatic dependent launch and
+                                             // fused attention half on
 }  // namespace
 
 int g_option(int opt) { return (opt >= 0 && opt < HIERA_OPT_COUNT) ? g_options[opt] : 0; }
@@ -969,7 +1006,7 @@ const char* hiera_kernel_name(int kind) {
       "patch_embed", "unroll_reroll", "gemm_qkv_lnfold", "gemm_fc1_lnfold_gelu",
       "gemm_bias_residual", "attention_window", "f32_gemm", "f32_attention",
       "f32_row_stats", "pack", "timeout_probe", "row_stats", "attention_tcgen05",
-      "mlp_fused"};
+      "mlp_fused", "attention_block_fused"};
   return (kind >= 0 && kind < K_COUNT) ? names[kind] : "unknown";
 }
 

@@ -17,8 +17,9 @@
 // TMEM holds three S/P buffers and the two O accumulators. Slot k = 2j + t (tile t, key tile
 // j) uses buffer k mod 3, so a softmax warpgroup never waits for its own previous P V
 // product before writing the next weights: buffer k mod 3 was last used by slot k - 3 (the
-// other tile), whose P V the MMA thread issues before S of slot k (issue order S_A(j),
-// P_A(j-1) V, S_B(j), P_B(j-1) V; the tensor core executes one thread's MMAs in order).
+// other tile), whose P V the MMA thread issues right before S of slot k (issue order
+// P_A(j-1) V, S_B(j), P_B(j-1) V, S_A(j+1); the tensor core executes one thread's MMAs in
+// order).
 // head_dim 56 is padded to 64: q/k channels 56..63 are zero; v's padding channel 56 is one,
 // so column 56 of O accumulates the softmax denominator from the very P values the tensor core
 // used; the output is O[:, :56] / O[:, 56]. V is read in its natural [keys][channels] layout
@@ -212,19 +213,18 @@ __global__ void __launch_bounds__(320, 1)
         tc_commit(&o_done[2 * t + (j & 1)]);
         return true;
       };
-      bool ok = mbar_wait(q_full, 0, p.limit_ns, p.status, abort_flag);
-      tc_fence_after();
+      auto wait_kv = [&](int j) -> bool {
+        const bool r = mbar_wait(&kv_full[j % KV_STAGES], (uint32_t)((j / KV_STAGES) & 1),
+                                 p.limit_ns, p.status, abort_flag);
+        tc_fence_after();
+        return r;
+      };
+      // Issue order P_A(j-1) V, S_B(j), P_B(j-1) V, S_A(j+1): each S waits only for the P V
+      // that freed its buffer (slot k - 3), so tile A's next scores do not wait for tile B's
+      // current weights.
+      bool ok = mbar_wait(q_full, 0, p.limit_ns, p.status, abort_flag) && wait_kv(0);
+      if (ok) issue_s(0, 0);
       for (int j = 0; ok && j <= n_tiles; ++j) {
-        if (j < n_tiles) {
-          const int s = j % KV_STAGES;
-          if (!mbar_wait(&kv_full[s], (uint32_t)((j / KV_STAGES) & 1), p.limit_ns, p.status,
-                         abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          issue_s(j, 0);  // buffer of slot 2j - 3 (P_B(j-2) V issued last iteration)
-        }
         if (j >= 1 && !issue_pv(j - 1, 0)) {
           ok = false;
           break;
@@ -236,6 +236,13 @@ __global__ void __launch_bounds__(320, 1)
             break;
           }
           tc_commit(&kv_empty[(j - 1) % KV_STAGES]);
+        }
+        if (j + 1 < n_tiles) {  // buffer of slot 2j - 1 (P_B(j-1) V just issued)
+          if (!wait_kv(j + 1)) {
+            ok = false;
+            break;
+          }
+          issue_s(j + 1, 0);
         }
       }
       if (!ok) *abort_flag = 1;
@@ -280,21 +287,23 @@ __global__ void __launch_bounds__(320, 1)
         for (int i = 0; i < KT; ++i)
           if (i >= kv_valid) sr[i] = __float_as_uint(-INFINITY);
       }
-      // row max: 8 independent chains over keys u, u+8, ..., u+120, two new keys per
-      // three-input max
-      static_assert(KT == 128, "max chains cover 16 keys each");
-      float mx[8];
+      // row max as a tree of three-input maxima: 128 -> 43 -> 15 -> 5 -> 2 -> 1 (depth 5;
+      // the 43 first-level maxima are independent)
+      static_assert(KT == 128, "max tree over 128 keys");
+      float m1[43];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        mx[u] = fmax3(__uint_as_float(sr[u]), __uint_as_float(sr[8 + u]),
-                      __uint_as_float(sr[16 + u]));
+      for (int i = 0; i < 42; ++i)
+        m1[i] = fmax3(__uint_as_float(sr[3 * i]), __uint_as_float(sr[3 * i + 1]),
+                      __uint_as_float(sr[3 * i + 2]));
+      m1[42] = fmaxf(__uint_as_float(sr[126]), __uint_as_float(sr[127]));
+      float m2[15];
 #pragma unroll
-        for (int c = 3; c < 15; c += 2)
-          mx[u] = fmax3(mx[u], __uint_as_float(sr[8 * c + u]), __uint_as_float(sr[8 * c + 8 + u]));
-        mx[u] = fmaxf(mx[u], __uint_as_float(sr[120 + u]));
-      }
-      const float mt = fmaxf(fmax3(mx[0], mx[1], mx[2]),
-                             fmax3(fmax3(mx[3], mx[4], mx[5]), mx[6], mx[7]));
+      for (int i = 0; i < 14; ++i) m2[i] = fmax3(m1[3 * i], m1[3 * i + 1], m1[3 * i + 2]);
+      m2[14] = m1[42];
+      const float m3[5] = {fmax3(m2[0], m2[1], m2[2]), fmax3(m2[3], m2[4], m2[5]),
+                           fmax3(m2[6], m2[7], m2[8]), fmax3(m2[9], m2[10], m2[11]),
+                           fmax3(m2[12], m2[13], m2[14])};
+      const float mt = fmaxf(fmax3(m3[0], m3[1], m3[2]), fmaxf(m3[3], m3[4]));
       float alpha = 1.f;
       bool resc = false;
       if (mt > m_run + thr) {

@@ -17,7 +17,7 @@ unsigned int* g_status_ptr();            // device address of the status word (c
 enum KernelId {
   K_PATCH_EMBED = 0, K_PERMUTE = 1, K_GEMM_QKV = 2, K_GEMM_GELU = 3, K_GEMM_STORE = 4,
   K_ATTN_WIN = 5, K_F32_GEMM = 6, K_F32_ATTN = 7, K_F32_STATS = 8, K_PACK = 9, K_PROBE = 10,
-  K_ROW_STATS = 11, K_ATTN_TC = 12, K_MLP_FUSED = 13, K_COUNT = 14
+  K_ROW_STATS = 11, K_ATTN_TC = 12, K_MLP_FUSED = 13, K_ATTN_BLOCK = 14, K_COUNT = 15
 };
 void profile_mark(int kind, cudaStream_t stream);  // no-op unless a session is open
 
@@ -125,6 +125,26 @@ hiera_status launch_attention_win(const AttnArgs& a, cudaStream_t stream);
 hiera_status launch_attention_tc(const AttnArgs& a, cudaStream_t stream);
 // The windowed kernel where it applies, else the general one.
 hiera_status launch_attention(const AttnArgs& a, cudaStream_t stream);
+
+// The attention half of a stage-0 block in one kernel (dim 112, 2 heads, windows of 64,
+// q_stride 1): x1 = x + proj(attention(norm1(x))) and x1's norm2 partials.
+struct AttnBlockArgs {
+  int B, tokens;
+  const void* x;            // bf16 [B, tokens, 112]
+  const void* stats_in;     // float2 [B * tokens][stats_parts] partials of x's rows
+  int stats_parts;
+  float ln_eps;
+  const void* w1;           // bf16 [336, 112] norm1-folded q | k | v weight
+  const float* colsum1;     // [336]
+  const float* colconst1;   // [336]
+  const void* wo;           // bf16 [112, 112] attention proj weight
+  const float* bias_o;      // [112]
+  void* x1;                 // bf16 [B, tokens, 112]
+  void* stats_out;          // float2 [B * tokens][2] (column halves), or nullptr
+};
+bool attention_block_supported(int B, int tokens, int d_in, int d_out, int heads, int q_stride,
+                               int window_tokens, int mask_unit_attn);
+hiera_status launch_attention_block(const AttnBlockArgs& a, cudaStream_t stream);
 
 // Raise `kern`'s dynamic shared-memory limit to `bytes` on the current device, once per
 // (kernel, device); thread-safe. False if the runtime refused.

@@ -44,7 +44,7 @@ def _expected(img, B):
 @pytest.mark.parametrize("fused", [True, False])
 def test_launch_flops_total_matches_the_architecture(fused):
     b = _bench()
-    launches = b.launch_flops(512, 8, fused_mlp=fused)
+    launches = b.launch_flops(512, 8, fused_mlp=fused, fused_attn=False)
     got = {}
     for cls, fl in launches:
         got[cls] = got.get(cls, 0.0) + fl
@@ -52,6 +52,11 @@ def test_launch_flops_total_matches_the_architecture(fused):
     assert got["gemm"] == pytest.approx(gemm, rel=1e-12)
     assert got["attention"] == pytest.approx(attn, rel=1e-12)
     assert got["patch_embed"] == pytest.approx(patch, rel=1e-12)
+    # with the stage-0 attention halves fused, the same total in fewer launches
+    fl = b.launch_flops(512, 8, fused_mlp=fused, fused_attn=True)
+    assert sum(f for _, f in fl) == pytest.approx(gemm + attn + patch, rel=1e-12)
+    assert sum(1 for c, _ in fl if c == "attn_block") == 2
+    assert len(fl) == len(launches) - 4
     # per image: 124.5 GF GEMM + 38.4 GF attention + 0.72 GF patch embedding
     assert gemm / 8 / 1e9 == pytest.approx(124.5, abs=0.05)
     assert attn / 8 / 1e9 == pytest.approx(38.4, abs=0.05)

@@ -32,7 +32,7 @@ UNIT_BOUND = 1e-2    # measured: at most 5.0e-3 (7.0e-3 with the widened score r
 
 
 def run_case(B, tokens, d_in, d_out, heads, q_stride, window, mua, dtype, seed, affine,
-             qk_scale=1.0):
+             qk_scale=1.0, fused_attn=False):
     transition = d_in != d_out
     p = syn.block_params(seed, d_in, d_out, transition, dtype=dtype, affine=affine)
     if qk_scale != 1.0:   # wider score range: q and k rows of the qkv weight scaled
@@ -46,7 +46,8 @@ def run_case(B, tokens, d_in, d_out, heads, q_stride, window, mua, dtype, seed, 
                         dtype=TORCH_DT[dtype])
     packed = hb.block_pack(desc, block_weights_dev(p, dtype))
     ws = torch.empty(hb.block_workspace_bytes(desc), dtype=torch.uint8, device="cuda")
-    y = hb.block_forward(desc, packed, dev(x, dtype), workspace=ws)
+    with hb.fused_attention(fused_attn):   # unfused: q, k, v, attention output in the workspace
+        y = hb.block_forward(desc, packed, dev(x, dtype), workspace=ws)
     assert hb.device_status() == 0
     ref = U.block_forward(x, p, heads, q_stride, window, mua)
     return host(y), ref, desc, packed, p, x, ws
@@ -160,7 +161,8 @@ def test_qkv_scatter_layout_bf16():
                         q_stride=qs, window_tokens=window)
     packed = hb.block_pack(desc, block_weights_dev(p, "bf16"))
     ws = torch.empty(hb.block_workspace_bytes(desc), dtype=torch.uint8, device="cuda")
-    hb.block_forward(desc, packed, dev(x), workspace=ws)
+    with hb.fused_attention(False):
+        hb.block_forward(desc, packed, dev(x), workspace=ws)
     torch.cuda.synchronize()
     offs = hb.block_workspace_layout(desc)
     nW = tokens // window
@@ -237,7 +239,7 @@ def test_block_intermediates_deterministic(name, fused):
     ref = None
     for rep in range(5):
         ws = torch.full((nbytes,), (rep * 53 + 7) % 256, dtype=torch.uint8, device="cuda")
-        with hb.fused_mlp(fused):
+        with hb.fused_mlp(fused), hb.fused_attention(False):
             y = hb.block_forward(desc, packed, x, workspace=ws)
         torch.cuda.synchronize()
         parts = [ws[o:o + n].clone() for o, n in zip(offs, sizes) if o >= 0] + [y.clone()]
@@ -246,4 +248,53 @@ def test_block_intermediates_deterministic(name, fused):
         else:
             for i, (a, b) in enumerate(zip(parts, ref)):
                 assert torch.equal(a, b), f"buffer {i} differs in repeat {rep}"
+    assert hb.device_status() == 0
+
+
+FUSED_ATTN_CASES = {
+    # stage-0 shapes the fused attention half takes: dim 112, 2 heads, windows of 64
+    "stage0_b2": (2, 256, 112, 112, 2, 1, 64, True),
+    "stage0_32x32": (1, 1024, 112, 112, 2, 1, 64, True),
+    "stage0_odd_tiles": (3, 384, 112, 112, 2, 1, 64, True),
+}
+
+
+@pytest.mark.parametrize("name", list(FUSED_ATTN_CASES))
+def test_fused_attention_half_matches_oracle(name):
+    """norm1 + qkv + windowed attention + proj + residual in one kernel (the block's
+    intermediates never reach memory): whole-output and per-row bounds against the
+    oracle, and within bf16 rounding of the separate kernels' result."""
+    args = FUSED_ATTN_CASES[name]
+    y, ref, desc, packed, p, x, _ = run_case(*args, dtype="bf16", seed=13, affine="random",
+                                             fused_attn=True)
+    assert np.isfinite(y).all()
+    assert rel_l2(y, ref) <= BF16_REL_L2, rel_l2(y, ref)
+    check_rows(y, ref)
+    with hb.fused_attention(False):
+        y_sep = host(hb.block_forward(desc, packed, dev(x)))
+    # the fused P V sums a window's keys in another order; the outputs agree to a few bf16
+    # ulps of the attention branch
+    assert rel_l2(y, y_sep) <= 2e-3, rel_l2(y, y_sep)
+
+
+def test_fused_attention_half_wide_scores():
+    y, ref, *_ = run_case(*FUSED_ATTN_CASES["stage0_32x32"], dtype="bf16", seed=14,
+                          affine="random", qk_scale=3.0, fused_attn=True)
+    assert rel_l2(y, ref) <= BF16_REL_L2, rel_l2(y, ref)
+    check_rows(y, ref)
+
+
+def test_fused_attention_half_deterministic_and_batch_independent():
+    B, tokens, d_in, d_out, heads, qs, window, mua = FUSED_ATTN_CASES["stage0_odd_tiles"]
+    p = syn.block_params(15, d_in, d_out, False, dtype="bf16", affine="random")
+    x = syn.activations(15, (B, tokens, d_in), dtype="bf16")
+    w = block_weights_dev(p, "bf16")
+    dB = hb.BlockDesc(B=B, tokens=tokens, dim_in=d_in, dim_out=d_out, heads=heads)
+    d1 = hb.BlockDesc(B=1, tokens=tokens, dim_in=d_in, dim_out=d_out, heads=heads)
+    pB, p1 = hb.block_pack(dB, w), hb.block_pack(d1, w)
+    yB = hb.block_forward(dB, pB, dev(x))
+    yB2 = hb.block_forward(dB, pB, dev(x))
+    y1 = hb.block_forward(d1, p1, dev(x[2:3]))
+    assert torch.equal(yB, yB2)
+    assert torch.equal(yB[2:3], y1)
     assert hb.device_status() == 0
