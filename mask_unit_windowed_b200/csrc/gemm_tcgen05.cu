@@ -99,10 +99,36 @@ struct Cfg {
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
+// Plain row-major outputs (EPI_STORE, EPI_GELU) leave through TMA tensor stores: each
+// epilogue warp stages its 32 rows x CH columns densely in shared memory and one lane stores
+// the block (rows past M are clipped by the tensor map).
+template <int EPI>
+struct TmaOut {
+  static constexpr bool value = EPI != EPI_QKV;
+};
+
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* smem_src, int c0,
+                                             int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(smem_src)), "r"(c0), "r"(c1)
+      : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// the bulk stores this thread committed have finished reading shared memory
+__device__ __forceinline__ void tma_store_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// ... and have completed
+__device__ __forceinline__ void tma_store_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 template <int BN, int EPI, bool FOLD, bool POOLED>
 __global__ void __launch_bounds__(320, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const KParams p) {
+                   const __grid_constant__ CUtensorMap tmO, const KParams p) {
   using C = Cfg<BN>;
   constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
@@ -437,12 +463,20 @@ __global__ void __launch_bounds__(320, 1)
         } else {
           dst_row = p.out + m * p.ldo + n0 + c_begin + c;
         }
-        // ---- stage the packed row in shared memory (XOR-swizzled 16-byte chunks)
+        // ---- stage the packed row in shared memory: XOR-swizzled 16-byte chunks for the
+        // copy-out below, or dense rows of CH values for a TMA store
         uint8_t* stg = stg_all + (ew << 12);
+        if (TmaOut<EPI>::value) {
+          if (lane == 0) tma_store_wait_read();  // the previous chunk's store has read stg
+          __syncwarp();
+        }
 #pragma unroll
         for (int g = 0; g < CH / 8; ++g) {
           const uint4 pk = pack8(&v[8 * g]);
-          *reinterpret_cast<uint4*>(stg + (lane << 7) + ((g ^ (lane & 7)) << 4)) = pk;
+          if (TmaOut<EPI>::value)
+            *reinterpret_cast<uint4*>(stg + lane * (CH * 2) + g * 16) = pk;
+          else
+            *reinterpret_cast<uint4*>(stg + (lane << 7) + ((g ^ (lane & 7)) << 4)) = pk;
           if (EPI == EPI_STORE && p.stats_out != nullptr) {
             // statistics of the values as stored (bf16)
             v[8 * g + 0] = bf16_lo(pk.x);
@@ -474,6 +508,13 @@ __global__ void __launch_bounds__(320, 1)
           const float dlt = cmean - st_mean;
           st_mean = fmaf(dlt, nb / nt_, st_mean);
           st_m2 = st_m2 + cm2 + dlt * dlt * (na * nb / nt_);
+        }
+        if (TmaOut<EPI>::value) {
+          fence_proxy_async_smem();  // this lane's staged row before the TMA engine reads it
+          __syncwarp();
+          if (lane == 0)
+            tma_store_2d(&tmO, stg, n0 + c_begin + c, (int)(m - rt + quarter * 32));
+          continue;
         }
         __syncwarp();
         // ---- copy out: 8 lanes per row, 4 rows per instruction, whole row segments
@@ -524,6 +565,8 @@ __global__ void __launch_bounds__(320, 1)
         aph ^= 1u;
       }
     }
+    // every TMA store of this warp has completed before the CTA exits
+    if (TmaOut<EPI>::value && lane == 0) tma_store_wait_all();
   }
 
   tc_fence_before();
@@ -560,6 +603,20 @@ bool encode_bf16(CUtensorMap* map, const void* base, int rank, const cuuint64_t*
   return encode_tmap_bf16_sw128(map, base, rank, dims, strides_bytes, box);
 }
 
+// 2-D bf16 tensor map without swizzle (the dense staging blocks of the TMA-store epilogue)
+bool encode_bf16_plain(CUtensorMap* map, const void* base, cuuint64_t cols, cuuint64_t rows,
+                       cuuint64_t row_bytes, cuuint32_t box_cols, cuuint32_t box_rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t str[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, str, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int BN, int EPI, bool FOLD, bool POOLED>
 hiera_status run(const TcGemmArgs& a, cudaStream_t stream) {
   using C = Cfg<BN>;
@@ -584,6 +641,11 @@ hiera_status run(const TcGemmArgs& a, cudaStream_t stream) {
     cuuint32_t box[2] = {BK, BN};
     if (!encode_bf16(&tmB, a.W, 2, dims, str, box)) return HIERA_ERR_CUDA;
   }
+  CUtensorMap tmO = tmA;  // unused by the q / k / v scatter
+  if (TmaOut<EPI>::value &&
+      !encode_bf16_plain(&tmO, a.out, (cuuint64_t)a.N, (cuuint64_t)a.M, (cuuint64_t)a.ldo * 2,
+                         (cuuint32_t)C::CH, 32))
+    return HIERA_ERR_CUDA;
   KParams p;
   p.M = a.M;
   p.N = a.N;
@@ -621,7 +683,7 @@ hiera_status run(const TcGemmArgs& a, cudaStream_t stream) {
   if (grid > tiles) grid = tiles;
   profile_mark(EPI == EPI_QKV ? K_GEMM_QKV : (EPI == EPI_GELU ? K_GEMM_GELU : K_GEMM_STORE),
                stream);
-  launch_k(kern, dim3(grid), dim3(320), C::SMEM_BYTES, stream, tmA, tmB, p);
+  launch_k(kern, dim3(grid), dim3(320), C::SMEM_BYTES, stream, tmA, tmB, tmO, p);
   return cudaGetLastError() == cudaSuccess ? HIERA_OK : HIERA_ERR_CUDA;
 }
 
