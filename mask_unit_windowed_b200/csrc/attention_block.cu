@@ -24,9 +24,11 @@
 // use; only the summation order inside the P V product differs (the two windows' keys are
 // interleaved), so the result agrees with the unfused path to rounding.
 // Roles (320 threads, persistent CTAs, tiles strided over the grid): warp 0 TMA producer
-// (x tiles, double-buffered; the q, k, v and proj weights through a two-slot ring), warp 1
-// TMEM owner and MMA issuer, warps 2-9 epilogue / softmax (two per TMEM lane quarter: head
-// or column half 0 and 1).
+// (the q, k, v and proj weights once per CTA, resident in shared memory; the x tile of each
+// tile, whose buffer then holds q, so the next x loads as soon as the scores are computed),
+// warp 1 TMEM owner and MMA issuer, warps 2-9 epilogue / softmax (two per TMEM lane quarter:
+// head or column half 0 and 1). The merged heads are written over k, which the scores no
+// longer need.
 #include <math.h>
 
 #include "common.cuh"
@@ -39,12 +41,11 @@ constexpr int FD = 112;                        // dim
 constexpr int FW_BYTES = 2 * FD * 128;          // one 112-row weight chunk, two 64-column blocks
 constexpr int FX_BYTES = 2 * 128 * 128;         // [128 rows][two 64-column blocks]
 constexpr int FH_BYTES = 128 * 128;             // one head's [128 rows][64] operand tile
-constexpr int F_OFF_X = 0;                      // x[2]; q and then the merged heads alias x[t&1]
-constexpr int F_OFF_K = F_OFF_X + 2 * FX_BYTES;
+constexpr int F_OFF_X = 0;                      // x, then q (per head)
+constexpr int F_OFF_K = F_OFF_X + FX_BYTES;     // k (per head), then the merged heads
 constexpr int F_OFF_V = F_OFF_K + 2 * FH_BYTES;
-constexpr int F_OFF_W = F_OFF_V + 2 * FH_BYTES;
-constexpr int F_RING = 2;
-constexpr int F_OFF_C = F_OFF_W + F_RING * FW_BYTES;      // colsum1[336], colconst1[336], bo[112]
+constexpr int F_OFF_W = F_OFF_V + 2 * FH_BYTES; // W_q, W_k, W_v, W_o, resident
+constexpr int F_OFF_C = F_OFF_W + 4 * FW_BYTES;           // colsum1[336], colconst1[336], bo[112]
 constexpr int F_OFF_BAR = F_OFF_C + (2 * 3 * FD + FD) * 4;
 constexpr int F_SMEM = F_OFF_BAR + 256 + 1024;
 // TMEM: q, k, v accumulators at 0, 128, 256; then S_h at 128 h and O_h at 256 + 64 h;
@@ -80,11 +81,10 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t* smem = smem_raw + pad;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + F_OFF_BAR);
-  uint64_t* x_full = bars;              // [2]
-  uint64_t* x_empty = x_full + 2;       // [2]
-  uint64_t* w_full = x_empty + 2;       // [F_RING]
-  uint64_t* w_empty = w_full + F_RING;  // [F_RING]
-  uint64_t* qkv_done = w_empty + F_RING;
+  uint64_t* x_full = bars;
+  uint64_t* x_empty = x_full + 1;       // the scores have consumed q (written over x)
+  uint64_t* w_full = x_empty + 1;
+  uint64_t* qkv_done = w_full + 1;
   uint64_t* qkv_staged = qkv_done + 1;  // 256
   uint64_t* s_full = qkv_staged + 1;
   uint64_t* p_full = s_full + 1;        // 256
@@ -105,14 +105,9 @@ __global__ void __launch_bounds__(320, 1)
   const int pairs = p.nW >> 1;  // window pairs (tiles) per image
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&x_full[i], 1);
-      mbar_init(&x_empty[i], 1);
-    }
-    for (int i = 0; i < F_RING; ++i) {
-      mbar_init(&w_full[i], 1);
-      mbar_init(&w_empty[i], 1);
-    }
+    mbar_init(x_full, 1);
+    mbar_init(x_empty, 1);
+    mbar_init(w_full, 1);
     mbar_init(qkv_done, 1);
     mbar_init(qkv_staged, 256);
     mbar_init(s_full, 1);
@@ -141,50 +136,33 @@ __global__ void __launch_bounds__(320, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      bool ok = true;
-      int wc = 0;  // weight chunks issued
-      long long xi = 0;
-      auto load_w = [&](const CUtensorMap* map, int row0) -> bool {
-        const int slot = wc % F_RING;
-        if (!mbar_wait(&w_empty[slot], (uint32_t)(((wc / F_RING) & 1) ^ 1), p.limit_ns, p.status,
-                       abort_flag))
-          return false;
-        uint8_t* dst = smem + F_OFF_W + slot * FW_BYTES;
-        mbar_arrive_expect_tx(&w_full[slot], FW_BYTES);
-        tma_load_2d(dst, map, &w_full[slot], 0, row0);
-        tma_load_2d(dst + FD * 128, map, &w_full[slot], 64, row0);
-        ++wc;
-        return true;
-      };
-      for (int t = 0; ok && t < n_local; ++t) {
+    if (lane == 0 && n_local > 0) {
+      // the four weight chunks once: W_q, W_k, W_v (rows of the packed qkv weight), W_o
+      mbar_arrive_expect_tx(w_full, 4 * FW_BYTES);
+      for (int g = 0; g < 4; ++g) {
+        uint8_t* dst = smem + F_OFF_W + g * FW_BYTES;
+        const CUtensorMap* map = g < 3 ? &tmW1 : &tmWo;
+        const int row0 = g < 3 ? g * FD : 0;
+        tma_load_2d(dst, map, w_full, 0, row0);
+        tma_load_2d(dst + FD * 128, map, w_full, 64, row0);
+      }
+      int issued = 0;
+      for (int t = 0; t < n_local; ++t) {
         const int tile = (int)blockIdx.x + t * (int)gridDim.x;
         const int b = tile / pairs, w0 = 2 * (tile - b * pairs);
-        const int xb = t & 1;
-        if (!mbar_wait(&x_empty[xb], (uint32_t)(((t >> 1) & 1) ^ 1), p.limit_ns, p.status,
-                       abort_flag)) {
-          ok = false;
+        if (!mbar_wait(x_empty, (uint32_t)((t & 1) ^ 1), p.limit_ns, p.status, abort_flag)) {
+          *abort_flag = 1;
           break;
         }
-        uint8_t* xd = smem + F_OFF_X + xb * FX_BYTES;
-        mbar_arrive_expect_tx(&x_full[xb], FX_BYTES);
-        tma_load_4d(xd, &tmX, &x_full[xb], 0, w0, 0, b);
-        tma_load_4d(xd + 128 * 128, &tmX, &x_full[xb], 64, w0, 0, b);
-        ++xi;
-        ok = load_w(&tmW1, 0) && load_w(&tmW1, FD) && load_w(&tmW1, 2 * FD) && load_w(&tmWo, 0);
+        uint8_t* xd = smem + F_OFF_X;
+        mbar_arrive_expect_tx(x_full, FX_BYTES);
+        tma_load_4d(xd, &tmX, x_full, 0, w0, 0, b);
+        tma_load_4d(xd + 128 * 128, &tmX, x_full, 64, w0, 0, b);
+        ++issued;
       }
-      if (!ok) *abort_flag = 1;
-      // let the copies in flight land before the CTA's shared memory goes away
-      for (int s = 0; s < F_RING; ++s)
-        if (wc > s) {
-          const int last = wc - 1 - ((wc - 1 - s) % F_RING);
-          mbar_wait(&w_full[s], (uint32_t)((last / F_RING) & 1), p.limit_ns, p.status);
-        }
-      for (int s = 0; s < 2; ++s)
-        if (xi > s) {
-          const long long last = xi - 1 - ((xi - 1 - s) % 2);
-          mbar_wait(&x_full[s], (uint32_t)((last >> 1) & 1), p.limit_ns, p.status);
-        }
+      // the copies in flight land before the CTA's shared memory goes away
+      mbar_wait(w_full, 0, p.limit_ns, p.status);
+      if (issued > 0) mbar_wait(x_full, (uint32_t)((issued - 1) & 1), p.limit_ns, p.status);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -194,17 +172,10 @@ __global__ void __launch_bounds__(320, 1)
       constexpr uint32_t IDESC_O = idesc_bf16_f32(128, 64) | IDESC_B_MN_MAJOR;
       const uint64_t desc0 = smem_desc_sw128(smem_u32(smem));
       bool ok = true;
-      int wc = 0;
-      // D[tmem] = A[128 x 112] W[112 x 112]^T: 7 K steps over two 64-column blocks
-      auto gemm112 = [&](uint32_t d, uint32_t a_off, bool& okr) {
-        const int slot = wc % F_RING;
-        if (!mbar_wait(&w_full[slot], (uint32_t)((wc / F_RING) & 1), p.limit_ns, p.status,
-                       abort_flag)) {
-          okr = false;
-          return;
-        }
-        tc_fence_after();
-        const uint32_t w_off = (uint32_t)(F_OFF_W + slot * FW_BYTES);
+      if (n_local > 0) ok = mbar_wait(w_full, 0, p.limit_ns, p.status, abort_flag);
+      // D[tmem] = A[128 x 112] W_g[112 x 112]^T: 7 K steps over two 64-column blocks
+      auto gemm112 = [&](uint32_t d, uint32_t a_off, int g) {
+        const uint32_t w_off = (uint32_t)(F_OFF_W + g * FW_BYTES);
 #pragma unroll
         for (int st = 0; st < FD / 16; ++st) {
           const uint32_t kb = (uint32_t)(st >> 2), kk = (uint32_t)(st & 3);
@@ -215,21 +186,18 @@ __global__ void __launch_bounds__(320, 1)
           else
             tc_mma_bf16_k<true>(d, ad, wd, IDESC_112);
         }
-        tc_commit(&w_empty[slot]);
-        ++wc;
       };
       for (int t = 0; ok && t < n_local; ++t) {
-        const int xb = t & 1;
         const uint32_t ph = (uint32_t)(t & 1);
-        const uint32_t x_off = (uint32_t)(F_OFF_X + xb * FX_BYTES);
-        if (!mbar_wait(&x_full[xb], (uint32_t)((t >> 1) & 1), p.limit_ns, p.status, abort_flag)) {
+        const uint32_t x_off = (uint32_t)F_OFF_X;
+        if (!mbar_wait(x_full, ph, p.limit_ns, p.status, abort_flag)) {
           ok = false;
           break;
         }
+        tc_fence_after();
         // (the previous tile's O was read before its merged heads were staged, which the
         // previous iteration waited for: TMEM columns 0..383 are free)
-        for (int g = 0; g < 3 && ok; ++g) gemm112(tmem + (uint32_t)(128 * g), x_off, ok);
-        if (!ok) break;
+        for (int g = 0; g < 3; ++g) gemm112(tmem + (uint32_t)(128 * g), x_off, g);
         tc_commit(qkv_done);
         // S_h = q_h k_h^T
         if (!mbar_wait(qkv_staged, ph, p.limit_ns, p.status, abort_flag)) {
@@ -247,6 +215,7 @@ __global__ void __launch_bounds__(320, 1)
           for (int kk = 1; kk < 4; ++kk)
             tc_mma_bf16_k<true>(sd, desc_advance(qd, 32u * kk), desc_advance(kd, 32u * kk), IDESC_S);
         }
+        tc_commit(x_empty);  // q consumed: the next x may overwrite it
         tc_commit(s_full);
         // O_h = P_h V_h (P over the S columns, 128 keys in 64 columns)
         if (!mbar_wait(p_full, ph, p.limit_ns, p.status, abort_flag)) {
@@ -272,9 +241,7 @@ __global__ void __launch_bounds__(320, 1)
           break;
         }
         tc_fence_after();
-        gemm112(tmem + F_PROJ_COL, x_off, ok);
-        if (!ok) break;
-        tc_commit(&x_empty[xb]);
+        gemm112(tmem + F_PROJ_COL, (uint32_t)F_OFF_K, 3);  // merged heads over k, W_o
         tc_commit(proj_full);
       }
       if (!ok) *abort_flag = 1;
@@ -300,7 +267,8 @@ __global__ void __launch_bounds__(320, 1)
       const int b = tile / pairs, w0 = 2 * (tile - b * pairs);
       const long long tok = (long long)b * p.N + (long long)jr * p.nW + w0 + par;
       const uint32_t ph = (uint32_t)(t & 1);
-      uint8_t* xq = smem + F_OFF_X + (t & 1) * FX_BYTES;  // q, then the merged heads
+      uint8_t* xq = smem + F_OFF_X;  // q (written over x)
+      uint8_t* om = smem + F_OFF_K;  // the merged heads (written over k)
       float fa = 1.f, fb = 0.f;
       ln_fold_coeffs(p.stats_in + tok * p.stats_parts, p.stats_parts, FD, p.ln_eps, fa, fb);
       // ---- 2. q, k, v of head hs: fold, bf16, operand tiles
@@ -392,7 +360,7 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
           for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(ov[8 * c8 + e]) * inv;
           const int ch = 7 * hs + c8;  // 16-byte chunk of the 112-channel row
-          *reinterpret_cast<uint4*>(xq + (ch >> 3) * 16384 + r * 128 +
+          *reinterpret_cast<uint4*>(om + (ch >> 3) * 16384 + r * 128 +
                                     ((((uint32_t)ch & 7u) ^ (uint32_t)(r & 7)) << 4)) = pack8(f);
         }
       }
