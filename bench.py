@@ -66,11 +66,14 @@ def peaks():
 
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of a kernel shape,
-# from one ncu capture of that kernel alone (three launches of the shape, this workload);
-# the summaries under profiles/ give the commands. Keyed by (kernel kind, GFLOP per launch
-# rounded to 0.01). A shape missing here reports traffic null; an entry must be removed
-# whenever its kernel changes.
-DRAM_BYTES_PER_LAUNCH = {}
+# from one ncu capture of one launch of that shape in this workload; the summaries under
+# profiles/ give the commands. Keyed by (kernel kind, GFLOP per launch rounded to 0.01). A
+# shape missing here reports traffic null; an entry must be removed whenever its kernel
+# changes.
+DRAM_BYTES_PER_LAUNCH = {
+    # stage-2 global attention, 8 x 8 x 1024 x 1024 (profiles/attention_tcgen05_stage2_512_b8.md)
+    ("attention_tcgen05", 15.03): 25_421_312,
+}
 
 
 def reroll_bytes(img: int, B: int):

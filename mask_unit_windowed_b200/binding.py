@@ -550,6 +550,7 @@ def kernel_name(kind: int) -> str:
 OPT_FUSED_MLP = 0
 OPT_PDL = 1
 OPT_FUSED_ATTN = 2
+OPT_GEMM_PAIR = 3
 
 
 def set_option(opt: int, value: int):
@@ -586,6 +587,12 @@ def fused_attention(enabled: bool) -> option:
     residual) as one kernel (True, the default) or as the separate kernels, which also write
     q, k, v and the attention output to the workspace."""
     return option(OPT_FUSED_ATTN, bool(enabled))
+
+
+def gemm_pair(enabled: bool) -> option:
+    """Run the 224-column-tile Linear layers on CTA pairs (True: one 256 x 224 tile per two
+    SMs, tcgen05.mma.cta_group::2) or one CTA per 128 x 224 tile (False, the default)."""
+    return option(OPT_GEMM_PAIR, bool(enabled))
 
 
 def pdl(enabled: bool) -> option:

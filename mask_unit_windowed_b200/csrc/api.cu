@@ -646,8 +646,8 @@ void profile_mark(int kind, cudaStream_t stream) {
 }
 
 namespace {
-int g_options[HIERA_OPT_COUNT] = {1, 1, 1};  // fused MLP, programmatic dependent launch and
-                                             // fused attention half on
+// fused MLP, programmatic dependent launch and fused attention half on; CTA-pair GEMMs off
+int g_options[HIERA_OPT_COUNT] = {1, 1, 1, 0};
 }  // namespace
 
 int g_option(int opt) { return (opt >= 0 && opt < HIERA_OPT_COUNT) ? g_options[opt] : 0; }

@@ -30,39 +30,14 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "gemm_shared.cuh"
 #include "internal.h"
 
 namespace hiera {
 namespace {
 
-constexpr int BM = 128;
-constexpr int BK = 64;
 constexpr int EPI_WARPS = 8;              // 2 per TMEM lane quarter, each half the columns
 constexpr int EPI_THREADS = EPI_WARPS * 32;
-
-struct KParams {
-  int M, N, K;
-  const float* colsum;
-  const float* colconst;
-  const bf16* bias16;
-  float ln_eps;
-  bf16* out;
-  const bf16* residual;
-  int ldo;
-  bf16* q;
-  bf16* k;
-  bf16* v;
-  bf16* r;
-  int tokens, nW, heads, d_out, Tq, Tkv;
-  uint64_t limit_ns;
-  unsigned int* status;
-  const float2* stats_in;  // FOLD: [M][stats_parts] partial (mean, M2) of A's rows
-  int stats_parts;
-  float2* stats_out;       // STORE: [M][stats_out_parts] partials of the output, or nullptr
-  int stats_out_parts;
-};
-
-constexpr int cmin(int a, int b) { return a < b ? a : b; }
 
 // element-wise max of two groups of 8 bf16 (finite values)
 __device__ __forceinline__ uint4 bf16x8_max(uint4 a, uint4 b) {
@@ -98,32 +73,6 @@ struct Cfg {
   static_assert(CONST_OFF % 16 == 0 && (HALF * 4) % 16 == 0, "16-byte constant loads");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
-
-// Plain row-major outputs (EPI_STORE, EPI_GELU) leave through TMA tensor stores: each
-// epilogue warp stages its 32 rows x CH columns densely in shared memory and one lane stores
-// the block (rows past M are clipped by the tensor map).
-template <int EPI>
-struct TmaOut {
-  static constexpr bool value = EPI != EPI_QKV;
-};
-
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* smem_src, int c0,
-                                             int c1) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-          reinterpret_cast<uint64_t>(map)),
-      "r"(smem_u32(smem_src)), "r"(c0), "r"(c1)
-      : "memory");
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-// the bulk stores this thread committed have finished reading shared memory
-__device__ __forceinline__ void tma_store_wait_read() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-// ... and have completed
-__device__ __forceinline__ void tma_store_wait_all() {
-  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
 
 template <int BN, int EPI, bool FOLD, bool POOLED>
 __global__ void __launch_bounds__(320, 1)
@@ -503,11 +452,8 @@ __global__ void __launch_bounds__(320, 1)
           float cm2 = 0.f;
 #pragma unroll
           for (int i = 0; i < CH; ++i) cm2 = fmaf(v[i] - cmean, v[i] - cmean, cm2);
-          // Chan et al. merge of this chunk into the running (count, mean, M2)
-          const float na = (float)c, nb = (float)CH, nt_ = na + nb;
-          const float dlt = cmean - st_mean;
-          st_mean = fmaf(dlt, nb / nt_, st_mean);
-          st_m2 = st_m2 + cm2 + dlt * dlt * (na * nb / nt_);
+          // merge this chunk into the running (count, mean, M2)
+          chan_merge(st_mean, st_m2, cmean, cm2, (float)c, (float)CH);
         }
         if (TmaOut<EPI>::value) {
           fence_proxy_async_smem();  // this lane's staged row before the TMA engine reads it
@@ -603,19 +549,6 @@ bool encode_bf16(CUtensorMap* map, const void* base, int rank, const cuuint64_t*
   return encode_tmap_bf16_sw128(map, base, rank, dims, strides_bytes, box);
 }
 
-// 2-D bf16 tensor map without swizzle (the dense staging blocks of the TMA-store epilogue)
-bool encode_bf16_plain(CUtensorMap* map, const void* base, cuuint64_t cols, cuuint64_t rows,
-                       cuuint64_t row_bytes, cuuint32_t box_cols, cuuint32_t box_rows) {
-  EncodeTiledFn fn = get_encode_fn();
-  if (fn == nullptr) return false;
-  const cuuint64_t dims[2] = {cols, rows};
-  const cuuint64_t str[1] = {row_bytes};
-  const cuuint32_t box[2] = {box_cols, box_rows};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, str, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 template <int BN, int EPI, bool FOLD, bool POOLED>
 hiera_status run(const TcGemmArgs& a, cudaStream_t stream) {
@@ -689,6 +622,19 @@ hiera_status run(const TcGemmArgs& a, cudaStream_t stream) {
 
 }  // namespace
 
+bool encode_bf16_plain(CUtensorMap* map, const void* base, cuuint64_t cols, cuuint64_t rows,
+                       cuuint64_t row_bytes, cuuint32_t box_cols, cuuint32_t box_rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t str[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, str, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool encode_tmap_bf16_sw128(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
                             const cuuint64_t* strides_bytes, const cuuint32_t* box) {
   EncodeTiledFn fn = get_encode_fn();
@@ -719,9 +665,13 @@ hiera_status launch_tc_gemm(int epi, const TcGemmArgs& a, cudaStream_t stream) {
       if (a.tokens % 4 != 0 || per < 2 || (per >= 32 ? per % 32 != 0 : 32 % per != 0))
         return HIERA_ERR_SHAPE;
     }
-    if (a.d_out % 224 == 0)
-      return pooled ? run<224, EPI_QKV, true, true>(a, stream)
-                    : run<224, EPI_QKV, true, false>(a, stream);
+    if (a.d_out % 224 == 0) {
+      if (pooled) return run<224, EPI_QKV, true, true>(a, stream);
+      // (the pair kernel writes q, k and v only: no residual-projection columns)
+      return g_option(HIERA_OPT_GEMM_PAIR) && a.N == 3 * a.d_out
+                 ? run_pair<EPI_QKV, true>(a, stream)
+                 : run<224, EPI_QKV, true, false>(a, stream);
+    }
     if (a.d_out % 112 == 0)
       return pooled ? run<112, EPI_QKV, true, true>(a, stream)
                     : run<112, EPI_QKV, true, false>(a, stream);
@@ -729,13 +679,17 @@ hiera_status launch_tc_gemm(int epi, const TcGemmArgs& a, cudaStream_t stream) {
   }
   if (epi == EPI_GELU) {
     if (!a.ln_fold) return HIERA_ERR_INVALID_ARG;
-    if (a.N % 224 == 0) return run<224, EPI_GELU, true, false>(a, stream);
+    if (a.N % 224 == 0)
+      return g_option(HIERA_OPT_GEMM_PAIR) ? run_pair<EPI_GELU, true>(a, stream)
+                                           : run<224, EPI_GELU, true, false>(a, stream);
     if (a.N % 112 == 0) return run<112, EPI_GELU, true, false>(a, stream);
     return HIERA_ERR_SHAPE;
   }
   if (a.ln_fold) return HIERA_ERR_INVALID_ARG;
   switch (store_bn(a.N)) {
-    case 224: return run<224, EPI_STORE, false, false>(a, stream);
+    case 224:
+      return g_option(HIERA_OPT_GEMM_PAIR) ? run_pair<EPI_STORE, false>(a, stream)
+                                           : run<224, EPI_STORE, false, false>(a, stream);
     case 128: return run<128, EPI_STORE, false, false>(a, stream);
     case 112: return run<112, EPI_STORE, false, false>(a, stream);
     case 64: return run<64, EPI_STORE, false, false>(a, stream);

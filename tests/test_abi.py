@@ -122,3 +122,16 @@ def test_binding_rejects_mismatched_tensors_before_any_launch():
     # shapes right, but host tensors: still refused before the library is called
     with pytest.raises(ValueError, match="CUDA"):
         hb.block_forward(d, packed, torch.empty(2, 256, 112, dtype=torch.bfloat16))
+
+
+def test_option_defaults_and_range():
+    """Library options are host state: fused MLP, programmatic launch and the fused attention
+    half default on, CTA-pair GEMMs off; unknown options and values are rejected."""
+    assert [hb.get_option(o) for o in (hb.OPT_FUSED_MLP, hb.OPT_PDL, hb.OPT_FUSED_ATTN,
+                                       hb.OPT_GEMM_PAIR)] == [1, 1, 1, 0]
+    L = hb.lib()
+    assert L.hiera_set_option(4, 1) == 1
+    assert L.hiera_set_option(hb.OPT_GEMM_PAIR, 2) == 1
+    with hb.gemm_pair(True):
+        assert hb.get_option(hb.OPT_GEMM_PAIR) == 1
+    assert hb.get_option(hb.OPT_GEMM_PAIR) == 0
