@@ -159,3 +159,20 @@ def test_global_small_sizes_use_the_general_kernel():
         v = syn.normal(seed, 3, (2, 3, 2, Tkv, HD), dtype="bf16")
         got, ref = run(q, k, v)
         check(got, ref)
+
+
+def test_global_more_ctas_than_sms():
+    """4 x 40 units x 2 query-tile pairs = 320 CTAs of the 128-key-tile kernel on 148 SMs
+    (several waves, ragged query and key tiles). Each unit's keys carry their own scale (1x
+    to 9x) and its last, ragged tile (44 of 300 keys) holds keys scaled 4x more, so a unit
+    whose running max or rescale went wrong would be far off."""
+    B, nW, heads, Tq, Tkv = 4, 1, 40, 300, 300
+    q = syn.normal(73, 1, (B, nW, heads, Tq, HD), dtype="bf16")
+    k = syn.normal(73, 2, (B, nW, heads, Tkv, HD))
+    unit = np.arange(B * nW * heads).reshape(B, nW, heads)
+    k = k * (1.0 + 2.0 * (unit % 5))[..., None, None]
+    k[..., 256:, :] *= 4.0
+    k = bf16(k)
+    v = syn.normal(73, 3, (B, nW, heads, Tkv, HD), dtype="bf16")
+    got, ref = run(q, k, v)
+    check(got, ref)
