@@ -351,6 +351,10 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     hb.set_option(hb.OPT_FUSED_MLP, 1 if args.mlp == "fused" else 0)
     hb.set_option(hb.OPT_PDL, 1 if args.pdl == "on" else 0)
     hb.set_option(hb.OPT_FUSED_ATTN, 1 if args.attn == "fused" else 0)
+    if args.gemm224 != "default":
+        hb.set_option(hb.OPT_GEMM224, {"8warp": hb.GEMM224_EIGHT_WARPS,
+                                       "16warp": hb.GEMM224_SIXTEEN_WARPS,
+                                       "pair": hb.GEMM224_PAIR}[args.gemm224])
     hbm_gbs, tf_burst, tf_sust, peak_src = peaks()
     B = args.batch
 
@@ -582,7 +586,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                    "l2": "flushed before every step (256 MiB write); within a step each "
                          "forward's working set (138 MB of weights + activations) exceeds L2",
                    "timing": "CUDA-graph replay of the library launches, per-step CUDA events",
-                   "mlp": args.mlp, "pdl": args.pdl, "attn": args.attn},
+                   "mlp": args.mlp, "pdl": args.pdl, "attn": args.attn,
+                   "gemm224": ["8warp", "16warp", "pair"][hb.get_option(hb.OPT_GEMM224)]},
         "ms_per_forward": ms_per_forward,
         "timed_seconds": total_ms / 1e3,
         "tflops": gflop_per_image * images / (total_ms * 1e-3) * 1e-3,
@@ -630,6 +635,10 @@ def main():
     ap.add_argument("--attn", choices=["fused", "unfused"], default="fused",
                     help="stage-0 attention half (norm1, qkv, attention, proj) as one kernel "
                          "(default) or three")
+    ap.add_argument("--gemm224", choices=["default", "8warp", "16warp", "pair"],
+                    default="default",
+                    help="kernel of the 224-column-tile Linear layers (library default, the "
+                         "eight- or sixteen-epilogue-warp CTA, or the CTA pair)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

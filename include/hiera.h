@@ -324,21 +324,23 @@ HIERA_API hiera_status hiera_backbone_forward(const hiera_backbone_desc* desc, c
  *                        0: the separate qkv GEMM, attention and proj GEMM. The two agree
  *                        to rounding (the fused P V product sums the window's keys in
  *                        another order).
- *   HIERA_OPT_GEMM_PAIR  0 (default): one CTA per 128 x 224 output tile. 1: the bf16 Linear
- *                        layers whose output columns come in tiles of 224 (dims 224, 448,
- *                        896; not the transition's pooled qkv) run on CTA pairs, one
- *                        256 x 224 tile per pair of SMs with tcgen05.mma.cta_group::2, each
- *                        SM loading its 128 input rows and half of the weight tile. Both
- *                        give the same bits; on B200 the pair form measured slower at the
- *                        backbone's shapes, hence the default.
- * hiera_set_option returns HIERA_ERR_INVALID_ARG for an unknown option or value;
+ *   HIERA_OPT_GEMM224    the kernel for the bf16 Linear layers whose output columns come in
+ *                        tiles of 224 (dims 224, 448, 896; not the transition's pooled qkv).
+ *                        0 (default): one CTA per 128 x 224 tile with eight epilogue warps.
+ *                        1: one CTA per 128 x 224 tile with sixteen epilogue warps (one
+ *                        56-column chunk each). 2: a CTA pair per 256 x 224 tile
+ *                        (tcgen05.mma.cta_group::2, each SM loading its 128 input rows and
+ *                        half of the weight tile) with the sixteen-warp epilogue. All three
+ *                        give the same bits.
+ * hiera_set_option returns HIERA_ERR_INVALID_ARG for an unknown option or value (0 or
+ * 1; 0 to 2 for HIERA_OPT_GEMM224);
  * hiera_get_option returns the current value (0 for an unknown option).
  * -------------------------------------------------------------------------------- */
 typedef enum {
   HIERA_OPT_FUSED_MLP = 0,
   HIERA_OPT_PDL = 1,
   HIERA_OPT_FUSED_ATTN = 2,
-  HIERA_OPT_GEMM_PAIR = 3,
+  HIERA_OPT_GEMM224 = 3,
   HIERA_OPT_COUNT = 4
 } hiera_option;
 HIERA_API hiera_status hiera_set_option(hiera_option opt, int value);

@@ -550,7 +550,8 @@ def kernel_name(kind: int) -> str:
 OPT_FUSED_MLP = 0
 OPT_PDL = 1
 OPT_FUSED_ATTN = 2
-OPT_GEMM_PAIR = 3
+OPT_GEMM224 = 3
+GEMM224_EIGHT_WARPS, GEMM224_SIXTEEN_WARPS, GEMM224_PAIR = 0, 1, 2
 
 
 def set_option(opt: int, value: int):
@@ -589,10 +590,11 @@ def fused_attention(enabled: bool) -> option:
     return option(OPT_FUSED_ATTN, bool(enabled))
 
 
-def gemm_pair(enabled: bool) -> option:
-    """Run the 224-column-tile Linear layers on CTA pairs (True: one 256 x 224 tile per two
-    SMs, tcgen05.mma.cta_group::2) or one CTA per 128 x 224 tile (False, the default)."""
-    return option(OPT_GEMM_PAIR, bool(enabled))
+def gemm224(mode: int) -> option:
+    """Kernel for the 224-column-tile Linear layers: GEMM224_EIGHT_WARPS (the default: one
+    CTA per 128 x 224 tile, eight epilogue warps), GEMM224_SIXTEEN_WARPS (one CTA, sixteen
+    epilogue warps) or GEMM224_PAIR (a CTA pair per 256 x 224 tile, tcgen05.mma.cta_group::2)."""
+    return option(OPT_GEMM224, int(mode))
 
 
 def pdl(enabled: bool) -> option:

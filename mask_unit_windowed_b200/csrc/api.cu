@@ -646,7 +646,8 @@ void profile_mark(int kind, cudaStream_t stream) {
 }
 
 namespace {
-// fused MLP, programmatic dependent launch and fused attention half on; CTA-pair GEMMs off
+// fused MLP, programmatic dependent launch and fused attention half on; the eight-warp
+// 224-column GEMM
 int g_options[HIERA_OPT_COUNT] = {1, 1, 1, 0};
 }  // namespace
 
@@ -994,7 +995,8 @@ int hiera_profile_end(hiera_stream_t stream) {
 
 hiera_status hiera_set_option(hiera_option opt, int value) {
   if (opt < 0 || opt >= HIERA_OPT_COUNT) return HIERA_ERR_INVALID_ARG;
-  if (value != 0 && value != 1) return HIERA_ERR_INVALID_ARG;
+  const int max_value = opt == HIERA_OPT_GEMM224 ? 2 : 1;
+  if (value < 0 || value > max_value) return HIERA_ERR_INVALID_ARG;
   g_options[opt] = value;
   return HIERA_OK;
 }

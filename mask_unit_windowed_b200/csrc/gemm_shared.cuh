@@ -77,8 +77,9 @@ __device__ __forceinline__ void tma_store_wait_all() {
 bool encode_bf16_plain(CUtensorMap* map, const void* base, cuuint64_t cols, cuuint64_t rows,
                        cuuint64_t row_bytes, cuuint32_t box_cols, cuuint32_t box_rows);
 
-// The CTA-pair GEMM (tile 256 x 224, cta_group::2) for the non-pooled 224-column variants.
-template <int EPI, bool FOLD>
-hiera_status run_pair(const TcGemmArgs& a, cudaStream_t stream);
+// The sixteen-epilogue-warp GEMMs for the non-pooled 224-column variants: one CTA per
+// 128 x 224 tile (PAIR false) or a CTA pair per 256 x 224 tile (cta_group::2, PAIR true).
+template <int EPI, bool FOLD, bool PAIR>
+hiera_status run_wide(const TcGemmArgs& a, cudaStream_t stream);
 
 }  // namespace hiera

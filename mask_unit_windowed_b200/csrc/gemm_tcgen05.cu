@@ -667,10 +667,11 @@ hiera_status launch_tc_gemm(int epi, const TcGemmArgs& a, cudaStream_t stream) {
     }
     if (a.d_out % 224 == 0) {
       if (pooled) return run<224, EPI_QKV, true, true>(a, stream);
-      // (the pair kernel writes q, k and v only: no residual-projection columns)
-      return g_option(HIERA_OPT_GEMM_PAIR) && a.N == 3 * a.d_out
-                 ? run_pair<EPI_QKV, true>(a, stream)
-                 : run<224, EPI_QKV, true, false>(a, stream);
+      // (the sixteen-warp kernels write q, k and v only: no residual-projection columns)
+      const int mode = a.N == 3 * a.d_out ? g_option(HIERA_OPT_GEMM224) : 0;
+      return mode == 1   ? run_wide<EPI_QKV, true, false>(a, stream)
+             : mode == 2 ? run_wide<EPI_QKV, true, true>(a, stream)
+                         : run<224, EPI_QKV, true, false>(a, stream);
     }
     if (a.d_out % 112 == 0)
       return pooled ? run<112, EPI_QKV, true, true>(a, stream)
@@ -679,17 +680,23 @@ hiera_status launch_tc_gemm(int epi, const TcGemmArgs& a, cudaStream_t stream) {
   }
   if (epi == EPI_GELU) {
     if (!a.ln_fold) return HIERA_ERR_INVALID_ARG;
-    if (a.N % 224 == 0)
-      return g_option(HIERA_OPT_GEMM_PAIR) ? run_pair<EPI_GELU, true>(a, stream)
-                                           : run<224, EPI_GELU, true, false>(a, stream);
+    if (a.N % 224 == 0) {
+      const int mode = g_option(HIERA_OPT_GEMM224);
+      return mode == 1   ? run_wide<EPI_GELU, true, false>(a, stream)
+             : mode == 2 ? run_wide<EPI_GELU, true, true>(a, stream)
+                         : run<224, EPI_GELU, true, false>(a, stream);
+    }
     if (a.N % 112 == 0) return run<112, EPI_GELU, true, false>(a, stream);
     return HIERA_ERR_SHAPE;
   }
   if (a.ln_fold) return HIERA_ERR_INVALID_ARG;
   switch (store_bn(a.N)) {
-    case 224:
-      return g_option(HIERA_OPT_GEMM_PAIR) ? run_pair<EPI_STORE, false>(a, stream)
-                                           : run<224, EPI_STORE, false, false>(a, stream);
+    case 224: {
+      const int mode = g_option(HIERA_OPT_GEMM224);
+      return mode == 1   ? run_wide<EPI_STORE, false, false>(a, stream)
+             : mode == 2 ? run_wide<EPI_STORE, false, true>(a, stream)
+                         : run<224, EPI_STORE, false, false>(a, stream);
+    }
     case 128: return run<128, EPI_STORE, false, false>(a, stream);
     case 112: return run<112, EPI_STORE, false, false>(a, stream);
     case 64: return run<64, EPI_STORE, false, false>(a, stream);
