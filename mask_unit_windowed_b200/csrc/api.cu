@@ -230,6 +230,7 @@ hiera_status attention_half_unfused(const Geom& g, const uint8_t* packed, const 
   const long long rows = (long long)g.B * g.tokens, qrows = (long long)g.B * g.Nq;
   // (a3-a6, a8 folded) norm1 + qkv (+ transition proj) with window scatter and q / r pooling
   TcGemmArgs a{};
+  a.w_static = 1;  // packed block weights
   a.M = (int)rows;
   a.N = g.N1;
   a.K = g.d_in;
@@ -268,6 +269,7 @@ hiera_status attention_half_unfused(const Geom& g, const uint8_t* packed, const 
   HIERA_TRY(launch_attention(at, st));
   // (a9) attention proj + residual
   TcGemmArgs pj{};
+  pj.w_static = 1;  // packed block weights
   pj.M = (int)qrows;
   pj.N = g.d_out;
   pj.K = g.d_out;
@@ -342,6 +344,7 @@ hiera_status forward_bf16(const Geom& g, const uint8_t* packed, const void* x, v
   }
   // (a10, a11) norm2 + fc1 + GELU
   TcGemmArgs f1{};
+  f1.w_static = 1;  // packed block weights
   f1.M = (int)qrows;
   f1.N = g.hid;
   f1.K = g.d_out;
@@ -358,6 +361,7 @@ hiera_status forward_bf16(const Geom& g, const uint8_t* packed, const void* x, v
   HIERA_TRY(launch_tc_gemm(EPI_GELU, f1, st));
   // (a12) fc2 + residual
   TcGemmArgs f2{};
+  f2.w_static = 1;  // packed block weights
   f2.M = (int)qrows;
   f2.N = g.d_out;
   f2.K = g.hid;

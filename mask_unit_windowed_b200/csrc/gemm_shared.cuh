@@ -31,6 +31,7 @@ struct KParams {
   int stats_parts;
   float2* stats_out;       // STORE: [M][stats_out_parts] partials of the output, or nullptr
   int stats_out_parts;
+  int w_static;            // W may be read before the wait for the previous kernel
 };
 
 constexpr int cmin(int a, int b) { return a < b ? a : b; }

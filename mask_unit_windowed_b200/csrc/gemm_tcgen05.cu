@@ -122,6 +122,18 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Packed weights are written by no kernel this one can overlap: the producer requests the
+  // first stages' W tiles before it waits for the previous kernel (whose output is A)
+  const int npre = (p.w_static && (int)blockIdx.x < num_tiles) ? cmin(STAGES, kblocks) : 0;
+  if (warp == 0 && npre > 0) {
+    const int nt0 = (int)blockIdx.x - ((int)blockIdx.x / n_tiles) * n_tiles;
+    for (int i = 0; i < npre; ++i) {
+      if (lane == 0) mbar_arrive_expect_tx(&full[i], C::STAGE_BYTES);
+      __syncwarp();
+      if (lane == ((2 * i + 1) & 7))
+        tma_load_2d(smem + i * C::STAGE_BYTES + C::A_BYTES, &tmB, &full[i], i * BK, nt0 * BN);
+    }
+  }
   griddep_wait();  // everything below reads or writes data of earlier kernels
   griddep_launch_dependents();
 
@@ -130,6 +142,7 @@ __global__ void __launch_bounds__(320, 1)
     // One thread's TMA loads complete one after another, so the loads of consecutive
     // stages are issued by different lanes (A and B of a stage by two lanes, rotating over
     // 8 lanes); every lane walks the same stage sequence and waits on the same barriers.
+    // The first npre stages' B tiles (and their barriers' byte counts) are in flight already.
     int s = 0;
     uint32_t ph = 0;
     long long issued = 0;
@@ -138,12 +151,13 @@ __global__ void __launch_bounds__(320, 1)
     for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
       const int mt = tile / n_tiles, nt = tile - (tile / n_tiles) * n_tiles;
       for (int kb = 0; kb < kblocks; ++kb) {
-        if (!warp_wait(&empty[s], ph ^ 1u, p.limit_ns, p.status, abort_flag)) {
+        const bool pre = issued < npre;  // (the first tile's first stages: ring not yet wrapped)
+        if (!pre && !warp_wait(&empty[s], ph ^ 1u, p.limit_ns, p.status, abort_flag)) {
           ok = false;
           break;
         }
         uint8_t* sa = smem + s * C::STAGE_BYTES;
-        if (lane == 0) mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
+        if (lane == 0 && !pre) mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
         __syncwarp();
         if (lane == rr) {
           if (POOLED) {
@@ -161,7 +175,8 @@ __global__ void __launch_bounds__(320, 1)
             tma_load_2d(sa, &tmA, &full[s], kb * BK, mt * BM);
           }
         }
-        if (lane == rr + 1) tma_load_2d(sa + C::A_BYTES, &tmB, &full[s], kb * BK, nt * BN);
+        if (lane == rr + 1 && !pre)
+          tma_load_2d(sa + C::A_BYTES, &tmB, &full[s], kb * BK, nt * BN);
         rr = (rr + 2) & 7;
         ++issued;
         if (++s == STAGES) {
@@ -606,6 +621,7 @@ hiera_status run(const TcGemmArgs& a, cudaStream_t stream) {
   p.stats_parts = a.stats_parts;
   p.stats_out = static_cast<float2*>(a.stats_out);
   p.stats_out_parts = a.stats_out_parts;
+  p.w_static = a.w_static;
 
   auto kern = tc_gemm_kernel<BN, EPI, FOLD, POOLED>;
   if (!ensure_smem_attr(reinterpret_cast<const void*>(kern), C::SMEM_BYTES)) return HIERA_ERR_CUDA;

@@ -54,6 +54,9 @@ struct TcGemmArgs {
   int tokens, nW, heads, d_out, Tq, Tkv;
   int pooled;             // 1: rows n, n+T/4, n+T/2, n+3T/4 of each image loaded together and
                           //    q / r columns max-pooled over them (q_stride 4)
+  int w_static;           // 1: W is never written by a kernel this launch can overlap (packed
+                          //    weights), so its first stages are requested before the wait for
+                          //    the previous kernel
 };
 
 hiera_status launch_tc_gemm(int epi, const TcGemmArgs& a, cudaStream_t stream);
