@@ -567,6 +567,22 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     if rank != 0:
         return
+    clock_rec = clocks.record()
+    if dom_key[0].startswith("attention"):
+        # The attention kernels are bound by their exponentials rather than the tensor pipe:
+        # one ex2.approx per score (B x heads x Tq x Tkv = GFLOP / (4 x 56) per launch) on the
+        # SM's MUFU unit, taken as 16 results per clock per SM (the rate the CUDA programming
+        # guide tables give for exp2 on recent compute capabilities), 148 SMs at the median
+        # SM clock of the timed region.
+        sms = torch.cuda.get_device_properties(local_rank).multi_processor_count
+        mhz = (clock_rec or {}).get("sm_mhz") or 1965.0
+        exps = dom_key[1] * 1e9 / (4 * 56)
+        ach = exps / (roofline["ms_per_launch"] * 1e-3)
+        peak = 16.0 * sms * mhz * 1e6
+        roofline["mufu_context"] = {"exp_per_launch": exps, "achieved_exp_per_s": ach,
+                                    "peak_exp_per_s": peak, "frac": ach / peak,
+                                    "peak_basis": "16 ex2 per clock per SM x SMs x median SM "
+                                                  "clock (assumed rate, not measured)"}
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         v, n = oracle_images_per_s(20.0, 3, 0)
@@ -603,7 +619,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "e2e": e2e,
         "unroll_reroll_hbm": reroll_hbm,
         "extra_workloads": extra,
-        "clocks": clocks.record(),
+        "clocks": clock_rec,
         "gpu_launches": n_launches * replays * args.steps,
         "launches_per_forward": n_launches,
         "per_launch": [[n, round(fl / 1e9, 3), round(ms * 1e3, 2)]

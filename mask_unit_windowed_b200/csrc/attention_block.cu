@@ -262,6 +262,20 @@ __global__ void __launch_bounds__(320, 1)
     }
     for (int i = threadIdx.x - 64; i < FD; i += 256) c_bo[i] = __ldg(p.bias_o + i);
     named_bar_sync(1, 256);
+    // the norm1 partials of this thread's row are loaded a tile ahead
+    auto tok_of = [&](int tt) -> long long {
+      const int tile = (int)blockIdx.x + tt * (int)gridDim.x;
+      const int b = tile / pairs, w0 = 2 * (tile - b * pairs);
+      return (long long)b * p.N + (long long)jr * p.nW + w0 + par;
+    };
+    float2 part[8];
+    auto load_parts = [&](int tt) {
+      const float2* sp = p.stats_in + tok_of(tt) * p.stats_parts;
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        part[j] = j < p.stats_parts ? __ldg(sp + j) : make_float2(0.f, 0.f);
+    };
+    if (n_local > 0) load_parts(0);
     for (int t = 0; t < n_local; ++t) {
       const int tile = (int)blockIdx.x + t * (int)gridDim.x;
       const int b = tile / pairs, w0 = 2 * (tile - b * pairs);
@@ -270,7 +284,8 @@ __global__ void __launch_bounds__(320, 1)
       uint8_t* xq = smem + F_OFF_X;  // q (written over x)
       uint8_t* om = smem + F_OFF_K;  // the merged heads (written over k)
       float fa = 1.f, fb = 0.f;
-      ln_fold_coeffs(p.stats_in + tok * p.stats_parts, p.stats_parts, FD, p.ln_eps, fa, fb);
+      ln_merge_parts(part, p.stats_parts, FD, p.ln_eps, fa, fb);
+      if (t + 1 < n_local) load_parts(t + 1);
       // ---- 2. q, k, v of head hs: fold, bf16, operand tiles
       if (!warp_wait(qkv_done, ph, p.limit_ns, p.status, abort_flag)) break;
       tc_fence_after();
@@ -376,8 +391,17 @@ __global__ void __launch_bounds__(320, 1)
         tc_fence_before();
         mbar_arrive(proj_read);
         float v[56];
+        // the proj bias of this column half, four per 16-byte shared-memory load (every lane
+        // reads the same address: one broadcast per load; 56 hs floats is 16-byte aligned)
+        const float4* bo4 = reinterpret_cast<const float4*>(c_bo + 56 * hs);
 #pragma unroll
-        for (int i = 0; i < 56; ++i) v[i] = __uint_as_float(rr[i]) + c_bo[56 * hs + i];
+        for (int g = 0; g < 14; ++g) {
+          const float4 b4 = bo4[g];
+          v[4 * g + 0] = __uint_as_float(rr[4 * g + 0]) + b4.x;
+          v[4 * g + 1] = __uint_as_float(rr[4 * g + 1]) + b4.y;
+          v[4 * g + 2] = __uint_as_float(rr[4 * g + 2]) + b4.z;
+          v[4 * g + 3] = __uint_as_float(rr[4 * g + 3]) + b4.w;
+        }
 #pragma unroll
         for (int g = 0; g < 7; ++g) {
           v[8 * g + 0] += bf16_lo(res[g].x);
@@ -404,13 +428,16 @@ __global__ void __launch_bounds__(320, 1)
           v[8 * g + 7] = bf16_hi(pk.w);
         }
         if (p.stats_out != nullptr) {
-          float s = 0.f;
+          // (mean, M2) of the 56 stored values, four interleaved accumulators per sum so the
+          // additions are not one serial chain
+          float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int i = 0; i < 56; ++i) s += v[i];
-          const float mean = s * (1.f / 56.f);
-          float m2 = 0.f;
+          for (int i = 0; i < 56; ++i) s4[i & 3] += v[i];
+          const float mean = ((s4[0] + s4[1]) + (s4[2] + s4[3])) * (1.f / 56.f);
+          float q4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int i = 0; i < 56; ++i) m2 = fmaf(v[i] - mean, v[i] - mean, m2);
+          for (int i = 0; i < 56; ++i) q4[i & 3] = fmaf(v[i] - mean, v[i] - mean, q4[i & 3]);
+          const float m2 = (q4[0] + q4[1]) + (q4[2] + q4[3]);
           p.stats_out[tok * 2 + hs] = make_float2(mean, m2);
         }
       }
