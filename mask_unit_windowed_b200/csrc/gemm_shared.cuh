@@ -32,6 +32,7 @@ struct KParams {
   float2* stats_out;       // STORE: [M][stats_out_parts] partials of the output, or nullptr
   int stats_out_parts;
   int w_static;            // W may be read before the wait for the previous kernel
+  int qkv_tma;             // q / k / v rows leave through TMA tensor stores (global attention)
 };
 
 constexpr int cmin(int a, int b) { return a < b ? a : b; }

@@ -56,7 +56,7 @@ struct Cfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STG_BYTES = 8 * 32 * 128;  // per epilogue warp: 32 rows x 128 B staging
   static constexpr int STAGES =
-      cmin(8, (227 * 1024 - 1024 - 256 - EPI_WARPS * BN * 4 - 128 - STG_BYTES) / STAGE_BYTES);
+      cmin(8, (227 * 1024 - 1024 - 256 - EPI_WARPS * BN * 4 - 1024 - STG_BYTES) / STAGE_BYTES);
   static constexpr int ACC_STRIDE = BN <= 128 ? 128 : 256;
   static constexpr int TMEM_COLS = 2 * ACC_STRIDE;
   static constexpr int HALF = BN / 2;                    // columns per epilogue thread
@@ -65,7 +65,9 @@ struct Cfg {
   // per epilogue warp: colsum and colconst (fp32) of its half of the tile's columns
   static constexpr int CONST_OFF = BAR_OFF + 256;
   static constexpr int CONST_BYTES = EPI_WARPS * 2 * (BN / 2) * 4;
-  static constexpr int STG_OFF = (CONST_OFF + CONST_BYTES + 127) / 128 * 128;
+  // (1024-byte aligned: a staged block of 128-byte swizzled rows is the layout of a
+  // SWIZZLE_128B tensor store)
+  static constexpr int STG_OFF = (CONST_OFF + CONST_BYTES + 1023) / 1024 * 1024;
   static constexpr int SMEM_BYTES = STG_OFF + STG_BYTES + 1024;
   static_assert(B_BYTES % 1024 == 0, "W tile must keep 1024-byte alignment");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128");
@@ -77,7 +79,8 @@ struct Cfg {
 template <int BN, int EPI, bool FOLD, bool POOLED>
 __global__ void __launch_bounds__(320, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmO, const KParams p) {
+                   const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmK2,
+                   const __grid_constant__ CUtensorMap tmV2, const KParams p) {
   using C = Cfg<BN>;
   constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
@@ -430,7 +433,8 @@ __global__ void __launch_bounds__(320, 1)
         // ---- stage the packed row in shared memory: XOR-swizzled 16-byte chunks for the
         // copy-out below, or dense rows of CH values for a TMA store
         uint8_t* stg = stg_all + (ew << 12);
-        if (TmaOut<EPI>::value) {
+        const bool qkv_tma = EPI == EPI_QKV && !POOLED && p.qkv_tma;
+        if (TmaOut<EPI>::value || qkv_tma) {
           if (lane == 0) tma_store_wait_read();  // the previous chunk's store has read stg
           __syncwarp();
         }
@@ -475,6 +479,20 @@ __global__ void __launch_bounds__(320, 1)
           __syncwarp();
           if (lane == 0)
             tma_store_2d(&tmO, stg, n0 + c_begin + c, (int)(m - rt + quarter * 32));
+          continue;
+        }
+        if (qkv_tma) {
+          // global attention (one window): the warp's 32 consecutive tokens of one image are 32
+          // consecutive 128-byte rows of the head's q / k / v block, stored by one TMA tensor
+          // store straight from the 128-byte-swizzled staging rows
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && valid) {
+            const int h = (n0 - which * p.d_out + c_begin + c) / 56;
+            const int T = which == 0 ? p.Tq : p.Tkv;
+            const CUtensorMap* map = which == 0 ? &tmO : (which == 1 ? &tmK2 : &tmV2);
+            tma_store_2d(map, stg, 0, (b * p.heads + h) * T + tok);
+          }
           continue;
         }
         __syncwarp();
@@ -527,7 +545,8 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
     // every TMA store of this warp has completed before the CTA exits
-    if (TmaOut<EPI>::value && lane == 0) tma_store_wait_all();
+    if ((TmaOut<EPI>::value || (EPI == EPI_QKV && !POOLED && p.qkv_tma)) && lane == 0)
+      tma_store_wait_all();
   }
 
   tc_fence_before();
@@ -589,11 +608,25 @@ hiera_status run(const TcGemmArgs& a, cudaStream_t stream) {
     cuuint32_t box[2] = {BK, BN};
     if (!encode_bf16(&tmB, a.W, 2, dims, str, box)) return HIERA_ERR_CUDA;
   }
-  CUtensorMap tmO = tmA;  // unused by the q / k / v scatter
+  CUtensorMap tmO = tmA, tmK2 = tmA, tmV2 = tmA;  // (unused unless set below)
   if (TmaOut<EPI>::value &&
       !encode_bf16_plain(&tmO, a.out, (cuuint64_t)a.N, (cuuint64_t)a.M, (cuuint64_t)a.ldo * 2,
                          (cuuint32_t)C::CH, 32))
     return HIERA_ERR_CUDA;
+  // q / k / v of a global-attention block (one window, no pooling, 32-token groups inside one
+  // image) leave through TMA tensor stores: [rows of 64 channels] maps, 32-row boxes
+  int qkv_tma = 0;
+  if (EPI == EPI_QKV && !POOLED && a.nW == 1 && a.tokens % 32 == 0 && a.Tq == a.tokens &&
+      a.Tkv == a.tokens && a.N == 3 * a.d_out) {
+    const cuuint64_t rows = (cuuint64_t)(a.M / a.tokens) * a.heads * a.tokens;
+    const cuuint64_t dims[2] = {64, rows};
+    const cuuint64_t str[1] = {128};
+    const cuuint32_t box[2] = {64, 32};
+    if (!encode_bf16(&tmO, a.q, 2, dims, str, box) || !encode_bf16(&tmK2, a.k, 2, dims, str, box) ||
+        !encode_bf16(&tmV2, a.v, 2, dims, str, box))
+      return HIERA_ERR_CUDA;
+    qkv_tma = 1;
+  }
   KParams p;
   p.M = a.M;
   p.N = a.N;
@@ -622,6 +655,7 @@ hiera_status run(const TcGemmArgs& a, cudaStream_t stream) {
   p.stats_out = static_cast<float2*>(a.stats_out);
   p.stats_out_parts = a.stats_out_parts;
   p.w_static = a.w_static;
+  p.qkv_tma = qkv_tma;
 
   auto kern = tc_gemm_kernel<BN, EPI, FOLD, POOLED>;
   if (!ensure_smem_attr(reinterpret_cast<const void*>(kern), C::SMEM_BYTES)) return HIERA_ERR_CUDA;
@@ -632,7 +666,7 @@ hiera_status run(const TcGemmArgs& a, cudaStream_t stream) {
   if (grid > tiles) grid = tiles;
   profile_mark(EPI == EPI_QKV ? K_GEMM_QKV : (EPI == EPI_GELU ? K_GEMM_GELU : K_GEMM_STORE),
                stream);
-  launch_k(kern, dim3(grid), dim3(320), C::SMEM_BYTES, stream, tmA, tmB, tmO, p);
+  launch_k(kern, dim3(grid), dim3(320), C::SMEM_BYTES, stream, tmA, tmB, tmO, tmK2, tmV2, p);
   return cudaGetLastError() == cudaSuccess ? HIERA_OK : HIERA_ERR_CUDA;
 }
 

@@ -759,6 +759,8 @@ hiera_status run_wide(const TcGemmArgs& a, cudaStream_t stream) {
   p.stats_parts = a.stats_parts;
   p.stats_out = static_cast<float2*>(a.stats_out);
   p.stats_out_parts = a.stats_out_parts;
+  p.w_static = 0;
+  p.qkv_tma = 0;
 
   auto kern = PAIR ? tc_gemm_pair_kernel<EPI, FOLD> : tc_gemm_wide_kernel<EPI, FOLD>;
   if (!ensure_smem_attr(reinterpret_cast<const void*>(kern), C::SMEM)) return HIERA_ERR_CUDA;
