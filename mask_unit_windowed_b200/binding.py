@@ -459,15 +459,19 @@ class BackbonePipeline:
     download the four features into pinned host memory. Uploads, the forward calls and
     downloads go to three streams with two device buffer sets, so the copies of a batch
     overlap the compute of its neighbours; the forwards themselves run one after another on
-    the compute stream (they share one workspace).
+    the compute stream (they share one workspace). With graph=True (the default) each
+    buffer set's hiera_backbone_forward call is captured once in a CUDA graph and replayed,
+    so the host does not re-enqueue its launches for every batch.
 
         pipe = BackbonePipeline(desc, packed)
         pipe.run(host_images, host_features)   # lists of pinned CPU tensors, one per batch
         pipe.synchronize()
     """
 
-    def __init__(self, desc: BackboneDesc, packed: torch.Tensor, device=None):
+    def __init__(self, desc: BackboneDesc, packed: torch.Tensor, device=None, graph=True):
         self.desc, self.packed = desc, packed
+        self.graph = graph
+        self._graphs = [None, None]
         dev = packed.device if device is None else torch.device(device)
         shape = (desc.B, desc.img, desc.img, 4)
         self.imgs = [torch.empty(shape, dtype=desc.dtype, device=dev) for _ in range(2)]
@@ -502,8 +506,21 @@ class BackbonePipeline:
             self.s_comp.wait_event(ev_in[i])
             if self._count >= 2:
                 self.s_comp.wait_event(ev_out[i])   # feature buffers i were downloaded
-            backbone_forward(self.desc, self.packed, self.imgs[i], feats=self.feats[i],
-                             workspace=self.ws, stream=self.s_comp)
+            if not self.graph:
+                backbone_forward(self.desc, self.packed, self.imgs[i], feats=self.feats[i],
+                                 workspace=self.ws, stream=self.s_comp)
+            else:
+                if self._graphs[i] is None:
+                    # first use of buffer set i: capture its forward (on the compute
+                    # stream, after the upload it waits for), then replay it
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g, stream=self.s_comp):
+                        backbone_forward(self.desc, self.packed, self.imgs[i],
+                                         feats=self.feats[i], workspace=self.ws,
+                                         stream=self.s_comp)
+                    self._graphs[i] = g
+                with torch.cuda.stream(self.s_comp):
+                    self._graphs[i].replay()
             ev_comp[i].record(self.s_comp)
             self.s_out.wait_event(ev_comp[i])
             with torch.cuda.stream(self.s_out):

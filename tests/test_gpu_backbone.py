@@ -147,16 +147,18 @@ def test_transition_block_65536_tokens_sampled_rows():
     assert rel_l2(got, ref) <= 1e-2
 
 
-def test_backbone_pipeline_host_to_host_bitwise():
+@pytest.mark.parametrize("graph", [True, False])
+def test_backbone_pipeline_host_to_host_bitwise(graph):
     """binding.BackbonePipeline (uploads, forward and downloads of consecutive batches
-    overlapping on three streams) gives every batch the same features as a plain call."""
+    overlapping on three streams; the forwards replayed from CUDA graphs or enqueued call by
+    call) gives every batch the same features as a plain call."""
     img, B = 64, 2
     p = syn.backbone_params(71, img, dtype="bf16", affine="random")
     desc = hb.BackboneDesc(B=B, img=img)
     packed = hb.backbone_pack(desc, weights_dev(p, "bf16"))
     hosts = [torch.from_numpy(syn.image(71 + k, B, img, dtype="bf16")).to(torch.bfloat16)
              .pin_memory() for k in range(5)]
-    pipe = hb.BackbonePipeline(desc, packed)
+    pipe = hb.BackbonePipeline(desc, packed, graph=graph)
     outs = [pipe.host_feature_buffers() for _ in hosts]
     pipe.run(hosts, outs)
     pipe.synchronize()
