@@ -27,13 +27,18 @@
 //   warp 1      TMEM owner (all 512 columns), fc1 tcgen05.mma issuer (one thread)
 //   warp 2      fc2 tcgen05.mma issuer (one thread)
 //   warps 3-18  epilogue, four warps per TMEM lane quarter (a warp reaches only the lanes
-//               32 (warp % 4) .. + 31): 16 columns of every hidden chunk each, and one
-//               56-column piece of the output each (D = 224; for D = 112 the first two
-//               warps of each quarter). Four warps per scheduler hide the latency of the
-//               GELU chains; the per-row LayerNorm partial of each 112-column half of a
-//               D = 224 row is merged from its two pieces in shared memory, in the order
-//               the stand-alone GEMM's epilogue merges them.
-// TMEM: output accumulator at column 0 (D columns), fc1 chunk accumulators from ACC1_COL.
+//               32 (warp % 4) .. + 31).
+//               D = 224: all sixteen take 16 columns of every hidden chunk and one 56-column
+//               piece of the output each; the per-row LayerNorm partial of each 112-column
+//               half is merged from its two pieces in shared memory, in the order the
+//               stand-alone GEMM's epilogue merges them.
+//               D = 112: two roles. Eight hidden warps take 32 columns of every hidden
+//               chunk; eight output warps take one 56-column piece of the output, from a
+//               double-buffered output accumulator, so a tile's output epilogue (bias,
+//               residual, rounding, partials, store) runs while the next tile's hidden
+//               chunks are produced.
+// TMEM: output accumulator(s) at column 0 (D = 112: 0 and 128), fc1 chunk accumulators from
+// ACC1_COL.
 #include "common.cuh"
 #include "internal.h"
 
@@ -55,7 +60,11 @@ struct MlpCfg {
   static constexpr int NX = D <= 128 ? 2 : 1;   // x tile buffers
   static constexpr int NB = 4;                  // fc1 accumulators in TMEM
   static constexpr int NH = 2;                  // hidden chunk buffers in shared memory
-  static constexpr int S1 = D <= 128 ? 4 : 2;   // W1 chunk ring
+  // D = 112: the epilogue warps split into eight hidden warps (32 columns of every hidden
+  // chunk each) and eight output warps (one 56-column piece each) with a double-buffered
+  // output accumulator, so a tile's output epilogue overlaps the next tile's hidden chunks
+  static constexpr bool SPLIT = D <= 128;
+  static constexpr int S1 = D <= 128 ? 3 : 2;   // W1 chunk ring
   static constexpr int S2 = D <= 128 ? 4 : 2;   // W2 chunk ring
   static constexpr int LAG = D <= 128 ? 2 : 1;  // W2 chunk j is loaded after W1 chunk j + LAG
   static constexpr int X_BYTES = KB1 * BM * 128;
@@ -66,16 +75,21 @@ struct MlpCfg {
   static constexpr int H_OFF = X_OFF + NX * X_BYTES;
   static constexpr int W1_OFF = H_OFF + NH * H_BYTES;
   static constexpr int W2_OFF = W1_OFF + S1 * W1_BYTES;
-  static constexpr int CONST_OFF = W2_OFF + S2 * W2_BYTES;   // colsum1, colconst1 [HID]
+  static constexpr int STG_OFF = W2_OFF + S2 * W2_BYTES;     // SPLIT: output staging
+  static constexpr int STG_BYTES = SPLIT ? 8 * 2048 : 0;     // (8 warps x 16 rows x 128 B)
+  static constexpr int CONST_OFF = STG_OFF + STG_BYTES;      // colsum1, colconst1 [HID]
   static constexpr int BAR_OFF = CONST_OFF + 2 * HID * 4;
   static constexpr int SMEM_BYTES = BAR_OFF + 512 + 2 * BM * 8 + 1024;  // + alignment slack
-  static constexpr int ACC1_COL = D <= 128 ? 128 : 256;
+  static constexpr int ACC1_COL = D <= 128 ? 256 : 256;  // (SPLIT: outputs at 0 and 128)
+  static constexpr int HID_THREADS = SPLIT ? EPI_THREADS / 2 : EPI_THREADS;  // hidden chunks
   static constexpr int TMEM_COLS = 512;
   static constexpr int PIECES = D / 56;                      // 56-column output pieces per row
   static constexpr int FIN_THREADS = PIECES * 4 * 32;        // threads that read the output
   static constexpr int XCH_OFF = BAR_OFF + 512;              // float2 [2][128] partial exchange
   static_assert(D % 56 == 0 && D % 16 == 0, "D is a multiple of 112");
-  static_assert(ACC1_COL >= D && ACC1_COL + NB * HC <= TMEM_COLS, "TMEM plan");
+  static_assert(ACC1_COL >= (SPLIT ? 128 + D : D) && ACC1_COL + NB * HC <= TMEM_COLS,
+                "TMEM plan");
+  static_assert(!SPLIT || PIECES == 2, "split roles: two output pieces per row");
   static_assert(LAG < S2 && LAG < NB, "issue lag within the rings");
   static_assert(W2_BYTES % 1024 == 0 && X_BYTES % 1024 == 0, "operand alignment");
   static_assert(NH * H_BYTES >= EPI_WARPS * 2048, "output staging aliases the hidden buffers");
@@ -147,9 +161,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* a1_empty = a1_full + C::NB;     // [NB]
   uint64_t* h_full = a1_empty + C::NB;      // [NH]
   uint64_t* h_empty = h_full + C::NH;       // [NH]
-  uint64_t* a2_full = h_empty + C::NH;
-  uint64_t* a2_empty = a2_full + 1;
-  uint64_t* drain = a2_empty + 1;
+  uint64_t* a2_full = h_empty + C::NH;      // [2] (one used unless SPLIT)
+  uint64_t* a2_empty = a2_full + 2;         // [2]
+  uint64_t* drain = a2_empty + 2;
   uint64_t* drain2 = drain + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain2 + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -172,14 +186,16 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int i = 0; i < C::NB; ++i) {
       mbar_init(&a1_full[i], 1);
-      mbar_init(&a1_empty[i], EPI_THREADS);
+      mbar_init(&a1_empty[i], C::HID_THREADS);
     }
     for (int i = 0; i < C::NH; ++i) {
-      mbar_init(&h_full[i], EPI_THREADS);
+      mbar_init(&h_full[i], C::HID_THREADS);
       mbar_init(&h_empty[i], 1);
     }
-    mbar_init(a2_full, 1);
-    mbar_init(a2_empty, C::FIN_THREADS);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&a2_full[i], 1);
+      mbar_init(&a2_empty[i], C::FIN_THREADS);
+    }
     mbar_init(drain, 1);
     mbar_init(drain2, 1);
     *abort_flag = 0;
@@ -344,8 +360,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++t) {
         for (int i = 0; i < C::NC; ++i) {
           const int hb = (int)(hc % C::NH);
-          // the output accumulator is free once the previous tile's epilogue read it
-          if ((i == 0 && !mbar_wait(a2_empty, (t & 1u) ^ 1u, p.limit_ns, p.status, abort_flag)) ||
+          // the output accumulator is free once the epilogue read it (SPLIT: the one of tile
+          // t - 2; otherwise of tile t - 1)
+          const int ob = C::SPLIT ? (int)(t & 1u) : 0;
+          const uint32_t oph = C::SPLIT ? ((t >> 1) & 1u) : (t & 1u);
+          if ((i == 0 && !mbar_wait(&a2_empty[ob], oph ^ 1u, p.limit_ns, p.status, abort_flag)) ||
               !mbar_wait(&h_full[hb], (uint32_t)((hc / C::NH) & 1), p.limit_ns, p.status,
                          abort_flag) ||
               !mbar_wait(&w2_full[s2], ph2, p.limit_ns, p.status, abort_flag)) {
@@ -355,13 +374,14 @@ __global__ void __launch_bounds__(THREADS, 1)
           tc_fence_after();
           const uint64_t hdesc = desc_advance(hdesc0, (uint32_t)(hb * C::H_BYTES));
           const uint64_t w2desc = desc_advance(w2desc0, (uint32_t)(s2 * C::W2_BYTES));
+          const uint32_t dout = tmem + (uint32_t)(ob * 128);
           if (i == 0)
-            tc_mma_bf16_k<false>(tmem, hdesc, w2desc, IDESC2);
+            tc_mma_bf16_k<false>(dout, hdesc, w2desc, IDESC2);
           else
-            tc_mma_bf16_k<true>(tmem, hdesc, w2desc, IDESC2);
+            tc_mma_bf16_k<true>(dout, hdesc, w2desc, IDESC2);
 #pragma unroll
           for (int kk = 1; kk < HC / 16; ++kk)
-            tc_mma_bf16_k<true>(tmem, desc_advance(hdesc, 32u * kk), desc_advance(w2desc, 32u * kk),
+            tc_mma_bf16_k<true>(dout, desc_advance(hdesc, 32u * kk), desc_advance(w2desc, 32u * kk),
                                 IDESC2);
           tc_commit(&w2_empty[s2]);
           tc_commit(&h_empty[hb]);
@@ -371,11 +391,161 @@ __global__ void __launch_bounds__(THREADS, 1)
             ph2 ^= 1u;
           }
         }
-        if (ok) tc_commit(a2_full);
+        if (ok) tc_commit(&a2_full[C::SPLIT ? (int)(t & 1u) : 0]);
       }
       if (!ok) *abort_flag = 1;
       tc_commit(drain2);
       mbar_wait(drain2, 0, p.limit_ns, p.status);
+    }
+  } else if constexpr (C::SPLIT) {
+    // ------------------------------------------------------------ epilogue, split roles
+    const int ew = warp - 3;
+    const int quarter = warp & 3;  // TMEM lanes 32 quarter .. + 31
+    const int cg = ew >> 2;        // 0, 1: output piece cg; 2, 3: hidden column half cg - 2
+    const int rt = quarter * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    bool ok = true;
+    if (cg >= 2) {
+      // ---- hidden chunks: fc1 accumulator -> LayerNorm fold -> GELU -> bf16 operand,
+      //      32 columns of every chunk per warp
+      const int hh = cg - 2;
+      uint32_t a1 = 0, hc = 0;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const long long m = (long long)tile * BM + rt;
+        float fa = 1.f, fb = 0.f;
+        if (m < p.M)
+          ln_fold_coeffs(p.stats_in + m * p.stats_parts, p.stats_parts, D, p.ln_eps, fa, fb);
+        for (int j = 0; j < C::NC; ++j) {
+          const int b = (int)(a1 % C::NB);
+          if (!warp_wait(&a1_full[b], (uint32_t)((a1 / C::NB) & 1), p.limit_ns, p.status,
+                         abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          uint32_t r[32];
+          tmem_load<32>(tmem + lane_base + (uint32_t)(C::ACC1_COL + b * HC + hh * 32), r);
+          tc_fence_before();
+          mbar_arrive(&a1_empty[b]);
+          ++a1;
+          const float4* cs4 = reinterpret_cast<const float4*>(c_sum + j * HC + hh * 32);
+          const float4* cc4 = reinterpret_cast<const float4*>(c_const + j * HC + hh * 32);
+          uint4 pk[4];
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const float4 s0 = cs4[2 * g], s1 = cs4[2 * g + 1];
+            const float4 k0 = cc4[2 * g], k1 = cc4[2 * g + 1];
+            const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+            const float kv[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+            float v[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              v[e] = gelu_fast(fmaf(fa, __uint_as_float(r[8 * g + e]), fmaf(fb, sv[e], kv[e])));
+            pk[g] = pack8(v);
+          }
+          const int hb = (int)(hc % C::NH);
+          if (!warp_wait(&h_empty[hb], (uint32_t)((hc / C::NH) & 1) ^ 1u, p.limit_ns, p.status,
+                         abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint8_t* hrow = sH + hb * C::H_BYTES + rt * 128;
+#pragma unroll
+          for (int g = 0; g < 4; ++g)
+            *reinterpret_cast<uint4*>(hrow + (((hh * 4 + g) ^ (rt & 7)) << 4)) = pk[g];
+          fence_proxy_async_smem();
+          mbar_arrive(&h_full[hb]);
+          ++hc;
+        }
+      }
+    } else {
+      // ---- output piece [56 cg, 56 cg + 56) of every tile: + b2 + residual, bf16, the
+      //      LayerNorm partial of this 56-column half, coalesced store; the accumulator of
+      //      tile t is buffer t & 1, so the next tile's fc2 runs meanwhile
+      const int c0 = cg * 56;
+      uint8_t* stg = smem + C::STG_OFF + (ew << 11);  // 16 rows x 128 B, this warp's own
+      uint32_t t = 0;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++t) {
+        const long long m = (long long)tile * BM + rt;
+        const bool row_ok = m < p.M;
+        uint4 res[7];
+        const bf16* xrow = p.x + m * D + c0;
+#pragma unroll
+        for (int i = 0; i < 7; ++i)
+          res[i] = row_ok ? __ldg(reinterpret_cast<const uint4*>(xrow) + i) : make_uint4(0u, 0u, 0u, 0u);
+        const int ob = (int)(t & 1u);
+        if (!warp_wait(&a2_full[ob], (uint32_t)((t >> 1) & 1u), p.limit_ns, p.status,
+                       abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const float4* b4 = reinterpret_cast<const float4*>(p.bias2 + c0);
+        const uint32_t obase = tmem + lane_base + (uint32_t)(ob * 128 + c0);
+        {
+          uint32_t r[32];
+          tmem_load<32>(obase, r);
+          out_groups<0, 4>(r, res, b4);
+        }
+        {
+          uint32_t r[24];
+          tc_ld_32x32b_x16(obase + 32, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+          tc_ld_32x32b_x8(obase + 48, *reinterpret_cast<uint32_t(*)[8]>(&r[16]));
+          tc_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 24; ++i) asm volatile("" : "+r"(r[i]));
+          tc_fence_before();
+          mbar_arrive(&a2_empty[ob]);
+          out_groups<4, 3>(r, res, b4);
+        }
+        if (p.stats_out != nullptr && row_ok) {
+          // statistics of the values as stored, in column order
+          float sm = 0.f;
+#pragma unroll
+          for (int g = 0; g < 7; ++g)
+            sm = (((((((sm + bf16_lo(res[g].x)) + bf16_hi(res[g].x)) + bf16_lo(res[g].y)) +
+                     bf16_hi(res[g].y)) + bf16_lo(res[g].z)) + bf16_hi(res[g].z)) +
+                  bf16_lo(res[g].w)) + bf16_hi(res[g].w);
+          const float st_mean = sm * (1.f / 56.f);
+          float st_m2 = 0.f;
+#pragma unroll
+          for (int g = 0; g < 7; ++g) {
+            const uint32_t w4[4] = {res[g].x, res[g].y, res[g].z, res[g].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float lo = bf16_lo(w4[e]) - st_mean, hi = bf16_hi(w4[e]) - st_mean;
+              st_m2 = fmaf(lo, lo, st_m2);
+              st_m2 = fmaf(hi, hi, st_m2);
+            }
+          }
+          p.stats_out[m * 2 + cg] = make_float2(st_mean, st_m2);
+        }
+        // staging: 16 rows at a time, then 8 lanes per row, 4 rows per store instruction
+        const unsigned long long my_dst = reinterpret_cast<unsigned long long>(p.out + m * D + c0);
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          if ((lane >> 4) == hh) {
+            const int sr = lane & 15;
+#pragma unroll
+            for (int g = 0; g < 7; ++g)
+              *reinterpret_cast<uint4*>(stg + (sr << 7) + ((g ^ (sr & 7)) << 4)) = res[g];
+          }
+          __syncwarp();
+#pragma unroll
+          for (int it = 0; it < 4; ++it) {
+            const int sr = it * 4 + (lane >> 3), ch = lane & 7;
+            const int row = hh * 16 + sr;
+            const unsigned long long dst = __shfl_sync(0xffffffffu, my_dst, row);
+            const int wr = __shfl_sync(0xffffffffu, row_ok ? 1 : 0, row);
+            if (wr && ch < 7) {
+              const uint4 val =
+                  *reinterpret_cast<const uint4*>(stg + (sr << 7) + ((ch ^ (sr & 7)) << 4));
+              *reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(dst) + ch * 8) = val;
+            }
+          }
+          __syncwarp();
+        }
+      }
     }
   } else {
     // ------------------------------------------------------------ epilogue
