@@ -371,7 +371,8 @@ HIERA_API hiera_status hiera_debug_timeout_probe(int limit_us, hiera_stream_t st
 
 /* Self-test of the tensor-core path's GELU: y[i] = GELU(x[i]) for n fp32 device values,
  * computed exactly as the fc1 epilogue does (x * sigmoid of a fitted odd polynomial for
- * logit(Phi(x)); |error| <= 3e-5 against x Phi(x)). */
+ * logit(Phi(x)), the sigmoid evaluated through tanh.approx; |error| <= 4e-5 against
+ * x Phi(x)). */
 HIERA_API hiera_status hiera_debug_gelu(const float* x, float* y, int n, hiera_stream_t stream);
 
 #ifdef __cplusplus

@@ -40,9 +40,11 @@ def test_workspace_too_small_rejected():
 
 
 def test_tensor_core_path_gelu_within_error_bound():
-    """The fc1 epilogue's GELU (x * sigmoid of a fitted odd polynomial for logit(Phi);
-    fit error 2.55e-5 at most, evaluated in fp32 with ex2.approx / rcp.approx) against the
-    fp64 definition x * Phi(x): |error| <= 3e-5 everywhere, 0 at x = 0, x to 2^-22 for
+    """The fc1 epilogue's GELU (x * sigmoid of a fitted odd polynomial g for logit(Phi),
+    the sigmoid taken as (1 + tanh(g / 2)) / 2 with tanh.approx.f32) against the fp64
+    definition x * Phi(x). The fit alone is within 2.53e-5 (fp64 evaluation); tanh.approx
+    adds at most |x| / 2 times its own error, 7.9e-6 as measured on sm_100a over [-12, 12].
+    So |error| <= 2.6e-5 + 4e-6 |x| and <= 4e-5 everywhere, 0 at x = 0, x to 2^-22 for
     x >= 6 and within 2e-8 of 0 for x <= -6."""
     import numpy as np
     from oracle import unrolled as U
@@ -50,7 +52,8 @@ def test_tensor_core_path_gelu_within_error_bound():
     y = hb.debug_gelu(torch.from_numpy(x).cuda()).cpu().numpy().astype(np.float64)
     ref = U.gelu(x.astype(np.float64))
     err = np.abs(y - ref)
-    assert np.all(err <= 3e-5), float(err.max())
+    assert np.all(err <= 2.6e-5 + 4e-6 * np.abs(x)), float((err - 4e-6 * np.abs(x)).max())
+    assert np.all(err <= 4e-5), float(err.max())
     assert y[np.argmin(np.abs(x))] == 0.0
     hi = x >= 6
     assert np.all(np.abs(y[hi] - x[hi]) <= 2.0 ** -22 * x[hi])
