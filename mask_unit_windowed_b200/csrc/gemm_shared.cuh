@@ -11,6 +11,31 @@ namespace hiera {
 constexpr int BM = 128;  // accumulator rows per CTA (TMEM lanes)
 constexpr int BK = 64;   // K per pipeline stage (one 128-byte swizzle row of bf16)
 
+// Division by a divisor fixed at launch as a multiply-high, an add and two shifts (Granlund
+// and Montgomery, "Division by invariant integers using multiplication", 1994: the variant
+// for any divisor d >= 1 with an m' of 32 bits, exact for every 32-bit unsigned dividend).
+// The per-tile row bookkeeping of the epilogue divides by the token count, the pooled token
+// count, the window count and the tile count; done with the hardware-less integer divide
+// sequence each costs a long dependent chain on the epilogue warps' critical path.
+struct FastDiv {
+  uint32_t d, mul, sh1, sh2;
+  __device__ __forceinline__ uint32_t div(uint32_t n) const {
+    const uint32_t t = __umulhi(mul, n);
+    return (t + ((n - t) >> sh1)) >> sh2;
+  }
+};
+
+inline FastDiv make_fastdiv(uint32_t d) {
+  FastDiv f{};
+  f.d = d < 1 ? 1 : d;
+  uint32_t l = 0;  // ceil(log2 d)
+  while ((1ull << l) < f.d) ++l;
+  f.mul = (uint32_t)(((1ull << 32) * ((1ull << l) - f.d)) / f.d + 1);
+  f.sh1 = l < 1 ? l : 1;
+  f.sh2 = l > 1 ? l - 1 : 0;
+  return f;
+}
+
 struct KParams {
   int M, N, K;
   const float* colsum;
@@ -32,8 +57,28 @@ struct KParams {
   float2* stats_out;       // STORE: [M][stats_out_parts] partials of the output, or nullptr
   int stats_out_parts;
   int w_static;            // W may be read before the wait for the previous kernel
-  int qkv_tma;             // q / k / v rows leave through TMA tensor stores (global attention)
+  int qkv_tma;             // q / k / v rows leave through TMA tensor stores: QKV_TMA_*
+  FastDiv fd_ntiles;       // N / BN column tiles
+  FastDiv fd_tokens;       // tokens per image
+  FastDiv fd_per;          // pooled tokens per image (tokens / 4)
+  FastDiv fd_nw;           // windows per image
+  FastDiv fd_dout;         // d_out (which of q / k / v / r a column tile holds)
 };
+
+// How the q / k / v head rows of the qkv GEMM leave (KParams::qkv_tma). A warp's 32 staged
+// rows (one head, 128 bytes each, in the 128-byte swizzle) are one TMA box when
+//   QKV_TMA_GLOBAL : one window: 32 consecutive tokens are 32 consecutive rows of the head's
+//                    [T][64] block (map [64][B * heads * T], box 64 x 32);
+//   QKV_TMA_WINDOWS: mask-unit windows, no pooling, 32 | nW: tokens j nW + w, w = w0..w0+31,
+//                    are row j of 32 consecutive windows (map [64][T][heads][B nW], box
+//                    64 x 1 x 1 x 32);
+//   QKV_TMA_POOLED : the pooled tiles of a transition (8 pooled positions x 4 candidates per
+//                    warp), k and v only, 8 | nW and nW | tokens / 4: candidate c of pooled
+//                    position np is token c tokens / 4 + np, i.e. in-window index
+//                    c (tokens / 4 nW) + np / nW of window np mod nW (map
+//                    [64][tokens / 4 nW][4][heads][B nW], box 64 x 1 x 4 x 1 x 8).
+// Otherwise (QKV_TMA_NONE) the lanes copy the staged rows out.
+constexpr int QKV_TMA_NONE = 0, QKV_TMA_GLOBAL = 1, QKV_TMA_WINDOWS = 2, QKV_TMA_POOLED = 3;
 
 constexpr int cmin(int a, int b) { return a < b ? a : b; }
 
@@ -63,6 +108,24 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void*
       "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
           reinterpret_cast<uint64_t>(map)),
       "r"(smem_u32(smem_src)), "r"(c0), "r"(c1)
+      : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, const void* smem_src, int c0,
+                                             int c1, int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(smem_src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void tma_store_5d(const CUtensorMap* map, const void* smem_src, int c0,
+                                             int c1, int c2, int c3, int c4) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5, %6}], [%1];" ::
+          "l"(reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(smem_src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
       : "memory");
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }

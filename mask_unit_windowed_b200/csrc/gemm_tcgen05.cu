@@ -129,7 +129,7 @@ __global__ void __launch_bounds__(320, 1)
   // first stages' W tiles before it waits for the previous kernel (whose output is A)
   const int npre = (p.w_static && (int)blockIdx.x < num_tiles) ? cmin(STAGES, kblocks) : 0;
   if (warp == 0 && npre > 0) {
-    const int nt0 = (int)blockIdx.x - ((int)blockIdx.x / n_tiles) * n_tiles;
+    const int nt0 = (int)blockIdx.x - (int)p.fd_ntiles.div(blockIdx.x) * n_tiles;
     for (int i = 0; i < npre; ++i) {
       if (lane == 0) mbar_arrive_expect_tx(&full[i], C::STAGE_BYTES);
       __syncwarp();
@@ -152,7 +152,7 @@ __global__ void __launch_bounds__(320, 1)
     bool ok = true;
     int rr = 0;
     for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-      const int mt = tile / n_tiles, nt = tile - (tile / n_tiles) * n_tiles;
+      const int mt = (int)p.fd_ntiles.div((uint32_t)tile), nt = tile - mt * n_tiles;
       for (int kb = 0; kb < kblocks; ++kb) {
         const bool pre = issued < npre;  // (the first tile's first stages: ring not yet wrapped)
         if (!pre && !warp_wait(&empty[s], ph ^ 1u, p.limit_ns, p.status, abort_flag)) {
@@ -167,7 +167,8 @@ __global__ void __launch_bounds__(320, 1)
             const int per = p.tokens >> 2;
             if (per >= 32) {
               const int pm0 = mt * 32;
-              tma_load_4d(sa, &tmA, &full[s], kb * BK, 0, pm0 % per, pm0 / per);
+              const int bb = (int)p.fd_per.div((uint32_t)pm0);
+              tma_load_4d(sa, &tmA, &full[s], kb * BK, 0, pm0 - bb * per, bb);
             } else {
               // 32 / per whole images per tile, one box of per x 4 rows each
               for (int i = 0; i < 32 / per; ++i)
@@ -255,11 +256,11 @@ __global__ void __launch_bounds__(320, 1)
     // global row of this thread's TMEM lane in a tile (pooled tiles interleave 4 rows per
     // pooled token)
     auto row_of = [&](int tile) -> long long {
-      const int mt = tile / n_tiles;
+      const int mt = (int)p.fd_ntiles.div((uint32_t)tile);
       if (POOLED) {
         const int per = p.tokens >> 2;
         const int pm = mt * 32 + (rt >> 2);
-        const int bb = pm / per, npp = pm - (pm / per) * per;
+        const int bb = (int)p.fd_per.div((uint32_t)pm), npp = pm - bb * per;
         return (long long)bb * p.tokens + (rt & 3) * per + npp;
       }
       return (long long)mt * BM + rt;
@@ -284,7 +285,7 @@ __global__ void __launch_bounds__(320, 1)
     float* col_const = col_sum + HALF;
     float nsum[CPL], nconst[CPL];
     auto load_consts = [&](int tile) {
-      const int c0 = (tile - (tile / n_tiles) * n_tiles) * BN + c_begin;
+      const int c0 = (tile - (int)p.fd_ntiles.div((uint32_t)tile) * n_tiles) * BN + c_begin;
 #pragma unroll
       for (int k = 0; k < CPL; ++k) {
         const int i = lane + 32 * k;
@@ -305,7 +306,7 @@ __global__ void __launch_bounds__(320, 1)
       load_consts(blockIdx.x);
     }
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-      const int mt = tile / n_tiles, nt = tile - (tile / n_tiles) * n_tiles;
+      const int mt = (int)p.fd_ntiles.div((uint32_t)tile), nt = tile - mt * n_tiles;
       const int n0 = nt * BN;
       // row bookkeeping
       const long long m = row_of(tile);
@@ -313,12 +314,12 @@ __global__ void __launch_bounds__(320, 1)
       if (POOLED) {
         const int per = p.tokens >> 2;
         const int pm = mt * 32 + (rt >> 2);
-        b = pm / per;
+        b = (int)p.fd_per.div((uint32_t)pm);
         np = pm - b * per;
         tok = (rt & 3) * per + np;
       } else if (EPI == EPI_QKV) {
-        b = (int)(m / p.tokens);
-        tok = (int)(m - (long long)b * p.tokens);
+        b = (int)p.fd_tokens.div((uint32_t)m);  // (M < 2^31)
+        tok = (int)m - b * p.tokens;
       }
       const bool row_ok = m < p.M;
       // residual of this row / half, in flight while the mainloop runs
@@ -356,7 +357,7 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_after();
       const uint32_t tbase = tmem + (uint32_t)(acc * C::ACC_STRIDE) +
                              ((uint32_t)(quarter * 32) << 16) + (uint32_t)c_begin;
-      const int which = (EPI == EPI_QKV) ? n0 / p.d_out : 0;
+      const int which = (EPI == EPI_QKV) ? (int)p.fd_dout.div((uint32_t)n0) : 0;
       const bool pool_this = POOLED && (which == 0 || which == 3);
       const bool writer = row_ok && (!pool_this || (rt & 3) == 0);
       float st_mean = 0.f, st_m2 = 0.f;  // running statistics of the stored half row
@@ -421,7 +422,7 @@ __global__ void __launch_bounds__(320, 1)
           } else {
             const int h = colw / 56;
             const int tt = pool_this ? np : tok;
-            const int w = tt % p.nW, j = tt / p.nW;
+            const int j = (int)p.fd_nw.div((uint32_t)tt), w = tt - j * p.nW;
             const int T = which == 0 ? p.Tq : p.Tkv;
             bf16* base = which == 0 ? p.q : (which == 1 ? p.k : p.v);
             dst_row = base + ((((long long)b * p.nW + w) * p.heads + h) * T + j) * 64;
@@ -433,8 +434,10 @@ __global__ void __launch_bounds__(320, 1)
         // ---- stage the packed row in shared memory: XOR-swizzled 16-byte chunks for the
         // copy-out below, or dense rows of CH values for a TMA store
         uint8_t* stg = stg_all + (ew << 12);
-        const bool qkv_tma = EPI == EPI_QKV && !POOLED && p.qkv_tma;
-        if (TmaOut<EPI>::value || qkv_tma) {
+        // q / k / v rows by TMA tensor store (pooled tiles: k and v only)
+        const bool qkv_tma = EPI == EPI_QKV && p.qkv_tma != QKV_TMA_NONE &&
+                             (!POOLED || which == 1 || which == 2);
+        if (TmaOut<EPI>::value || (EPI == EPI_QKV && p.qkv_tma != QKV_TMA_NONE)) {
           if (lane == 0) tma_store_wait_read();  // the previous chunk's store has read stg
           __syncwarp();
         }
@@ -482,16 +485,24 @@ __global__ void __launch_bounds__(320, 1)
           continue;
         }
         if (qkv_tma) {
-          // global attention (one window): the warp's 32 consecutive tokens of one image are 32
-          // consecutive 128-byte rows of the head's q / k / v block, stored by one TMA tensor
-          // store straight from the 128-byte-swizzled staging rows
+          // the warp's 32 staged 128-byte rows (128-byte swizzle) are one box of the head's
+          // q / k / v layout (QKV_TMA_* in gemm_shared.cuh); lane 0's row is the box origin
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0 && valid) {
             const int h = (n0 - which * p.d_out + c_begin + c) / 56;
-            const int T = which == 0 ? p.Tq : p.Tkv;
             const CUtensorMap* map = which == 0 ? &tmO : (which == 1 ? &tmK2 : &tmV2);
-            tma_store_2d(map, stg, 0, (b * p.heads + h) * T + tok);
+            if (POOLED) {
+              // k / v of a transition: lane 0 holds candidate 0 of pooled position np
+              const int jj = (int)p.fd_nw.div((uint32_t)np);
+              tma_store_5d(map, stg, 0, jj, 0, h, b * p.nW + np - jj * p.nW);
+            } else if (p.qkv_tma == QKV_TMA_WINDOWS) {
+              const int j = (int)p.fd_nw.div((uint32_t)tok);
+              tma_store_4d(map, stg, 0, j, h, b * p.nW + tok - j * p.nW);
+            } else {
+              const int T = which == 0 ? p.Tq : p.Tkv;
+              tma_store_2d(map, stg, 0, (b * p.heads + h) * T + tok);
+            }
           }
           continue;
         }
@@ -545,7 +556,7 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
     // every TMA store of this warp has completed before the CTA exits
-    if ((TmaOut<EPI>::value || (EPI == EPI_QKV && !POOLED && p.qkv_tma)) && lane == 0)
+    if ((TmaOut<EPI>::value || (EPI == EPI_QKV && p.qkv_tma != QKV_TMA_NONE)) && lane == 0)
       tma_store_wait_all();
   }
 
@@ -613,19 +624,40 @@ hiera_status run(const TcGemmArgs& a, cudaStream_t stream) {
       !encode_bf16_plain(&tmO, a.out, (cuuint64_t)a.N, (cuuint64_t)a.M, (cuuint64_t)a.ldo * 2,
                          (cuuint32_t)C::CH, 32))
     return HIERA_ERR_CUDA;
-  // q / k / v of a global-attention block (one window, no pooling, 32-token groups inside one
-  // image) leave through TMA tensor stores: [rows of 64 channels] maps, 32-row boxes
-  int qkv_tma = 0;
-  if (EPI == EPI_QKV && !POOLED && a.nW == 1 && a.tokens % 32 == 0 && a.Tq == a.tokens &&
-      a.Tkv == a.tokens && a.N == 3 * a.d_out) {
-    const cuuint64_t rows = (cuuint64_t)(a.M / a.tokens) * a.heads * a.tokens;
-    const cuuint64_t dims[2] = {64, rows};
-    const cuuint64_t str[1] = {128};
-    const cuuint32_t box[2] = {64, 32};
-    if (!encode_bf16(&tmO, a.q, 2, dims, str, box) || !encode_bf16(&tmK2, a.k, 2, dims, str, box) ||
-        !encode_bf16(&tmV2, a.v, 2, dims, str, box))
-      return HIERA_ERR_CUDA;
-    qkv_tma = 1;
+  // q / k / v head rows leave through TMA tensor stores where a warp's 32 rows form one box
+  // (QKV_TMA_* in gemm_shared.cuh); every map covers the whole [B][nW][heads][T][64] layout
+  int qkv_tma = QKV_TMA_NONE;
+  if (EPI == EPI_QKV && a.tokens % 32 == 0 && a.nW >= 1 && a.tokens % a.nW == 0) {
+    const int B = a.M / a.tokens;
+    const int T = a.tokens / a.nW;  // keys per window
+    const cuuint64_t bw = (cuuint64_t)B * a.nW;
+    if (!POOLED && a.nW == 1 && a.Tq == T && a.Tkv == T && a.N == 3 * a.d_out) {
+      const cuuint64_t dims[2] = {64, bw * a.heads * T};
+      const cuuint64_t str[1] = {128};
+      const cuuint32_t box[2] = {64, 32};
+      if (!encode_bf16(&tmO, a.q, 2, dims, str, box) ||
+          !encode_bf16(&tmK2, a.k, 2, dims, str, box) || !encode_bf16(&tmV2, a.v, 2, dims, str, box))
+        return HIERA_ERR_CUDA;
+      qkv_tma = QKV_TMA_GLOBAL;
+    } else if (!POOLED && a.nW % 32 == 0 && a.Tq == T && a.Tkv == T && a.N == 3 * a.d_out) {
+      const cuuint64_t dims[4] = {64, (cuuint64_t)T, (cuuint64_t)a.heads, bw};
+      const cuuint64_t str[3] = {128, (cuuint64_t)T * 128, (cuuint64_t)a.heads * T * 128};
+      const cuuint32_t box[4] = {64, 1, 1, 32};
+      if (!encode_bf16(&tmO, a.q, 4, dims, str, box) ||
+          !encode_bf16(&tmK2, a.k, 4, dims, str, box) || !encode_bf16(&tmV2, a.v, 4, dims, str, box))
+        return HIERA_ERR_CUDA;
+      qkv_tma = QKV_TMA_WINDOWS;
+    } else if (POOLED && a.nW % 8 == 0 && (a.tokens / 4) % a.nW == 0 && (a.tokens / 4) % 8 == 0 &&
+               a.Tkv == T) {
+      const int TP = a.tokens / 4 / a.nW;  // in-window rows per pooling candidate
+      const cuuint64_t dims[5] = {64, (cuuint64_t)TP, 4, (cuuint64_t)a.heads, bw};
+      const cuuint64_t str[4] = {128, (cuuint64_t)TP * 128, (cuuint64_t)T * 128,
+                                 (cuuint64_t)a.heads * T * 128};
+      const cuuint32_t box[5] = {64, 1, 4, 1, 8};
+      if (!encode_bf16(&tmK2, a.k, 5, dims, str, box) || !encode_bf16(&tmV2, a.v, 5, dims, str, box))
+        return HIERA_ERR_CUDA;
+      qkv_tma = QKV_TMA_POOLED;
+    }
   }
   KParams p;
   p.M = a.M;
@@ -656,6 +688,11 @@ hiera_status run(const TcGemmArgs& a, cudaStream_t stream) {
   p.stats_out_parts = a.stats_out_parts;
   p.w_static = a.w_static;
   p.qkv_tma = qkv_tma;
+  p.fd_ntiles = make_fastdiv((uint32_t)(a.N / BN));
+  p.fd_tokens = make_fastdiv((uint32_t)a.tokens);
+  p.fd_per = make_fastdiv((uint32_t)(a.tokens / 4));
+  p.fd_nw = make_fastdiv((uint32_t)a.nW);
+  p.fd_dout = make_fastdiv((uint32_t)a.d_out);
 
   auto kern = tc_gemm_kernel<BN, EPI, FOLD, POOLED>;
   if (!ensure_smem_attr(reinterpret_cast<const void*>(kern), C::SMEM_BYTES)) return HIERA_ERR_CUDA;

@@ -761,6 +761,11 @@ hiera_status run_wide(const TcGemmArgs& a, cudaStream_t stream) {
   p.stats_out_parts = a.stats_out_parts;
   p.w_static = 0;
   p.qkv_tma = 0;
+  p.fd_ntiles = make_fastdiv((uint32_t)(a.N / 224));
+  p.fd_tokens = make_fastdiv((uint32_t)a.tokens);
+  p.fd_per = make_fastdiv((uint32_t)(a.tokens / 4));
+  p.fd_nw = make_fastdiv((uint32_t)a.nW);
+  p.fd_dout = make_fastdiv((uint32_t)a.d_out);
 
   auto kern = PAIR ? tc_gemm_pair_kernel<EPI, FOLD> : tc_gemm_wide_kernel<EPI, FOLD>;
   if (!ensure_smem_attr(reinterpret_cast<const void*>(kern), C::SMEM)) return HIERA_ERR_CUDA;
