@@ -275,6 +275,7 @@ __global__ void __launch_bounds__(320, 1)
       for (int j = 0; j < 8; ++j)
         part[j] = j < p.stats_parts ? __ldg(sp + j) : make_float2(0.f, 0.f);
     };
+    const LnConsts lnc = ln_consts(p.stats_parts, FD);
     if (n_local > 0) load_parts(0);
     for (int t = 0; t < n_local; ++t) {
       const int tile = (int)blockIdx.x + t * (int)gridDim.x;
@@ -284,7 +285,7 @@ __global__ void __launch_bounds__(320, 1)
       uint8_t* xq = smem + F_OFF_X;  // q (written over x)
       uint8_t* om = smem + F_OFF_K;  // the merged heads (written over k)
       float fa = 1.f, fb = 0.f;
-      ln_merge_parts(part, p.stats_parts, FD, p.ln_eps, fa, fb);
+      ln_merge_parts(part, p.stats_parts, lnc, p.ln_eps, fa, fb);
       if (t + 1 < n_local) load_parts(t + 1);
       // ---- 2. q, k, v of head hs: fold, bf16, operand tiles
       if (!warp_wait(qkv_done, ph, p.limit_ns, p.status, abort_flag)) break;

@@ -402,12 +402,22 @@ __device__ __forceinline__ uint4 pack8(const float* v) {
 // LayerNorm of a row of K values from P partial (mean, M2) pairs over K / P values each
 // (Chan et al. merge with equal counts): LN(x) W^T + b = fa (x W'^T) + fb s + c with
 // fa = rstd, fb = -mean rstd (s, c the packed column constants of the folded weight).
-__device__ __forceinline__ void ln_merge_parts(const float2 (&part)[8], int P, int K, float eps,
-                                               float& fa, float& fb) {
+// Constants of the LayerNorm of a row of K values kept as P partials (P a power of two, so
+// 1 / P is exact): computed once per kernel, so that merging a row's partials needs no
+// division on the epilogue's critical path.
+struct LnConsts {
+  float inv_p, k_over_p, inv_k;
+};
+__device__ __forceinline__ LnConsts ln_consts(int P, int K) {
+  return {1.0f / (float)P, (float)(K / P), 1.0f / (float)K};
+}
+
+__device__ __forceinline__ void ln_merge_parts(const float2 (&part)[8], int P, const LnConsts& c,
+                                               float eps, float& fa, float& fb) {
   float mean = 0.f;
 #pragma unroll
   for (int j = 0; j < 8; ++j) mean += part[j].x;
-  mean /= (float)P;
+  mean *= c.inv_p;
   float m2 = 0.f, dev2 = 0.f;
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
@@ -417,17 +427,18 @@ __device__ __forceinline__ void ln_merge_parts(const float2 (&part)[8], int P, i
       dev2 = fmaf(dlt, dlt, dev2);
     }
   }
-  m2 = fmaf((float)(K / P), dev2, m2);
-  fa = rsqrtf(m2 / (float)K + eps);
+  m2 = fmaf(c.k_over_p, dev2, m2);
+  fa = rsqrtf(fmaf(m2, c.inv_k, eps));
   fb = -mean * fa;
 }
 
-__device__ __forceinline__ void ln_fold_coeffs(const float2* __restrict__ sp, int P, int K,
-                                               float eps, float& fa, float& fb) {
+__device__ __forceinline__ void ln_fold_coeffs(const float2* __restrict__ sp, int P,
+                                               const LnConsts& c, float eps, float& fa,
+                                               float& fb) {
   float2 part[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) part[j] = j < P ? __ldg(sp + j) : make_float2(0.f, 0.f);
-  ln_merge_parts(part, P, K, eps, fa, fb);
+  ln_merge_parts(part, P, c, eps, fa, fb);
 }
 
 // ------------------------------------------------------------------ Unroll map

@@ -301,6 +301,7 @@ __global__ void __launch_bounds__(320, 1)
     };
     // the store epilogue (residual prefetch already holds many registers, few tiles per
     // CTA) loads them at the tile's start instead
+    const LnConsts lnc = ln_consts(p.stats_parts, p.K);
     if ((int)blockIdx.x < num_tiles && FOLD) {
       load_parts(blockIdx.x);
       load_consts(blockIdx.x);
@@ -336,7 +337,7 @@ __global__ void __launch_bounds__(320, 1)
       }
       // LayerNorm statistics of this row, merged from the producer's partials
       float fa = 1.f, fb = 0.f;  // v = fa * acc + fb * colsum + colconst
-      if (FOLD && row_ok) ln_merge_parts(part, p.stats_parts, p.K, p.ln_eps, fa, fb);
+      if (FOLD && row_ok) ln_merge_parts(part, p.stats_parts, lnc, p.ln_eps, fa, fb);
       // this warp's column constants of this tile into its slots (loaded a tile ahead)
       if (!FOLD) load_consts(tile);
       __syncwarp();  // every lane is done with the last tile's

@@ -205,6 +205,7 @@ __device__ __forceinline__ void wide_epilogue(const KParams& p, const CUtensorMa
       if (PAIR) st_cluster_u32(cluster_addr((const void*)bb.abort_flag, rank ^ 1u), 1u);
     }
   };
+  const LnConsts lnc = ln_consts(p.stats_parts, p.K);
   for (int tile = cl; tile < num_tiles; tile += n_cl, ++tcount) {
     const int mt = tile / n_tiles, nt = tile - (tile / n_tiles) * n_tiles;
     const int n0 = nt * WBN;
@@ -220,7 +221,7 @@ __device__ __forceinline__ void wide_epilogue(const KParams& p, const CUtensorMa
     // LayerNorm coefficients of this row (v = fa * acc + fb * colsum + colconst) and this
     // warp's column constants
     float fa = 1.f, fb = 0.f;
-    if (FOLD && row_ok) ln_fold_coeffs(p.stats_in + m * p.stats_parts, p.stats_parts, p.K,
+    if (FOLD && row_ok) ln_fold_coeffs(p.stats_in + m * p.stats_parts, p.stats_parts, lnc,
                                        p.ln_eps, fa, fb);
     __syncwarp();  // every lane is done with the last tile's constants
 #pragma unroll

@@ -410,11 +410,22 @@ __global__ void __launch_bounds__(THREADS, 1)
       //      32 columns of every chunk per warp
       const int hh = cg - 2;
       uint32_t a1 = 0, hc = 0;
+      // the norm2 partials of this thread's row are loaded a tile ahead
+      float2 part[8];
+      auto load_parts = [&](int tile) {
+        const long long m = (long long)tile * BM + rt;
+        const float2* sp = p.stats_in + (m < p.M ? m : 0) * p.stats_parts;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          part[j] = j < p.stats_parts ? __ldg(sp + j) : make_float2(0.f, 0.f);
+      };
+      const LnConsts lnc = ln_consts(p.stats_parts, D);
+      if ((int)blockIdx.x < num_tiles) load_parts(blockIdx.x);
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         const long long m = (long long)tile * BM + rt;
         float fa = 1.f, fb = 0.f;
-        if (m < p.M)
-          ln_fold_coeffs(p.stats_in + m * p.stats_parts, p.stats_parts, D, p.ln_eps, fa, fb);
+        if (m < p.M) ln_merge_parts(part, p.stats_parts, lnc, p.ln_eps, fa, fb);
+        if (tile + (int)gridDim.x < num_tiles) load_parts(tile + gridDim.x);
         for (int j = 0; j < C::NC; ++j) {
           const int b = (int)(a1 % C::NB);
           if (!warp_wait(&a1_full[b], (uint32_t)((a1 / C::NB) & 1), p.limit_ns, p.status,
@@ -561,8 +572,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       const long long m = (long long)tile * BM + rt;
       const bool row_ok = m < p.M;
       float fa = 1.f, fb = 0.f;
+      // (the constants are formed here rather than kept live across the loop: registers)
       if (ok && row_ok)
-        ln_fold_coeffs(p.stats_in + m * p.stats_parts, p.stats_parts, D, p.ln_eps, fa, fb);
+        ln_fold_coeffs(p.stats_in + m * p.stats_parts, p.stats_parts,
+                       ln_consts(p.stats_parts, D), p.ln_eps, fa, fb);
       // ---- hidden chunks: fc1 accumulator -> LayerNorm fold -> GELU -> bf16 operand
       for (int j = 0; j < C::NC && ok; ++j) {
         const int b = (int)(a1 % C::NB);
