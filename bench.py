@@ -351,6 +351,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     hb.set_option(hb.OPT_FUSED_MLP, 1 if args.mlp == "fused" else 0)
     hb.set_option(hb.OPT_PDL, 1 if args.pdl == "on" else 0)
     hb.set_option(hb.OPT_FUSED_ATTN, 1 if args.attn == "fused" else 0)
+    hb.set_option(hb.OPT_SPLIT_BATCH, 1 if args.split == "on" else 0)
     if args.gemm224 != "default":
         hb.set_option(hb.OPT_GEMM224, {"8warp": hb.GEMM224_EIGHT_WARPS,
                                        "16warp": hb.GEMM224_SIXTEEN_WARPS,
@@ -391,6 +392,10 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             forward()
     torch.cuda.synchronize()
     n_launches = prof.count
+    # (the profiled forward runs as one batch: the library does not split a batch while a
+    # launch profile is open; split, each half makes the same launches)
+    split = args.split == "on" and B >= 2
+    launches_per_forward = n_launches * (2 if split else 1)
 
     # ---- warm-up steps (one forward each), which also size a step: R forwards such that
     # the K timed steps last about a second
@@ -468,7 +473,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                 "traffic_unit": "bytes per launch (dram__bytes_read.sum + "
                                 "dram__bytes_write.sum, one ncu capture of this kernel)",
                 "timing": "per-launch CUDA events in an instrumented graph of the same "
-                          "forward, mean of 5 replays, L2 flushed before each"}
+                          "forward run as one batch on one stream (the events bracket "
+                          "consecutive launches), mean of 5 replays, L2 flushed before each"}
     shape_list = sorted(({"kernel": k[0], "gflop_per_launch": k[1], **{kk: vv for kk, vv in
                           e.items() if kk not in ("kind",)}} for k, e in shapes.items()),
                         key=lambda e: -e["ms"])
@@ -603,6 +609,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                          "forward's working set (138 MB of weights + activations) exceeds L2",
                    "timing": "CUDA-graph replay of the library launches, per-step CUDA events",
                    "mlp": args.mlp, "pdl": args.pdl, "attn": args.attn,
+                   "split_batch": (f"two concurrent halves of {(B + 1) // 2} and {B // 2} "
+                                   "images on two streams" if split else "off"),
                    "gemm224": ["8warp", "16warp", "pair"][hb.get_option(hb.OPT_GEMM224)]},
         "ms_per_forward": ms_per_forward,
         "timed_seconds": total_ms / 1e3,
@@ -620,8 +628,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "unroll_reroll_hbm": reroll_hbm,
         "extra_workloads": extra,
         "clocks": clock_rec,
-        "gpu_launches": n_launches * replays * args.steps,
-        "launches_per_forward": n_launches,
+        "gpu_launches": launches_per_forward * replays * args.steps,
+        "launches_per_forward": launches_per_forward,
         "per_launch": [[n, round(fl / 1e9, 3), round(ms * 1e3, 2)]
                        for (n, ms), (_, fl) in zip(per_launch, flops)],
     }
@@ -651,6 +659,9 @@ def main():
     ap.add_argument("--attn", choices=["fused", "unfused"], default="fused",
                     help="stage-0 attention half (norm1, qkv, attention, proj) as one kernel "
                          "(default) or three")
+    ap.add_argument("--split", choices=["on", "off"], default="on",
+                    help="run each batch as two concurrent halves on two streams (library "
+                         "default) or as one batch")
     ap.add_argument("--gemm224", choices=["default", "8warp", "16warp", "pair"],
                     default="default",
                     help="kernel of the 224-column-tile Linear layers (library default, the "

@@ -276,6 +276,14 @@ HIERA_API hiera_status hiera_patch_embed(const void* img, const void* packed_pat
  * mask_unit_attn_stage2_first: 0 = block 5 global (as the plan's table lists stage 2);
  * 1 = block 5 keeps mask-unit attention (16 keys, 4 pooled queries per unit).
  * Features: feats[s] is NHWC [B, img/2^(s+2), img/2^(s+2), 112*2^s].
+ * hiera_backbone_workspace_bytes is enough for the call as one batch and as two
+ * concurrent halves (HIERA_OPT_SPLIT_BATCH below), whichever the option selects. With
+ * the split, hiera_backbone_forward enqueues images [0, ceil(B/2)) on `stream` and the
+ * rest on a second stream owned by the calling thread (one per device), forked from and
+ * joined back into `stream` with events: the call stays ordered with the caller's work on
+ * `stream` and may be captured into a CUDA graph from it (the second stream joins the
+ * capture). A call is not to be made while a capture begun by the same thread on another
+ * stream is still open.
  * -------------------------------------------------------------------------------- */
 typedef struct {
   int B;
@@ -332,6 +340,11 @@ HIERA_API hiera_status hiera_backbone_forward(const hiera_backbone_desc* desc, c
  *                        (tcgen05.mma.cta_group::2, each SM loading its 128 input rows and
  *                        half of the weight tile) with the sixteen-warp epilogue. All three
  *                        give the same bits.
+ *   HIERA_OPT_SPLIT_BATCH 1 (default): hiera_backbone_forward with B >= 2 runs its images as
+ *                        two concurrent half batches on two streams (each kernel sizes its
+ *                        grid to the SM count; the halves' kernels fill the SMs one chain
+ *                        leaves idle in kernel tails and partial waves). 0: one batch on
+ *                        `stream`. Every image's features are the same bits either way.
  * hiera_set_option returns HIERA_ERR_INVALID_ARG for an unknown option or value (0 or
  * 1; 0 to 2 for HIERA_OPT_GEMM224);
  * hiera_get_option returns the current value (0 for an unknown option).
@@ -341,7 +354,8 @@ typedef enum {
   HIERA_OPT_PDL = 1,
   HIERA_OPT_FUSED_ATTN = 2,
   HIERA_OPT_GEMM224 = 3,
-  HIERA_OPT_COUNT = 4
+  HIERA_OPT_SPLIT_BATCH = 4,
+  HIERA_OPT_COUNT = 5
 } hiera_option;
 HIERA_API hiera_status hiera_set_option(hiera_option opt, int value);
 HIERA_API int hiera_get_option(hiera_option opt);
@@ -354,8 +368,9 @@ HIERA_API int hiera_get_option(hiera_option opt);
  * marked). `events` are cudaEvent_t handles created by the caller with timing enabled.
  * hiera_profile_end() records events[n] on `stream` (n = launches seen, if n <
  * capacity) and returns n, so launch i took elapsed(events[i], events[i+1]) when all
- * launches went to one stream. Works under CUDA-graph stream capture (the records
- * become event nodes). Not thread-safe: one session at a time per process.
+ * launches went to one stream; while a session is open hiera_backbone_forward therefore
+ * does not split its batch (HIERA_OPT_SPLIT_BATCH). Works under CUDA-graph stream capture
+ * (the records become event nodes). Not thread-safe: one session at a time per process.
  * hiera_kernel_name() names a kernel id (static string).
  * -------------------------------------------------------------------------------- */
 HIERA_API hiera_status hiera_profile_begin(void* const* events, int capacity, int* kinds);

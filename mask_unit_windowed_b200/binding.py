@@ -569,6 +569,7 @@ OPT_PDL = 1
 OPT_FUSED_ATTN = 2
 OPT_GEMM224 = 3
 GEMM224_EIGHT_WARPS, GEMM224_SIXTEEN_WARPS, GEMM224_PAIR = 0, 1, 2
+OPT_SPLIT_BATCH = 4
 
 
 def set_option(opt: int, value: int):
@@ -612,6 +613,12 @@ def gemm224(mode: int) -> option:
     CTA per 128 x 224 tile, eight epilogue warps), GEMM224_SIXTEEN_WARPS (one CTA, sixteen
     epilogue warps) or GEMM224_PAIR (a CTA pair per 256 x 224 tile, tcgen05.mma.cta_group::2)."""
     return option(OPT_GEMM224, int(mode))
+
+
+def split_batch(enabled: bool) -> option:
+    """Run a backbone call's images as two concurrent half batches on two streams (True,
+    the default, for B >= 2) or as one batch on the call's stream."""
+    return option(OPT_SPLIT_BATCH, bool(enabled))
 
 
 def pdl(enabled: bool) -> option:

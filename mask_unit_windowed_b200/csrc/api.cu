@@ -559,6 +559,103 @@ BackboneWs backbone_ws_layout(const hiera_backbone_desc* bd, const BlockPlan pla
   return L;
 }
 
+// A call's images are independent, and every kernel of the forward sizes its grid to the SM
+// count: run as two concurrent half batches on two streams, the halves' kernels take the SMs
+// that a single chain of kernels leaves idle in its kernel tails and partial waves
+// (HIERA_OPT_SPLIT_BATCH). The second stream and the fork / join events belong to the
+// calling thread (one set per device), so calls from other threads never share them.
+struct AuxStreams {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+thread_local AuxStreams t_aux[kMaxDev];
+
+// The calling thread's second stream on the current device, created on first use (never
+// inside a stream capture: with `capturing` set and no stream yet, *out stays nullptr and
+// the call runs as one batch). hiera_backbone_pack creates it ahead of time.
+hiera_status aux_streams(AuxStreams** out, bool capturing) {
+  *out = nullptr;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return HIERA_ERR_CUDA;
+  AuxStreams& a = t_aux[dev];
+  if (a.s == nullptr) {
+    if (capturing) return HIERA_OK;
+    if (cudaStreamCreateWithFlags(&a.s, cudaStreamNonBlocking) != cudaSuccess) {
+      a.s = nullptr;
+      return HIERA_ERR_CUDA;
+    }
+    if (cudaEventCreateWithFlags(&a.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&a.join, cudaEventDisableTiming) != cudaSuccess)
+      return HIERA_ERR_CUDA;
+  }
+  *out = &a;
+  return HIERA_OK;
+}
+
+// the two halves of a split batch: images [0, B1) and [B1, B)
+void split_descs(const hiera_backbone_desc* d, hiera_backbone_desc* h1, hiera_backbone_desc* h2) {
+  *h1 = *d;
+  *h2 = *d;
+  h1->B = (d->B + 1) / 2;
+  h2->B = d->B - h1->B;
+}
+
+bool profile_open();
+// (not while a launch profile is open: its events bracket consecutive launches on one stream)
+bool split_applies(const hiera_backbone_desc* d) {
+  return g_option(HIERA_OPT_SPLIT_BATCH) != 0 && d->B >= 2 && !profile_open();
+}
+
+// workspace of a split call: the first half's, then (256-byte aligned) the second half's
+size_t split_ws_bytes(const hiera_backbone_desc* d, size_t* second_off) {
+  hiera_backbone_desc h1, h2;
+  split_descs(d, &h1, &h2);
+  BlockPlan p1[kDepth], p2[kDepth];
+  if (backbone_plan(&h1, p1) != HIERA_OK || backbone_plan(&h2, p2) != HIERA_OK) return 0;
+  const size_t a = up256(backbone_ws_layout(&h1, p1).total);
+  if (second_off != nullptr) *second_off = a;
+  return a + backbone_ws_layout(&h2, p2).total;
+}
+
+// One forward of the backbone for desc->B images, enqueued on one stream.
+hiera_status backbone_run(const hiera_backbone_desc* desc, const BlockPlan plan[kDepth],
+                          const uint8_t* pk, const void* img_nhwc, void* const feats[4],
+                          uint8_t* ws, cudaStream_t st) {
+  const BackbonePack P = backbone_pack_layout(desc, plan);
+  const BackboneWs W = backbone_ws_layout(desc, plan);
+  const int bf = desc->dtype == HIERA_BF16 ? 1 : 0;
+  const int es = bf ? 2 : 4;
+  const int G0 = desc->img / 4;
+  uint8_t* act[2] = {ws + W.act0, ws + W.act1};
+  float2* stp[2] = {(float2*)(ws + W.st0), (float2*)(ws + W.st1)};
+  // (a0-a2) patch embedding + pos_embed + Unroll, fused; in bf16 it also emits the LayerNorm
+  // partials of its output (two 56-channel halves per token) for block 0's norm1
+  HIERA_TRY(launch_patch_embed(img_nhwc, pk + P.patch_w, pk + P.pos, act[0],
+                               bf ? stp[0] : nullptr, desc->B, desc->img, bf, st));
+  int cur = 0, s_idx = 0, parts = 2;
+  for (int i = 0; i < kDepth; ++i) {
+    Geom g;
+    make_geom(&plan[i].d, &g);
+    const uint8_t* bp = pk + P.blocks[i];
+    uint8_t* out = act[cur ^ 1];
+    HIERA_TRY(g.bf16 ? forward_bf16(g, bp, act[cur], out, ws + W.block, st, stp[cur], parts,
+                                    stp[cur ^ 1])
+                     : forward_f32(g, bp, act[cur], out, ws + W.block, st));
+    parts = store_stats_parts(g.d_out);
+    cur ^= 1;
+    if (s_idx < 4 && i == kStageEnds[s_idx]) {
+      // (a13) Reroll the stage output to NHWC
+      const int s = plan[i].stage;
+      const int Gs = G0 >> s;
+      if (launch_permute(false, act[cur], feats[s_idx], desc->B, Gs, kStageDim[s], 3 - s, es,
+                         st) != cudaSuccess)
+        return HIERA_ERR_CUDA;
+      ++s_idx;
+    }
+  }
+  return HIERA_OK;
+}
+
 // Library-owned scratch for hiera_block_forward_noalloc (see include/hiera.h): a static
 // device array, so calls through that entry point allocate nothing. Host code needs the
 // array's device address, looked up once per device with that device current.
@@ -638,6 +735,8 @@ struct ProfileSession {
   int count = 0;
   bool open = false;
 } g_prof;
+
+bool profile_open() { return g_prof.open; }
 }  // namespace
 
 void profile_mark(int kind, cudaStream_t stream) {
@@ -652,7 +751,7 @@ void profile_mark(int kind, cudaStream_t stream) {
 namespace {
 // fused MLP, programmatic dependent launch and fused attention half on; the eight-warp
 // 224-column GEMM
-int g_options[HIERA_OPT_COUNT] = {1, 1, 1, 0};
+int g_options[HIERA_OPT_COUNT] = {1, 1, 1, 0, 1};
 }  // namespace
 
 int g_option(int opt) { return (opt >= 0 && opt < HIERA_OPT_COUNT) ? g_options[opt] : 0; }
@@ -905,6 +1004,14 @@ hiera_status hiera_backbone_pack(const hiera_backbone_desc* desc, const hiera_ba
     if (!weights_aligned(&w->blocks[i])) return HIERA_ERR_ALIGNMENT;
   }
   HIERA_TRY(check_device());
+  {
+    // the calling thread's second stream for split-batch forwards, made here, outside any
+    // capture the forward may later be enqueued in
+    AuxStreams* aux = nullptr;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing((cudaStream_t)stream, &cap) != cudaSuccess) return HIERA_ERR_CUDA;
+    HIERA_TRY(aux_streams(&aux, cap != cudaStreamCaptureStatusNone));
+  }
   const cudaStream_t st = (cudaStream_t)stream;
   uint8_t* p = static_cast<uint8_t*>(packed);
   const int bf = desc->dtype == HIERA_BF16 ? 1 : 0;
@@ -922,7 +1029,9 @@ hiera_status hiera_backbone_pack(const hiera_backbone_desc* desc, const hiera_ba
 size_t hiera_backbone_workspace_bytes(const hiera_backbone_desc* desc) {
   BlockPlan plan[kDepth];
   if (backbone_plan(desc, plan) != HIERA_OK) return 0;
-  return backbone_ws_layout(desc, plan).total;
+  // enough for the call as one batch and as two concurrent halves, whatever the option
+  const size_t whole = backbone_ws_layout(desc, plan).total;
+  return desc->B >= 2 ? std::max(whole, split_ws_bytes(desc, nullptr)) : whole;
 }
 
 hiera_status hiera_backbone_forward(const hiera_backbone_desc* desc, const void* packed,
@@ -938,44 +1047,51 @@ hiera_status hiera_backbone_forward(const hiera_backbone_desc* desc, const void*
   }
   if (!aligned16(packed) || !aligned16(img_nhwc) || !aligned16(workspace))
     return HIERA_ERR_ALIGNMENT;
-  const BackbonePack P = backbone_pack_layout(desc, plan);
-  const BackboneWs W = backbone_ws_layout(desc, plan);
-  if (workspace_bytes < W.total) return HIERA_ERR_WORKSPACE;
-  HIERA_TRY(check_device());
   const cudaStream_t st = (cudaStream_t)stream;
   const uint8_t* pk = static_cast<const uint8_t*>(packed);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const int bf = desc->dtype == HIERA_BF16 ? 1 : 0;
-  const int es = bf ? 2 : 4;
-  const int G0 = desc->img / 4;
-  uint8_t* act[2] = {ws + W.act0, ws + W.act1};
-  float2* stp[2] = {(float2*)(ws + W.st0), (float2*)(ws + W.st1)};
-  // (a0-a2) patch embedding + pos_embed + Unroll, fused; in bf16 it also emits the LayerNorm
-  // partials of its output (two 56-channel halves per token) for block 0's norm1
-  HIERA_TRY(launch_patch_embed(img_nhwc, pk + P.patch_w, pk + P.pos, act[0],
-                               bf ? stp[0] : nullptr, desc->B, desc->img, bf, st));
-  int cur = 0, s_idx = 0, parts = 2;
-  for (int i = 0; i < kDepth; ++i) {
-    Geom g;
-    make_geom(&plan[i].d, &g);
-    const uint8_t* bp = pk + P.blocks[i];
-    uint8_t* out = act[cur ^ 1];
-    HIERA_TRY(g.bf16 ? forward_bf16(g, bp, act[cur], out, ws + W.block, st, stp[cur], parts,
-                                    stp[cur ^ 1])
-                     : forward_f32(g, bp, act[cur], out, ws + W.block, st));
-    parts = store_stats_parts(g.d_out);
-    cur ^= 1;
-    if (s_idx < 4 && i == kStageEnds[s_idx]) {
-      // (a13) Reroll the stage output to NHWC
-      const int s = plan[i].stage;
-      const int Gs = G0 >> s;
-      if (launch_permute(false, act[cur], feats[s_idx], desc->B, Gs, kStageDim[s], 3 - s, es,
-                         st) != cudaSuccess)
-        return HIERA_ERR_CUDA;
-      ++s_idx;
-    }
+  if (!split_applies(desc)) {
+    if (workspace_bytes < backbone_ws_layout(desc, plan).total) return HIERA_ERR_WORKSPACE;
+    HIERA_TRY(check_device());
+    return backbone_run(desc, plan, pk, img_nhwc, feats, ws, st);
   }
-  return HIERA_OK;
+  size_t off2 = 0;
+  if (workspace_bytes < split_ws_bytes(desc, &off2)) return HIERA_ERR_WORKSPACE;
+  HIERA_TRY(check_device());
+  hiera_backbone_desc h1, h2;
+  split_descs(desc, &h1, &h2);
+  BlockPlan p1[kDepth], p2[kDepth];
+  HIERA_TRY(backbone_plan(&h1, p1));
+  HIERA_TRY(backbone_plan(&h2, p2));
+  // the second half's image and feature rows follow the first half's B1 images
+  const size_t es = desc->dtype == HIERA_BF16 ? 2 : 4;
+  const size_t G0 = (size_t)desc->img / 4;
+  const uint8_t* img2 = static_cast<const uint8_t*>(img_nhwc) +
+                        (size_t)h1.B * desc->img * desc->img * 4 * es;
+  void* feats2[4];
+  for (int s = 0; s < 4; ++s) {
+    const size_t Gs = G0 >> s;
+    feats2[s] = static_cast<uint8_t*>(feats[s]) + (size_t)h1.B * Gs * Gs * kStageDim[s] * es;
+  }
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cap) != cudaSuccess) return HIERA_ERR_CUDA;
+  AuxStreams* aux = nullptr;
+  HIERA_TRY(aux_streams(&aux, cap != cudaStreamCaptureStatusNone));
+  if (aux == nullptr) {
+    if (workspace_bytes < backbone_ws_layout(desc, plan).total) return HIERA_ERR_WORKSPACE;
+    return backbone_run(desc, plan, pk, img_nhwc, feats, ws, st);
+  }
+  // fork: the second stream starts after everything the caller's stream holds so far
+  if (cudaEventRecord(aux->fork, st) != cudaSuccess ||
+      cudaStreamWaitEvent(aux->s, aux->fork, 0) != cudaSuccess)
+    return HIERA_ERR_CUDA;
+  const hiera_status r1 = backbone_run(&h1, p1, pk, img_nhwc, feats, ws, st);
+  const hiera_status r2 = backbone_run(&h2, p2, pk, img2, feats2, ws + off2, aux->s);
+  // join (also after a failed launch, so that the streams, or a capture, stay consistent)
+  if (cudaEventRecord(aux->join, aux->s) != cudaSuccess ||
+      cudaStreamWaitEvent(st, aux->join, 0) != cudaSuccess)
+    return HIERA_ERR_CUDA;
+  return r1 != HIERA_OK ? r1 : r2;
 }
 
 hiera_status hiera_profile_begin(void* const* events, int capacity, int* kinds) {

@@ -253,6 +253,9 @@ __global__ void __launch_bounds__(320, 1)
       const int ix0 = 4 * (ox0 + px) - 3;  // first image column of this pixel's window
       uint8_t* arow = smem + PE_OFF_A + b * PE_A_BYTES + px * 128;
       const bf16* ib = p.img + (long long)bi * p.img_side * p.img_side * CIN;
+      // all 49 pixel loads of the window first (one round trip to L2 per tile rather than
+      // one per kernel row), then the 49 shared-memory stores
+      uint2 v[KSZ * KSZ];
 #pragma unroll
       for (int ky = 0; ky < KSZ; ++ky) {
         const int iy = 4 * oy - 3 + ky;
@@ -261,14 +264,17 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
         for (int kx = 0; kx < KSZ; ++kx) {
           const int ix = ix0 + kx;
-          uint2 v = make_uint2(0u, 0u);
+          v[ky * KSZ + kx] = make_uint2(0u, 0u);
           if (row_in && ix >= 0 && ix < p.img_side)
-            v = __ldg(reinterpret_cast<const uint2*>(irow + (long long)ix * CIN));
-          const int k = (ky * KSZ + kx) * CIN;             // compile-time after unrolling
-          const int kb = k >> 6, kc = k & 63;
-          *reinterpret_cast<uint2*>(arow + kb * 16384 + ((((uint32_t)(kc >> 3)) ^ sw) << 4) +
-                                    (kc & 7) * 2) = v;
+            v[ky * KSZ + kx] = __ldg(reinterpret_cast<const uint2*>(irow + (long long)ix * CIN));
         }
+      }
+#pragma unroll
+      for (int i = 0; i < KSZ * KSZ; ++i) {
+        const int k = i * CIN;  // (ky * 7 + kx) * 4, compile-time after unrolling
+        const int kb = k >> 6, kc = k & 63;
+        *reinterpret_cast<uint2*>(arow + kb * 16384 + ((((uint32_t)(kc >> 3)) ^ sw) << 4) +
+                                  (kc & 7) * 2) = v[i];
       }
       fence_proxy_async_smem();  // generic-proxy writes before the tensor core reads them
       mbar_arrive(&a_full[b]);

@@ -125,13 +125,17 @@ def test_binding_rejects_mismatched_tensors_before_any_launch():
 
 
 def test_option_defaults_and_range():
-    """Library options are host state: fused MLP, programmatic launch and the fused attention
-    half default on, the 224-column GEMMs on the eight-warp kernel; unknown options and
-    values are rejected."""
+    """Library options are host state: fused MLP, programmatic launch, the fused attention
+    half and the split batch default on, the 224-column GEMMs on the eight-warp kernel;
+    unknown options and values are rejected."""
     assert [hb.get_option(o) for o in (hb.OPT_FUSED_MLP, hb.OPT_PDL, hb.OPT_FUSED_ATTN,
-                                       hb.OPT_GEMM224)] == [1, 1, 1, 0]
+                                       hb.OPT_GEMM224, hb.OPT_SPLIT_BATCH)] == [1, 1, 1, 0, 1]
     L = hb.lib()
-    assert L.hiera_set_option(4, 1) == 1
+    assert L.hiera_set_option(5, 1) == 1
+    assert L.hiera_set_option(hb.OPT_SPLIT_BATCH, 2) == 1
+    with hb.split_batch(False):
+        assert hb.get_option(hb.OPT_SPLIT_BATCH) == 0
+    assert hb.get_option(hb.OPT_SPLIT_BATCH) == 1
     assert L.hiera_set_option(hb.OPT_GEMM224, 3) == 1
     assert L.hiera_set_option(hb.OPT_PDL, 2) == 1
     for mode in (hb.GEMM224_SIXTEEN_WARPS, hb.GEMM224_PAIR):

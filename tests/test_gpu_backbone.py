@@ -147,6 +147,36 @@ def test_transition_block_65536_tokens_sampled_rows():
     assert rel_l2(got, ref) <= 1e-2
 
 
+@pytest.mark.parametrize("img,B,dtype", [(64, 3, "bf16"), (128, 8, "bf16"), (64, 2, "f32")])
+def test_split_batch_matches_one_batch_bitwise(img, B, dtype):
+    """A call run as two concurrent half batches on two streams (the default for B >= 2;
+    an odd B splits as ceil(B/2) + floor(B/2)) gives the same bits as the call run as one
+    batch, eagerly and replayed from a CUDA graph captured on the caller's stream."""
+    p = syn.backbone_params(41, img, dtype=dtype, affine="random")
+    x = dev(syn.image(41, B, img, dtype=dtype), dtype)
+    desc = hb.BackboneDesc(B=B, img=img, dtype=TORCH_DT[dtype])
+    packed = hb.backbone_pack(desc, weights_dev(p, dtype))
+    with hb.split_batch(False):
+        one = hb.backbone_forward(desc, packed, x)
+    assert hb.get_option(hb.OPT_SPLIT_BATCH) == 1
+    two = hb.backbone_forward(desc, packed, x)
+    torch.cuda.synchronize()
+    for s, (a, b) in enumerate(zip(one, two)):
+        assert torch.equal(a, b), (s, (a.float() - b.float()).abs().max().item())
+    # graph capture of the split call: the second stream joins the capture
+    ws = torch.empty(hb.backbone_workspace_bytes(desc), dtype=torch.uint8, device="cuda")
+    feats = [torch.full(f.shape, float("nan"), dtype=f.dtype, device="cuda") for f in one]
+    stream = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        hb.backbone_forward(desc, packed, x, feats=feats, workspace=ws)
+    g.replay()
+    torch.cuda.synchronize()
+    assert hb.device_status() == 0
+    for s, (a, b) in enumerate(zip(one, feats)):
+        assert torch.equal(a, b), s
+
+
 @pytest.mark.parametrize("graph", [True, False])
 def test_backbone_pipeline_host_to_host_bitwise(graph):
     """binding.BackbonePipeline (uploads, forward and downloads of consecutive batches
