@@ -282,8 +282,10 @@ HIERA_API hiera_status hiera_patch_embed(const void* img, const void* packed_pat
  * rest on a second stream owned by the calling thread (one per device), forked from and
  * joined back into `stream` with events: the call stays ordered with the caller's work on
  * `stream` and may be captured into a CUDA graph from it (the second stream joins the
- * capture). A call is not to be made while a capture begun by the same thread on another
- * stream is still open.
+ * capture). The second stream is created by the thread's first hiera_backbone_pack (or,
+ * failing that, its first split call outside a capture; a call made inside a capture
+ * before the thread has one runs as one batch). A call is not to be made while a capture
+ * begun by the same thread on another stream is still open.
  * -------------------------------------------------------------------------------- */
 typedef struct {
   int B;
