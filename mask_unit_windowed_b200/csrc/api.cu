@@ -677,9 +677,16 @@ hiera_status static_scratch_address(void** out) {
   return HIERA_OK;
 }
 
+// The tensor-core path's GELU as its epilogues evaluate it: on pairs with the packed fp32
+// instructions (an odd n's last value alone, through the scalar form, which gives the same
+// bits).
 __global__ void gelu_probe_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) y[i] = gelu_fast(x[i]);
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    f2_unpack(gelu_fast2(f2_pack(x[i], x[i + 1])), y[i], y[i + 1]);
+  } else if (i < n) {
+    y[i] = gelu_fast(x[i]);
+  }
 }
 
 __global__ void timeout_probe_kernel(uint64_t limit_ns, unsigned int* status) {
@@ -1136,7 +1143,7 @@ hiera_status hiera_debug_gelu(const float* x, float* y, int n, hiera_stream_t st
   if (x == nullptr || y == nullptr || n < 1) return HIERA_ERR_INVALID_ARG;
   HIERA_TRY(check_device());
   profile_mark(K_PROBE, (cudaStream_t)stream);
-  gelu_probe_kernel<<<(n + 255) / 256, 256, 0, (cudaStream_t)stream>>>(x, y, n);
+  gelu_probe_kernel<<<((n + 1) / 2 + 255) / 256, 256, 0, (cudaStream_t)stream>>>(x, y, n);
   return cudaGetLastError() == cudaSuccess ? HIERA_OK : HIERA_ERR_CUDA;
 }
 

@@ -356,6 +356,49 @@ __device__ __forceinline__ float gelu_fast(float x) {
   return fmaf(h, t, h);
 }
 
+// Two fp32 values in one 64-bit register pair for sm_100's packed fp32 instructions
+// (fma.rn.f32x2, mul.rn.f32x2): each half is the IEEE operation on its own value, the same
+// bits as the scalar instruction, in half the issue slots. The epilogues whose arithmetic is
+// bound by instruction issue (the GELU of fc1 and of the fused MLP) work on pairs.
+typedef unsigned long long f32x2;
+__device__ __forceinline__ f32x2 f2_pack(float lo, float hi) {
+  f32x2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(f32x2 v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ f32x2 f2_fma(f32x2 a, f32x2 b, f32x2 c) {
+  f32x2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ f32x2 f2_mul(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// gelu_fast of two values with the packed instructions: the same operations in the same
+// order on each value, so the same bits as two gelu_fast calls.
+__device__ __forceinline__ f32x2 gelu_fast2(f32x2 x) {
+  const f32x2 sq = f2_mul(x, x);
+  float s0, s1;
+  f2_unpack(sq, s0, s1);
+  const f32x2 x2 = f2_pack(fminf(s0, 36.0f), fminf(s1, 36.0f));
+  f32x2 p = f2_fma(f2_pack(-3.51580345e-04f, -3.51580345e-04f), x2,
+                   f2_pack(3.70059155e-02f, 3.70059155e-02f));
+  p = f2_fma(p, x2, f2_pack(7.97507650e-01f, 7.97507650e-01f));
+  float u0, u1;
+  f2_unpack(f2_mul(x, p), u0, u1);
+  float t0, t1;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t0) : "f"(u0));
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t1) : "f"(u1));
+  const f32x2 h = f2_mul(f2_pack(0.5f, 0.5f), x);
+  return f2_fma(h, f2_pack(t0, t1), h);
+}
+
 // ------------------------------------------------------------------ tcgen05 epilogue helpers
 // Every lane observes the barrier phase itself (so each has acquired the producer's
 // writes), then the warp agrees on the outcome so that it stays converged for the

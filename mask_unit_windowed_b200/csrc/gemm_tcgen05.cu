@@ -383,13 +383,24 @@ __global__ void __launch_bounds__(320, 1)
             sc[2] = s4.z;
             sc[3] = s4.w;
           }
+          if constexpr (EPI == EPI_GELU) {
+            // fold and GELU on pairs (packed fp32: the scalar path's bits, half the issues)
+            const f32x2 fa2 = f2_pack(fa, fa), fb2 = f2_pack(fb, fb);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int i = 4 * g + e;
-            float x = FOLD ? fmaf(fa, __uint_as_float(r[i]), fmaf(fb, sc[e], kc[e]))
-                           : __uint_as_float(r[i]) + kc[e];
-            if (EPI == EPI_GELU) x = gelu_fast(x);
-            v[i] = x;
+            for (int e = 0; e < 4; e += 2) {
+              const int i = 4 * g + e;
+              const f32x2 x = f2_fma(fa2, f2_pack(__uint_as_float(r[i]), __uint_as_float(r[i + 1])),
+                                     f2_fma(fb2, f2_pack(sc[e], sc[e + 1]),
+                                            f2_pack(kc[e], kc[e + 1])));
+              f2_unpack(gelu_fast2(x), v[i], v[i + 1]);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int i = 4 * g + e;
+              v[i] = FOLD ? fmaf(fa, __uint_as_float(r[i]), fmaf(fb, sc[e], kc[e]))
+                          : __uint_as_float(r[i]) + kc[e];
+            }
           }
         }
         // ---- finish the values of this chunk (residual; the q / residual pooling of a

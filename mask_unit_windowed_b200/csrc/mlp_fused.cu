@@ -449,9 +449,14 @@ __global__ void __launch_bounds__(THREADS, 1)
             const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
             const float kv[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
             float v[8];
+            const f32x2 fa2 = f2_pack(fa, fa), fb2 = f2_pack(fb, fb);
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-              v[e] = gelu_fast(fmaf(fa, __uint_as_float(r[8 * g + e]), fmaf(fb, sv[e], kv[e])));
+            for (int e = 0; e < 8; e += 2) {  // fold + GELU on pairs (packed fp32)
+              const f32x2 x = f2_fma(fa2, f2_pack(__uint_as_float(r[8 * g + e]),
+                                                  __uint_as_float(r[8 * g + e + 1])),
+                                     f2_fma(fb2, f2_pack(sv[e], sv[e + 1]), f2_pack(kv[e], kv[e + 1])));
+              f2_unpack(gelu_fast2(x), v[e], v[e + 1]);
+            }
             pk[g] = pack8(v);
           }
           const int hb = (int)(hc % C::NH);
@@ -600,9 +605,14 @@ __global__ void __launch_bounds__(THREADS, 1)
           const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
           const float kv[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
           float v[8];
+          const f32x2 fa2 = f2_pack(fa, fa), fb2 = f2_pack(fb, fb);
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            v[e] = gelu_fast(fmaf(fa, __uint_as_float(r[8 * g + e]), fmaf(fb, sv[e], kv[e])));
+          for (int e = 0; e < 8; e += 2) {  // fold + GELU on pairs (packed fp32)
+            const f32x2 x = f2_fma(fa2, f2_pack(__uint_as_float(r[8 * g + e]),
+                                                __uint_as_float(r[8 * g + e + 1])),
+                                   f2_fma(fb2, f2_pack(sv[e], sv[e + 1]), f2_pack(kv[e], kv[e + 1])));
+            f2_unpack(gelu_fast2(x), v[e], v[e + 1]);
+          }
           pk[g] = pack8(v);
         }
         const int hb = (int)(hc % C::NH);
