@@ -306,8 +306,13 @@ __global__ void __launch_bounds__(320, 1)
             const float sc[4] = {s4.x, s4.y, s4.z, s4.w};
             const float kc[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              v[4 * h2 + e] = fmaf(fa, __uint_as_float(rr[8 * c8 + 4 * h2 + e]), fmaf(fb, sc[e], kc[e]));
+            for (int e = 0; e < 4; e += 2)  // the fold on pairs (packed fp32, the scalar bits)
+              f2_unpack(f2_fma(f2_pack(fa, fa),
+                               f2_pack(__uint_as_float(rr[8 * c8 + 4 * h2 + e]),
+                                       __uint_as_float(rr[8 * c8 + 4 * h2 + e + 1])),
+                               f2_fma(f2_pack(fb, fb), f2_pack(sc[e], sc[e + 1]),
+                                      f2_pack(kc[e], kc[e + 1]))),
+                        v[4 * h2 + e], v[4 * h2 + e + 1]);
           }
           *reinterpret_cast<uint4*>(row + (((uint32_t)c8 ^ (uint32_t)(r & 7)) << 4)) = pack8(v);
         }
@@ -344,9 +349,13 @@ __global__ void __launch_bounds__(320, 1)
         for (int hh = 0; hh < 2; ++hh) {
           uint32_t pw[32];
 #pragma unroll
-          for (int u = 0; u < 32; ++u) {
-            const float e = ex2_approx(fmaf(own[32 * hh + u], sl2, -ms));
-            pw[u] = par ? pack_trunc2(0.f, e) : pack_trunc2(e, 0.f);
+          for (int u = 0; u < 32; u += 2) {
+            float x0, x1;  // two keys' exponents in one packed FMA
+            f2_unpack(f2_fma(f2_pack(own[32 * hh + u], own[32 * hh + u + 1]), f2_pack(sl2, sl2),
+                             f2_pack(-ms, -ms)), x0, x1);
+            const float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
+            pw[u] = par ? pack_trunc2(0.f, e0) : pack_trunc2(e0, 0.f);
+            pw[u + 1] = par ? pack_trunc2(0.f, e1) : pack_trunc2(e1, 0.f);
           }
           tc_st_32x32b_x32(sc + (uint32_t)(32 * hh), pw);
         }
@@ -374,7 +383,9 @@ __global__ void __launch_bounds__(320, 1)
         for (int c8 = 0; c8 < 7; ++c8) {
           float f[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(ov[8 * c8 + e]) * inv;
+          for (int e = 0; e < 8; e += 2)
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(ov[8 * c8 + e]), __uint_as_float(ov[8 * c8 + e + 1])),
+                             f2_pack(inv, inv)), f[e], f[e + 1]);
           const int ch = 7 * hs + c8;  // 16-byte chunk of the 112-channel row
           *reinterpret_cast<uint4*>(om + (ch >> 3) * 16384 + r * 128 +
                                     ((((uint32_t)ch & 7u) ^ (uint32_t)(r & 7)) << 4)) = pack8(f);
@@ -395,24 +406,23 @@ __global__ void __launch_bounds__(320, 1)
         // the proj bias of this column half, four per 16-byte shared-memory load (every lane
         // reads the same address: one broadcast per load; 56 hs floats is 16-byte aligned)
         const float4* bo4 = reinterpret_cast<const float4*>(c_bo + 56 * hs);
+        // (proj + bias) + residual on pairs (packed fp32, the scalar bits)
 #pragma unroll
         for (int g = 0; g < 14; ++g) {
           const float4 b4 = bo4[g];
-          v[4 * g + 0] = __uint_as_float(rr[4 * g + 0]) + b4.x;
-          v[4 * g + 1] = __uint_as_float(rr[4 * g + 1]) + b4.y;
-          v[4 * g + 2] = __uint_as_float(rr[4 * g + 2]) + b4.z;
-          v[4 * g + 3] = __uint_as_float(rr[4 * g + 3]) + b4.w;
+          f2_unpack(f2_add(f2_pack(__uint_as_float(rr[4 * g + 0]), __uint_as_float(rr[4 * g + 1])),
+                           f2_pack(b4.x, b4.y)), v[4 * g + 0], v[4 * g + 1]);
+          f2_unpack(f2_add(f2_pack(__uint_as_float(rr[4 * g + 2]), __uint_as_float(rr[4 * g + 3])),
+                           f2_pack(b4.z, b4.w)), v[4 * g + 2], v[4 * g + 3]);
         }
 #pragma unroll
         for (int g = 0; g < 7; ++g) {
-          v[8 * g + 0] += bf16_lo(res[g].x);
-          v[8 * g + 1] += bf16_hi(res[g].x);
-          v[8 * g + 2] += bf16_lo(res[g].y);
-          v[8 * g + 3] += bf16_hi(res[g].y);
-          v[8 * g + 4] += bf16_lo(res[g].z);
-          v[8 * g + 5] += bf16_hi(res[g].z);
-          v[8 * g + 6] += bf16_lo(res[g].w);
-          v[8 * g + 7] += bf16_hi(res[g].w);
+          const uint32_t rw[4] = {res[g].x, res[g].y, res[g].z, res[g].w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            f2_unpack(f2_add(f2_pack(v[8 * g + 2 * q], v[8 * g + 2 * q + 1]),
+                             f2_pack(bf16_lo(rw[q]), bf16_hi(rw[q]))),
+                      v[8 * g + 2 * q], v[8 * g + 2 * q + 1]);
         }
         uint4* dst = reinterpret_cast<uint4*>(p.x1 + tok * FD + 56 * hs);
 #pragma unroll

@@ -322,10 +322,13 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t pw[32];
+        const f32x2 sl2x2 = f2_pack(sl2, sl2), nms2 = f2_pack(-ms, -ms);
 #pragma unroll
         for (int u = 0; u < 32; ++u) {
-          const float x0 = fmaf(__uint_as_float(sr[64 * h + 2 * u]), sl2, -ms);   // -inf -> 0
-          const float x1 = fmaf(__uint_as_float(sr[64 * h + 2 * u + 1]), sl2, -ms);
+          // s log2(e)/sqrt(56) - m for a pair of keys in one packed FMA (-inf -> 0 below)
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[64 * h + 2 * u]),
+                                   __uint_as_float(sr[64 * h + 2 * u + 1])), sl2x2, nms2), x0, x1);
           pw[u] = pack_bf16x2_trunc(ex2_approx(x0), ex2_approx(x1));
         }
         tc_st_32x32b_x32(lane_base + s_col + (uint32_t)(32 * h), pw);
@@ -377,14 +380,15 @@ __global__ void __launch_bounds__(320, 1)
         const int bimg = unit / (p.heads * p.nW);
         const long long Nq = (long long)p.Tq * p.nW;
         bf16* dst = p.o + ((long long)bimg * Nq + (long long)qrow * p.nW + w) * p.d_out + h * 56;
+        const f32x2 inv2 = f2_pack(inv, inv);
 #pragma unroll
         for (int c = 0; c < 7; ++c) {
-          uint4 pk;
-          pk.x = pack_bf16x2(__uint_as_float(ov[8 * c + 0]) * inv, __uint_as_float(ov[8 * c + 1]) * inv);
-          pk.y = pack_bf16x2(__uint_as_float(ov[8 * c + 2]) * inv, __uint_as_float(ov[8 * c + 3]) * inv);
-          pk.z = pack_bf16x2(__uint_as_float(ov[8 * c + 4]) * inv, __uint_as_float(ov[8 * c + 5]) * inv);
-          pk.w = pack_bf16x2(__uint_as_float(ov[8 * c + 6]) * inv, __uint_as_float(ov[8 * c + 7]) * inv);
-          *reinterpret_cast<uint4*>(dst + 8 * c) = pk;
+          float f[8];
+#pragma unroll
+          for (int e = 0; e < 8; e += 2)
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(ov[8 * c + e]), __uint_as_float(ov[8 * c + e + 1])),
+                             inv2), f[e], f[e + 1]);
+          *reinterpret_cast<uint4*>(dst + 8 * c) = pack8(f);
         }
       }
     }

@@ -269,9 +269,12 @@ __global__ void __launch_bounds__(320, 1)
         const float ms = m * sl2;
         uint32_t pw[TKV / 2];
 #pragma unroll
-        for (int u = 0; u < TKV / 2; ++u)
-          pw[u] = pack_trunc(ex2_approx(fmaf(mine[2 * u], sl2, -ms)),
-                             ex2_approx(fmaf(mine[2 * u + 1], sl2, -ms)));
+        for (int u = 0; u < TKV / 2; ++u) {
+          float x0, x1;  // a pair of keys in one packed FMA
+          f2_unpack(f2_fma(f2_pack(mine[2 * u], mine[2 * u + 1]), f2_pack(sl2, sl2),
+                           f2_pack(-ms, -ms)), x0, x1);
+          pw[u] = pack_trunc(ex2_approx(x0), ex2_approx(x1));
+        }
         // P into the S columns it came from (the thread has read its scores): this lane's
         // weights in its own unit's columns, zero in every other column of the row
         uint32_t zero[16];
@@ -324,7 +327,9 @@ __global__ void __launch_bounds__(320, 1)
         for (int c = 0; c < 7; ++c) {
           float f[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(ov[8 * c + e]) * inv;
+          for (int e = 0; e < 8; e += 2)
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(ov[8 * c + e]), __uint_as_float(ov[8 * c + e + 1])),
+                             f2_pack(inv, inv)), f[e], f[e + 1]);
           *reinterpret_cast<uint4*>(dst + 8 * c) = pack8(f);
         }
       }

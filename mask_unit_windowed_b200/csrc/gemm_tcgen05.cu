@@ -396,10 +396,14 @@ __global__ void __launch_bounds__(320, 1)
             }
           } else {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
+            for (int e = 0; e < 4; e += 2) {  // (pairs: packed fp32, the scalar bits)
               const int i = 4 * g + e;
-              v[i] = FOLD ? fmaf(fa, __uint_as_float(r[i]), fmaf(fb, sc[e], kc[e]))
-                          : __uint_as_float(r[i]) + kc[e];
+              const f32x2 acc2 = f2_pack(__uint_as_float(r[i]), __uint_as_float(r[i + 1]));
+              const f32x2 kc2 = f2_pack(kc[e], kc[e + 1]);
+              f2_unpack(FOLD ? f2_fma(f2_pack(fa, fa), acc2,
+                                      f2_fma(f2_pack(fb, fb), f2_pack(sc[e], sc[e + 1]), kc2))
+                             : f2_add(acc2, kc2),
+                        v[i], v[i + 1]);
             }
           }
         }
@@ -410,14 +414,12 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
           for (int g = 0; g < CH / 8; ++g) {
             const uint4 rr = res[(c / 8 + g) < NV ? (c / 8 + g) : 0];
-            v[8 * g + 0] += bf16_lo(rr.x);
-            v[8 * g + 1] += bf16_hi(rr.x);
-            v[8 * g + 2] += bf16_lo(rr.y);
-            v[8 * g + 3] += bf16_hi(rr.y);
-            v[8 * g + 4] += bf16_lo(rr.z);
-            v[8 * g + 5] += bf16_hi(rr.z);
-            v[8 * g + 6] += bf16_lo(rr.w);
-            v[8 * g + 7] += bf16_hi(rr.w);
+            const uint32_t rw[4] = {rr.x, rr.y, rr.z, rr.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              f2_unpack(f2_add(f2_pack(v[8 * g + 2 * q], v[8 * g + 2 * q + 1]),
+                               f2_pack(bf16_lo(rw[q]), bf16_hi(rw[q]))),
+                        v[8 * g + 2 * q], v[8 * g + 2 * q + 1]);
           }
         }
         // ---- destination of this lane's row for this chunk
