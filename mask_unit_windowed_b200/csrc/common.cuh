@@ -404,6 +404,52 @@ __device__ __forceinline__ f32x2 gelu_fast2(f32x2 x) {
   return f2_fma(h, f2_pack(t0, t1), h);
 }
 
+// (mean, M2) of the N values of a row piece in column order, as four interleaved partial
+// sums (values i = q mod 4 in accumulator q) combined as (a0 + a1) + (a2 + a3): chains a
+// quarter as long as one running sum. Every kernel that writes LayerNorm partials of such a
+// piece uses this order (stats_piece on fp32 values, stats_piece_bf16 on packed bf16 rows), so
+// the fused and unfused paths produce the same bits.
+template <int N>
+__device__ __forceinline__ void stats_piece(const float (&v)[N], float& mean, float& m2) {
+  static_assert(N % 4 == 0, "four accumulators");
+  float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int i = 0; i < N; ++i) s4[i & 3] += v[i];
+  mean = ((s4[0] + s4[1]) + (s4[2] + s4[3])) * (1.f / (float)N);
+  float q4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int i = 0; i < N; ++i) q4[i & 3] = fmaf(v[i] - mean, v[i] - mean, q4[i & 3]);
+  m2 = (q4[0] + q4[1]) + (q4[2] + q4[3]);
+}
+// the same on NG * 8 values held as packed bf16 (value 8 g + 2 e + h is word e's half h)
+template <int NG>
+__device__ __forceinline__ void stats_piece_bf16(const uint4 (&w)[NG], float& mean, float& m2) {
+  float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int g = 0; g < NG; ++g) {
+    const uint32_t w4[4] = {w[g].x, w[g].y, w[g].z, w[g].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      s4[(2 * e) & 3] += __uint_as_float(w4[e] << 16);
+      s4[(2 * e + 1) & 3] += __uint_as_float(w4[e] & 0xFFFF0000u);
+    }
+  }
+  mean = ((s4[0] + s4[1]) + (s4[2] + s4[3])) * (1.f / (float)(NG * 8));
+  float q4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int g = 0; g < NG; ++g) {
+    const uint32_t w4[4] = {w[g].x, w[g].y, w[g].z, w[g].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float lo = __uint_as_float(w4[e] << 16) - mean;
+      const float hi = __uint_as_float(w4[e] & 0xFFFF0000u) - mean;
+      q4[(2 * e) & 3] = fmaf(lo, lo, q4[(2 * e) & 3]);
+      q4[(2 * e + 1) & 3] = fmaf(hi, hi, q4[(2 * e + 1) & 3]);
+    }
+  }
+  m2 = (q4[0] + q4[1]) + (q4[2] + q4[3]);
+}
+
 // ------------------------------------------------------------------ tcgen05 epilogue helpers
 // Every lane observes the barrier phase itself (so each has acquired the producer's
 // writes), then the warp agrees on the outcome so that it stays converged for the

@@ -481,13 +481,8 @@ __global__ void __launch_bounds__(320, 1)
           *reinterpret_cast<uint4*>(stg + (lane << 7) + ((7 ^ (lane & 7)) << 4)) =
               make_uint4(which == 2 ? 0x3F80u : 0u, 0u, 0u, 0u);
         if (EPI == EPI_STORE && p.stats_out != nullptr && row_ok) {
-          float s = 0.f;
-#pragma unroll
-          for (int i = 0; i < CH; ++i) s += v[i];
-          const float cmean = s * (1.f / (float)CH);
-          float cm2 = 0.f;
-#pragma unroll
-          for (int i = 0; i < CH; ++i) cm2 = fmaf(v[i] - cmean, v[i] - cmean, cm2);
+          float cmean, cm2;
+          stats_piece<CH>(v, cmean, cm2);
           // merge this chunk into the running (count, mean, M2)
           chan_merge(st_mean, st_m2, cmean, cm2, (float)c, (float)CH);
         }

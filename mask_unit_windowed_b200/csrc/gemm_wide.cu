@@ -317,13 +317,8 @@ __device__ __forceinline__ void wide_epilogue(const KParams& p, const CUtensorMa
       // chunks. The second quarter's warp writes buffer tcount % 3 only after this tile's MMA,
       // which waited for this warp's accumulator release of the tile before the one where this
       // warp last read that buffer.
-      float sum = 0.f;
-#pragma unroll
-      for (int i = 0; i < CH; ++i) sum += v[i];
-      const float cmean = sum * (1.f / (float)CH);
-      float cm2 = 0.f;
-#pragma unroll
-      for (int i = 0; i < CH; ++i) cm2 = fmaf(v[i] - cmean, v[i] - cmean, cm2);
+      float cmean, cm2;
+      stats_piece<CH>(v, cmean, cm2);
       const int pr = quarter * 2 + half, buf = tcount % W_XCH_BUFS;
       float2* slot = xch + (buf * 8 + pr) * 32 + lane;
       uint64_t* xb = &bb.xch_full[pr * W_XCH_BUFS + buf];

@@ -515,25 +515,9 @@ __global__ void __launch_bounds__(THREADS, 1)
           out_groups<4, 3>(r, res, b4);
         }
         if (p.stats_out != nullptr && row_ok) {
-          // statistics of the values as stored, in column order
-          float sm = 0.f;
-#pragma unroll
-          for (int g = 0; g < 7; ++g)
-            sm = (((((((sm + bf16_lo(res[g].x)) + bf16_hi(res[g].x)) + bf16_lo(res[g].y)) +
-                     bf16_hi(res[g].y)) + bf16_lo(res[g].z)) + bf16_hi(res[g].z)) +
-                  bf16_lo(res[g].w)) + bf16_hi(res[g].w);
-          const float st_mean = sm * (1.f / 56.f);
-          float st_m2 = 0.f;
-#pragma unroll
-          for (int g = 0; g < 7; ++g) {
-            const uint32_t w4[4] = {res[g].x, res[g].y, res[g].z, res[g].w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float lo = bf16_lo(w4[e]) - st_mean, hi = bf16_hi(w4[e]) - st_mean;
-              st_m2 = fmaf(lo, lo, st_m2);
-              st_m2 = fmaf(hi, hi, st_m2);
-            }
-          }
+          // statistics of the values as stored (the order every partial's producer uses)
+          float st_mean, st_m2;
+          stats_piece_bf16<7>(res, st_mean, st_m2);
           p.stats_out[m * 2 + cg] = make_float2(st_mean, st_m2);
         }
         // staging: 16 rows at a time, then 8 lanes per row, 4 rows per store instruction
@@ -665,24 +649,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             out_groups<4, 3>(r, res, b4);
           }
           if (p.stats_out != nullptr) {
-            // statistics of the values as stored, in column order
-            float s = 0.f;
-#pragma unroll
-            for (int g = 0; g < 7; ++g)
-              s = (((((((s + bf16_lo(res[g].x)) + bf16_hi(res[g].x)) + bf16_lo(res[g].y)) +
-                      bf16_hi(res[g].y)) + bf16_lo(res[g].z)) + bf16_hi(res[g].z)) +
-                   bf16_lo(res[g].w)) + bf16_hi(res[g].w);
-            st_mean = s * (1.f / 56.f);
-#pragma unroll
-            for (int g = 0; g < 7; ++g) {
-              const uint32_t w4[4] = {res[g].x, res[g].y, res[g].z, res[g].w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float lo = bf16_lo(w4[e]) - st_mean, hi = bf16_hi(w4[e]) - st_mean;
-                st_m2 = fmaf(lo, lo, st_m2);
-                st_m2 = fmaf(hi, hi, st_m2);
-              }
-            }
+            // statistics of the values as stored (the order every partial's producer uses)
+            stats_piece_bf16<7>(res, st_mean, st_m2);
           }
           // staging (2 KB per warp, aliasing the idle hidden buffers): 16 rows at a time,
           // then 8 lanes per row, 4 rows per store instruction
